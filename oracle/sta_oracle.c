@@ -1,0 +1,280 @@
+/*
+ * sta_oracle.c -- plain fp64 CPU reference for Sliding Tile Attention (STA).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
+ * call this file; only tests/, the smoke check and the bench's CPU-baseline leg
+ * use it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (sources: "Fast Video Generation with Sliding Tile
+ * Attention"; the podcast transcript at hotaipapers.com, segment on tiles and
+ * on dense / empty / mixed blocks; the atlas.scime.ai summary, "Approach";
+ * the dianyo.github.io ICML-2025 post, STA section "Observation & Proposed
+ * Method"):
+ *
+ *   - The video latent is L_t x L_h x L_w tokens in raster order (t, h, w; w
+ *     fastest).  It is cut into tiles: contiguous spatio-temporal cubes of
+ *     T_t x T_h x T_w tokens.
+ *   - Every query tile attends to the key tiles inside a 3D window of tiles
+ *     centred on it; the window slides tile by tile, so all queries of one
+ *     tile share one key set and every (query tile, key tile) block is either
+ *     fully attended or fully skipped.
+ *   - The window size is given per head, in tokens.
+ *   - Attention inside the attended set is exact softmax attention.
+ *
+ * Readings of points the pages leave open (each one is listed in the design
+ * notes with its justification):
+ *   - window extent in tiles e_d = min(W_d / T_d, n_d) (a window larger than
+ *     the volume covers the volume);
+ *   - the window is shifted to stay inside the volume: start
+ *     s_d = clamp(q_d - floor(e_d / 2), 0, n_d - e_d), so an even window puts
+ *     its extra tile on the lower side;
+ *   - LSE is the natural log of sum_j exp(scale * q . k_j) over attended keys;
+ *   - scale is applied as the double value of the fp32 softmax scale;
+ *   - inputs are bf16 values, widened exactly to double.
+ *
+ * The oracle never builds a tile list and never permutes tokens: it evaluates
+ * the token-level mask straight from token coordinates, in raster order.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int32_t lat[3];  /* L_t, L_h, L_w in tokens */
+    int32_t tile[3]; /* T_t, T_h, T_w in tokens */
+} ora_geom;
+
+/* Status codes of this file (not the library's). */
+#define ORA_OK 0
+#define ORA_BAD_ARG 1
+#define ORA_NO_MEM 2
+
+static double bf16_bits_to_double(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static int geom_ok(const ora_geom* g)
+{
+    for (int d = 0; d < 3; ++d) {
+        if (g->lat[d] <= 0 || g->tile[d] <= 0) return 0;
+        if (g->lat[d] % g->tile[d] != 0) return 0;
+    }
+    return 1;
+}
+
+static int window_ok(const ora_geom* g, const int32_t* win)
+{
+    for (int d = 0; d < 3; ++d) {
+        if (win[d] <= 0 || win[d] % g->tile[d] != 0) return 0;
+    }
+    return 1;
+}
+
+int64_t ora_num_tokens(const ora_geom* g)
+{
+    return (int64_t)g->lat[0] * g->lat[1] * g->lat[2];
+}
+
+static void unravel(const ora_geom* g, int64_t token, int32_t c[3])
+{
+    c[2] = (int32_t)(token % g->lat[2]);
+    token /= g->lat[2];
+    c[1] = (int32_t)(token % g->lat[1]);
+    c[0] = (int32_t)(token / g->lat[1]);
+}
+
+/* Window start (in tiles) along one axis: centred on query tile q, extent e
+ * tiles, shifted to stay inside [0, n). */
+static int32_t window_start(int32_t q, int32_t e, int32_t n)
+{
+    int32_t s = q - e / 2;
+    if (s < 0) s = 0;
+    if (s > n - e) s = n - e;
+    return s;
+}
+
+/* Token-level STA mask: may query token qi attend to key token kj under the
+ * window `win` (tokens per axis)?  Returns 1 or 0; -1 on bad arguments. */
+static int key_allowed(const ora_geom* g, const int32_t* win, int64_t qi, int64_t kj)
+{
+    int32_t qc[3], kc[3];
+    unravel(g, qi, qc);
+    unravel(g, kj, kc);
+    for (int d = 0; d < 3; ++d) {
+        int32_t n = g->lat[d] / g->tile[d];
+        int32_t e = win[d] / g->tile[d];
+        if (e > n) e = n;
+        int32_t s = window_start(qc[d] / g->tile[d], e, n);
+        int32_t k_tile = kc[d] / g->tile[d];
+        if (k_tile < s || k_tile >= s + e) return 0;
+    }
+    return 1;
+}
+
+int ora_key_allowed(const ora_geom* g, const int32_t* win, int64_t qi, int64_t kj)
+{
+    if (!geom_ok(g) || !window_ok(g, win)) return -1;
+    int64_t n_tok = ora_num_tokens(g);
+    if (qi < 0 || qi >= n_tok || kj < 0 || kj >= n_tok) return -1;
+    return key_allowed(g, win, qi, kj);
+}
+
+/* Whole mask row of query token qi: out[j] = allowed(qi, j), j in [0, N). */
+int ora_mask_row(const ora_geom* g, const int32_t* win, int64_t qi, uint8_t* out)
+{
+    if (!geom_ok(g) || !window_ok(g, win) || out == NULL) return ORA_BAD_ARG;
+    int64_t n_tok = ora_num_tokens(g);
+    if (qi < 0 || qi >= n_tok) return ORA_BAD_ARG;
+    for (int64_t j = 0; j < n_tok; ++j) out[j] = (uint8_t)key_allowed(g, win, qi, j);
+    return ORA_OK;
+}
+
+/* Position of raster token `token` in tile-major order: tiles in raster order
+ * over the tile grid, tokens inside a tile in raster order over the tile's own
+ * (t, h, w) offsets.  The pages only say a tile is a contiguous cube of tokens;
+ * this fixed order is the reading every layout test uses. */
+int64_t ora_tile_major_index(const ora_geom* g, int64_t token)
+{
+    if (!geom_ok(g)) return -1;
+    if (token < 0 || token >= ora_num_tokens(g)) return -1;
+    int32_t c[3];
+    unravel(g, token, c);
+    int64_t n_h = g->lat[1] / g->tile[1];
+    int64_t n_w = g->lat[2] / g->tile[2];
+    int64_t tile_id = ((int64_t)(c[0] / g->tile[0]) * n_h + c[1] / g->tile[1]) * n_w + c[2] / g->tile[2];
+    int64_t local = ((int64_t)(c[0] % g->tile[0]) * g->tile[1] + c[1] % g->tile[1]) * g->tile[2] + c[2] % g->tile[2];
+    return tile_id * ((int64_t)g->tile[0] * g->tile[1] * g->tile[2]) + local;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention                                                                  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *k, *v; /* [B, H, N, d] raster order, bf16 bits */
+    const ora_geom* g;
+    int64_t heads;
+    int32_t d;
+    const int32_t* win; /* [H][3] tokens */
+    double scale;
+    const int64_t* rows; /* nrows pairs (bh, token) */
+    int64_t nrows;
+    double *out_o, *out_lse;
+    int64_t next; /* shared row counter */
+    pthread_mutex_t lock;
+    int status;
+} ora_job;
+
+static int64_t job_take(ora_job* job)
+{
+    pthread_mutex_lock(&job->lock);
+    int64_t r = job->next++;
+    pthread_mutex_unlock(&job->lock);
+    return r;
+}
+
+static void* attention_worker(void* arg)
+{
+    ora_job* job = (ora_job*)arg;
+    const int64_t n_tok = ora_num_tokens(job->g);
+    const int32_t d = job->d;
+    double* score = (double*)malloc(sizeof(double) * (size_t)n_tok);
+    uint8_t* allowed = (uint8_t*)malloc((size_t)n_tok);
+    double* qrow = (double*)malloc(sizeof(double) * (size_t)d);
+    double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!score || !allowed || !qrow || !acc) {
+        pthread_mutex_lock(&job->lock);
+        job->status = ORA_NO_MEM;
+        pthread_mutex_unlock(&job->lock);
+        free(score); free(allowed); free(qrow); free(acc);
+        return NULL;
+    }
+    for (;;) {
+        int64_t r = job_take(job);
+        if (r >= job->nrows) break;
+        int64_t bh = job->rows[2 * r];
+        int64_t qi = job->rows[2 * r + 1];
+        int64_t h = bh % job->heads;
+        const int32_t* win = job->win + 3 * h;
+        const uint16_t* qp = job->q + (bh * n_tok + qi) * d;
+        const uint16_t* kbase = job->k + bh * n_tok * d;
+        const uint16_t* vbase = job->v + bh * n_tok * d;
+        for (int32_t c = 0; c < d; ++c) qrow[c] = bf16_bits_to_double(qp[c]);
+
+        /* 1. token-level mask and scores s_j = scale * q . k_j */
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n_tok; ++j) {
+            allowed[j] = (uint8_t)key_allowed(job->g, win, qi, j);
+            if (!allowed[j]) continue;
+            const uint16_t* kp = kbase + j * d;
+            double dot = 0.0;
+            for (int32_t c = 0; c < d; ++c) dot += qrow[c] * bf16_bits_to_double(kp[c]);
+            score[j] = job->scale * dot;
+            if (score[j] > m) m = score[j];
+        }
+        /* 2. softmax: l = sum exp(s_j - m); O = sum exp(s_j - m) v_j / l */
+        double l = 0.0;
+        for (int32_t c = 0; c < d; ++c) acc[c] = 0.0;
+        for (int64_t j = 0; j < n_tok; ++j) {
+            if (!allowed[j]) continue;
+            double w = exp(score[j] - m);
+            l += w;
+            const uint16_t* vp = vbase + j * d;
+            for (int32_t c = 0; c < d; ++c) acc[c] += w * bf16_bits_to_double(vp[c]);
+        }
+        for (int32_t c = 0; c < d; ++c) job->out_o[r * d + c] = acc[c] / l;
+        /* 3. LSE = m + ln l (natural log, scaled-score units) */
+        job->out_lse[r] = m + log(l);
+    }
+    free(score); free(allowed); free(qrow); free(acc);
+    return NULL;
+}
+
+/* STA attention for an explicit list of query rows.
+ *   q, k, v     : bf16 bits, [batch, heads, N, d], raster token order
+ *   win         : [heads][3] window in tokens, multiples of the tile
+ *   softmax_scale: fp32 scale; used as (double)softmax_scale
+ *   rows        : nrows pairs (bh = b * heads + h, raster query token)
+ *   out_o       : nrows * d doubles; out_lse: nrows doubles
+ *   nthreads    : worker threads (>= 1)
+ * Returns ORA_OK, ORA_BAD_ARG or ORA_NO_MEM. */
+int ora_sta_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                      const ora_geom* g, int64_t batch, int64_t heads, int32_t d,
+                      const int32_t* win, float softmax_scale,
+                      const int64_t* rows, int64_t nrows,
+                      double* out_o, double* out_lse, int32_t nthreads)
+{
+    if (!q || !k || !v || !g || !win || !rows || !out_o || !out_lse) return ORA_BAD_ARG;
+    if (batch <= 0 || heads <= 0 || d <= 0 || nrows < 0 || nthreads <= 0) return ORA_BAD_ARG;
+    if (!geom_ok(g)) return ORA_BAD_ARG;
+    for (int64_t h = 0; h < heads; ++h)
+        if (!window_ok(g, win + 3 * h)) return ORA_BAD_ARG;
+    int64_t n_tok = ora_num_tokens(g);
+    for (int64_t r = 0; r < nrows; ++r) {
+        if (rows[2 * r] < 0 || rows[2 * r] >= batch * heads) return ORA_BAD_ARG;
+        if (rows[2 * r + 1] < 0 || rows[2 * r + 1] >= n_tok) return ORA_BAD_ARG;
+    }
+    ora_job job;
+    job.q = q; job.k = k; job.v = v; job.g = g; job.heads = heads; job.d = d;
+    job.win = win; job.scale = (double)softmax_scale; job.rows = rows; job.nrows = nrows;
+    job.out_o = out_o; job.out_lse = out_lse; job.next = 0; job.status = ORA_OK;
+    pthread_mutex_init(&job.lock, NULL);
+    pthread_t* tid = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!tid) { pthread_mutex_destroy(&job.lock); return ORA_NO_MEM; }
+    int started = 0;
+    for (int32_t t = 0; t < nthreads; ++t) {
+        if (pthread_create(&tid[t], NULL, attention_worker, &job) != 0) break;
+        ++started;
+    }
+    if (started == 0) attention_worker(&job);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    free(tid);
+    pthread_mutex_destroy(&job.lock);
+    return job.status;
+}
