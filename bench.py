@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the STA forward hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+    raster Q, K, V  --sta_tile_reorder x3-->  tile-major
+    sta_forward (plan built once per geometry / window set, outside the step)
+    tile-major O, LSE  --sta_tile_unreorder x2-->  raster
+on the 720p 5 s HunyuanVideo-shaped workload (B=1, 24 heads, d=128, latent
+30x48x80, tile 6x8x8, window 18x24x24).  Inputs (3 x 707.8 MB) are larger than
+L2, so no flush is needed between steps.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sta|reference]
+Under torchrun each rank runs its own batch (weak scaling, no collective on the
+data path); the timed region is bracketed by a barrier and device syncs and the
+max over ranks is reported.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import sta_inputs  # noqa: E402
+
+METRIC = "STA fwd effective TFLOP/s & tensor-pipe % of peak; speedup vs full window"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FWD_SOURCES = ["sparse_attention_video_sta_b200/csrc/sta_forward.cu",
+               "sparse_attention_video_sta_b200/csrc/sta_ptx.cuh",
+               "sparse_attention_video_sta_b200/csrc/sta_internal.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sta_fwd_720p_traffic.json")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="sta", choices=["sta", "reference"])
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip e2e, full-window, permutation and CPU-baseline legs")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def sources_hash():
+    h = hashlib.sha256()
+    for rel in FWD_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic():
+    """DRAM bytes per forward launch from the committed ncu summary, or None
+    when the kernel sources changed since the counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("sources_hash") == sources_hash():
+            return float(t["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        os.unlink(self.file.name)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_baseline(w, n_tiles: int, heads):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    q, k, v = sta_inputs.make_qkv(w, heads=heads)
+    wins = sta_inputs.windows(w).tolist()
+    n_grid = [w.latent[i] // w.tile[i] for i in range(3)]
+    centre = ((n_grid[0] // 2) * n_grid[1] + n_grid[1] // 2) * n_grid[2] + n_grid[2] // 2
+    tiles = [centre + i for i in range(n_tiles)]
+    toks = np.concatenate([oracle.tile_tokens(w.latent, w.tile, t) for t in tiles])
+    rows = np.array([(h, t) for h in heads for t in toks], dtype=np.int64)
+    flops = 0.0
+    for h, t in rows:
+        e = [min(wins[h % w.heads][i] // w.tile[i], n_grid[i]) for i in range(3)]
+        flops += 4.0 * e[0] * e[1] * e[2] * (w.tile[0] * w.tile[1] * w.tile[2]) * w.head_dim
+    cores = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.sta_attention(q, k, v, w.latent, w.tile, wins, w.softmax_scale, rows=rows, nthreads=cores)
+    dt = time.perf_counter() - t0
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{len(rows)} query rows ({n_tiles} centre tiles x {len(heads)} heads) of "
+                      f"{w.name}; FLOPs counted over attended keys as on the GPU"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    heads = [0]
+    q, k, v = sta_inputs.make_qkv(w, heads=heads)
+    wins = sta_inputs.windows(w).tolist()
+    n_grid = [w.latent[i] // w.tile[i] for i in range(3)]
+    n_tiles = n_grid[0] * n_grid[1] * n_grid[2]
+    vol = w.tile[0] * w.tile[1] * w.tile[2]
+    rows_per_step = 128
+    cores = os.cpu_count() or 1
+
+    def step(i):
+        tile = (i * 37) % n_tiles
+        toks = oracle.tile_tokens(w.latent, w.tile, tile)[:rows_per_step]
+        rows = np.array([(0, t) for t in toks], dtype=np.int64)
+        oracle.sta_attention(q, k, v, w.latent, w.tile, wins, w.softmax_scale, rows=rows, nthreads=cores)
+        e = [min(wins[0][j] // w.tile[j], n_grid[j]) for j in range(3)]
+        return len(rows) * 4.0 * e[0] * e[1] * e[2] * vol * w.head_dim
+
+    for i in range(args.warmup):
+        step(i)
+    flops = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        flops += step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"{rows_per_step} query rows of one tile of head 0 per step, {w.name}"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+                       "latent": list(w.latent), "tile": list(w.tile)},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    w = sta_inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import sparse_attention_video_sta_b200 as sta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------------------------------------------------------- inputs
+    B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
+    shape = (B, H, N, d)
+    gen = torch.Generator(device=dev).manual_seed(w.seed * 1000 + rank)
+    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
+    f = sta_inputs.head_factors(w)
+    for t in (q, k, v):
+        for b in range(B):
+            for h in range(H):
+                x = torch.randn((N, d), generator=gen, device=dev, dtype=torch.float32)
+                if f is not None:
+                    x.mul_(float(f[h]))
+                t[b, h].copy_(x)
+    wins = sta_inputs.windows(w).tolist()
+    plan = sta.sta_plan(w.latent, w.tile, B, H, wins)
+    flops = plan.flops(d)
+    qt, kt, vt, ot = (torch.empty_like(q) for _ in range(4))
+    lset = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty_like(lset)
+    scale = w.softmax_scale
+    L, T = w.latent, w.tile
+    ev_fwd = []
+
+    def step(record=False):
+        sta.sta_tile_reorder(q, qt, L, T)
+        sta.sta_tile_reorder(k, kt, L, T)
+        sta.sta_tile_reorder(v, vt, L, T)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+        sta.sta_forward(plan, qt, kt, vt, ot, lset, scale)
+        if record:
+            e1.record()
+            ev_fwd.append((e0, e1))
+        sta.sta_tile_unreorder(ot, o, L, T)
+        sta.sta_tile_unreorder(lset, lse, L, T, token_dim=2)
+
+    launches_per_step = 6
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    status = sta.sta_last_device_status(plan)
+    if status != 0:
+        raise RuntimeError(f"device status {sta.sta_status_string(status)} after warm-up")
+
+    sampler = ClockSampler(dev.index) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(args.steps):
+        step(record=True)
+    stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_local = start.elapsed_time(stop) / args.steps
+    fwd_ms_local = statistics.mean(a.elapsed_time(b) for a, b in ev_fwd)
+    ms = max_over_ranks(ms_local)
+    fwd_ms = max_over_ranks(fwd_ms_local)
+    status = sta.sta_last_device_status(plan)
+    if status != 0:
+        raise RuntimeError(f"device status {sta.sta_status_string(status)} after timing")
+
+    value = world * flops / (ms * 1e-3) / 1e12
+    fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+
+    extras = {}
+    e2e = None
+    if not args.no_extras:
+        # ------------------------------------------- full-window denominator
+        full = sta.sta_plan(L, T, B, H, [tuple(L)] * H)
+        for _ in range(2):
+            sta.sta_forward(full, qt, kt, vt, ot, lset, scale)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record()
+        for _ in range(reps):
+            sta.sta_forward(full, qt, kt, vt, ot, lset, scale)
+        e1.record()
+        torch.cuda.synchronize()
+        full_ms = max_over_ranks(e0.elapsed_time(e1) / reps)
+        ideal = full.stats()[0] / plan.stats()[0]
+        extras["full_window"] = {"ms": full_ms, "tflops": full.flops(d) / (full_ms * 1e-3) / 1e12,
+                                 "speedup": full_ms / fwd_ms, "ideal_speedup": ideal,
+                                 "frac_of_ideal": (full_ms / fwd_ms) / ideal}
+        if sta.sta_last_device_status(full) != 0:
+            raise RuntimeError("device status error in the full-window run")
+        full.destroy()
+        # ------------------------------------------- permutation bandwidth
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            sta.sta_tile_reorder(q, qt, L, T)
+        e1.record()
+        torch.cuda.synchronize()
+        perm_ms = e0.elapsed_time(e1) / 5
+        nbytes = q.numel() * q.element_size()
+        extras["permutation"] = {"ms": perm_ms, "gbs": 2 * nbytes / (perm_ms * 1e-3) / 1e9,
+                                 "peak_gbs": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
+                                 "bytes_per_launch": 2 * nbytes}
+        extras["permutation"]["frac"] = extras["permutation"]["gbs"] / extras["permutation"]["peak_gbs"]
+        # ------------------------------------------- end to end from pinned host memory
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+        e2e_steps = max(2, min(args.steps, 5))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * nbytes,
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_extras:
+        cpu = cpu_baseline(w, n_tiles=2, heads=[0])
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "heads": H, "head_dim": d, "latent": list(L),
+                       "tile": list(T), "window": wins[0] if w.window else "per-head",
+                       "tokens": N, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (3 x %.1f MB per step), no flush" % (q.numel() * 2 / 1e6),
+                       "step": "reorder Q,K,V + sta_forward + unreorder O,LSE; plan built once"},
+            "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": fwd_tflops / peak, "traffic": measured_traffic(),
+                         "kernel": "sta_fwd_kernel<128>",
+                         "peak_source": f"bf16_tflops_sustained ({peak_kind})",
+                         "frac_of_burst": fwd_tflops / float(peaks.get("bf16_tflops", 1590.0))},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            **extras,
+        }
+        print(json.dumps(line), flush=True)
+    plan.destroy()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

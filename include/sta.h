@@ -1,0 +1,158 @@
+/*
+ * sta.h -- C ABI of the Sliding Tile Attention (STA) forward library (libsta).
+ *
+ * The method: "Fast Video Generation with Sliding Tile Attention".  A video
+ * latent of L_t x L_h x L_w tokens is cut into tiles, contiguous cubes of
+ * T_t x T_h x T_w tokens whose size equals one attention block (podcast
+ * transcript at hotaipapers.com, segment on tiles and FlashAttention blocks).
+ * Each query tile attends, with exact softmax, only to the key/value tiles
+ * inside a 3D window of tiles centred on it; the window slides tile by tile, so
+ * all queries of a tile share one key set and every computed block is dense
+ * (same transcript, segment on dense / empty / mixed blocks; dianyo.github.io
+ * ICML-2025 post, STA section "Observation & Proposed Method").  The window is
+ * chosen per head (transcript, segment on head specialisation).
+ *
+ * Readings fixed by this library where the pages are silent:
+ *   - window extent in tiles e_d = min(W_d / T_d, n_d), n_d = L_d / T_d;
+ *   - window start s_d = clamp(q_d - floor(e_d / 2), 0, n_d - e_d): the window
+ *     is shifted to stay inside the volume (this is the reading that gives the
+ *     91% sparsity the atlas.scime.ai summary reports for w = (18,24,24));
+ *   - tile-major token order: tiles in raster order over the tile grid, tokens
+ *     inside a tile in raster order over (t, h, w) offsets, w fastest;
+ *   - LSE = m + ln(sum exp(s - m)) in natural-log, scaled-score units.
+ *
+ * Conventions for every call:
+ *   - All tensors are row-major [B, heads, N, d] with N = L_t * L_h * L_w,
+ *     owned by the caller, device-resident, contiguous.  q/k/v/o must be
+ *     16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device work
+ *     is enqueued asynchronously on it; nothing here synchronises except
+ *     sta_plan, sta_plan_destroy and sta_last_device_status.
+ *   - Calls return a status and never throw, abort or print.  Argument errors
+ *     are detected before any launch.  Faults and device-side timeouts of
+ *     launched work are reported by sta_last_device_status.
+ */
+#ifndef STA_H_
+#define STA_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define STA_API __attribute__((visibility("default")))
+#else
+#define STA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STA_OK = 0,
+    STA_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, geometry mismatch */
+    STA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. head_dim) */
+    STA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    STA_ERR_TIMEOUT = 4,     /* a device-side wait ran past its time limit */
+    STA_ERR_OOM = 5          /* device or host allocation failed */
+} sta_status;
+
+/* Latent and tile extents in tokens, (t, h, w) order. */
+typedef struct {
+    int32_t lat_t, lat_h, lat_w;
+    int32_t tile_t, tile_h, tile_w;
+} sta_geom;
+
+/* Opaque plan: the per-head key-tile lists and the work list of one
+ * (geometry, batch, heads, windows) problem.  Library-owned. */
+typedef struct sta_plan_s* sta_plan_t;
+
+/* Build a plan and upload it to the current CUDA device.
+ *   g          : geometry; every L_d must be a positive multiple of T_d.
+ *   batch      : B >= 1;  heads: H >= 1
+ *   window_thw : host array [heads][3], window per head in tokens; every entry
+ *                a positive multiple of the tile extent on its axis (windows
+ *                wider than the volume are clamped to it)
+ *   stream     : stream for the upload (the call waits for it to finish)
+ *   out        : receives the plan handle
+ * The plan holds, per distinct window, the ascending list of key-tile ids of
+ * every query tile (CSR), and a work list of (b, h, query row block) items in
+ * descending order of list length.  Allocates device memory; free it with
+ * sta_plan_destroy.  Errors: INVALID_ARG, UNSUPPORTED (tile volume not a
+ * multiple of 128 tokens), OOM, CUDA. */
+STA_API sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
+                    const int32_t* window_thw, void* stream, sta_plan_t* out);
+
+/* Same plan, host side only (no device memory, no CUDA call): for inspection
+ * with sta_plan_query / sta_plan_stats on machines without a GPU.  A host-only
+ * plan is rejected by sta_forward with INVALID_ARG. */
+STA_API sta_status sta_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
+                         const int32_t* window_thw, sta_plan_t* out);
+
+/* Release a plan and its device memory (synchronises the device first).
+ * NULL is accepted.  The handle must not be in use by queued work. */
+STA_API sta_status sta_plan_destroy(sta_plan_t p);
+
+/* Key-tile list of query tile `q_tile` (raster tile id) for head `head`:
+ * writes min(count, cap) ascending tile ids to kv_ids (host) and the full
+ * length to *count.  INVALID_ARG on a bad head / tile / pointer. */
+STA_API sta_status sta_plan_query(sta_plan_t p, int32_t head, int32_t q_tile,
+                          int32_t* kv_ids, int32_t cap, int32_t* count);
+
+/* Plan totals: computed (query tile, key tile) pairs over all batches and
+ * heads, and number of work items.  Either pointer may be NULL. */
+STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, int64_t* work_items);
+
+/* Copy the plan's work list to host memory, four int32 per item:
+ * (b * heads + h, first 128-row query block, second block or -1, window id).
+ * Row block r covers tile-major rows [128 r, 128 r + 128) of its head.  Writes
+ * min(count, cap) items and the full count to *count.  For tests/inspection. */
+STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
+
+/* Raster -> tile-major token permutation.
+ *   src, dst  : device, [outer, N, row_bytes] bytes, distinct buffers
+ *   outer     : B * heads (any count >= 1)
+ *   row_bytes : bytes of one token row (d * element size; 4 for a fp32 LSE
+ *               row); rows move intact, bit-exact
+ * dst[o, tile_major(i)] = src[o, i] for every raster token i. */
+STA_API sta_status sta_tile_reorder(const void* src, void* dst, int64_t outer,
+                            int32_t row_bytes, const sta_geom* g, void* stream);
+
+/* Inverse permutation: dst[o, i] = src[o, tile_major(i)]. */
+STA_API sta_status sta_tile_unreorder(const void* src, void* dst, int64_t outer,
+                              int32_t row_bytes, const sta_geom* g, void* stream);
+
+/* STA forward on tile-major tensors.
+ *   q, k, v : device bf16 [B, heads, N, d], tile-major token order
+ *   o       : device bf16 [B, heads, N, d], tile-major (written)
+ *   lse     : device fp32 [B, heads, N], tile-major (written): natural-log
+ *             log-sum-exp of the scaled scores of each query row
+ *   head_dim: d, 64 or 128 (else UNSUPPORTED)
+ *   softmax_scale: multiplies q . k before the softmax (e.g. 1/sqrt(d));
+ *             finite and > 0, else INVALID_ARG
+ * For every (b, h) and query tile q, over the key tiles of the plan's list:
+ * S = scale * Q_q K^T, exact online softmax with running max and sum in fp32,
+ * O = softmax(S) V rounded to bf16.  Allocates nothing; enqueues one kernel on
+ * `stream`.  The plan must come from sta_plan on the current device. */
+STA_API sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v,
+                       void* o, float* lse, int32_t head_dim, float softmax_scale,
+                       void* stream);
+
+/* Synchronise `stream`, then report (and clear) the first asynchronous error
+ * of work enqueued with this plan: CUDA for a launch or execution fault,
+ * TIMEOUT when a device-side wait gave up. */
+STA_API sta_status sta_last_device_status(sta_plan_t p, void* stream);
+
+/* Static string naming a status code. */
+STA_API const char* sta_status_string(sta_status s);
+
+/* Debug only: when `enable` is non-zero, the next sta_forward calls make the
+ * kernel's first wait run out on a barrier nothing arrives at (time limit
+ * `limit_ms`), so the timeout path can be tested; the kernel then issues no
+ * copy or MMA and exits, and sta_last_device_status returns TIMEOUT. */
+STA_API sta_status sta_debug_inject_timeout(int32_t enable, int32_t limit_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STA_H_ */

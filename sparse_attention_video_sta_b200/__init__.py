@@ -1,0 +1,314 @@
+"""Sliding Tile Attention (STA) forward for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of the C-ABI library ``libsta.so`` (declared in
+``include/sta.h``).  This module only marshals arguments -- tensor pointers,
+sizes and the current CUDA stream -- and checks that tensor shapes match the
+plan; every step of the computation runs in the library's CUDA kernels.  There
+is no CPU fallback: importing this package fails if ``libsta.so`` is missing.
+
+The functions carry the C names:
+
+    sta_plan / sta_plan_host -> Plan  (per-head key-tile lists + work list)
+    sta_tile_reorder / sta_tile_unreorder  (raster <-> tile-major tokens)
+    sta_forward                             (STA attention on tile-major tensors)
+    sta_last_device_status, sta_status_string, sta_debug_inject_timeout
+
+and ``sta_attention`` chains them for raster-order tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "StaError", "Plan", "sta_plan", "sta_plan_host", "sta_tile_reorder", "sta_tile_unreorder",
+    "sta_forward", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
+    "sta_attention", "library_path", "EXPORTED_SYMBOLS",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG_DIR, "libsta.so")
+
+STA_OK = 0
+STA_ERR_INVALID_ARG = 1
+STA_ERR_UNSUPPORTED = 2
+STA_ERR_CUDA = 3
+STA_ERR_TIMEOUT = 4
+STA_ERR_OOM = 5
+
+EXPORTED_SYMBOLS = (
+    "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
+    "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward", "sta_last_device_status",
+    "sta_status_string", "sta_debug_inject_timeout",
+)
+
+
+class _Geom(ctypes.Structure):
+    _fields_ = [("lat_t", ctypes.c_int32), ("lat_h", ctypes.c_int32), ("lat_w", ctypes.c_int32),
+                ("tile_t", ctypes.c_int32), ("tile_h", ctypes.c_int32), ("tile_w", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"libsta.so not found at {_LIB_PATH}; build it with "
+            "`python sparse_attention_video_sta_b200/_build.py` (nvcc, sm_100a)")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    G = ctypes.POINTER(_Geom)
+    i32p, i64p = ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int64)
+    sig = {
+        "sta_plan": [G, i32, i32, i32p, vp, ctypes.POINTER(vp)],
+        "sta_plan_host": [G, i32, i32, i32p, ctypes.POINTER(vp)],
+        "sta_plan_destroy": [vp],
+        "sta_plan_query": [vp, i32, i32, i32p, i32, i32p],
+        "sta_plan_stats": [vp, i64p, i64p],
+        "sta_plan_work_items": [vp, i32p, i64, i64p],
+        "sta_tile_reorder": [vp, vp, i64, i32, G, vp],
+        "sta_tile_unreorder": [vp, vp, i64, i32, G, vp],
+        "sta_forward": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
+        "sta_last_device_status": [vp, vp],
+        "sta_debug_inject_timeout": [i32, i32],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    L.sta_status_string.argtypes = [ctypes.c_int]
+    L.sta_status_string.restype = ctypes.c_char_p
+    return L
+
+
+_lib = _load()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def sta_status_string(status: int) -> str:
+    return _lib.sta_status_string(int(status)).decode()
+
+
+class StaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {sta_status_string(status)}")
+
+
+def _check(status: int, what: str) -> None:
+    if status != STA_OK:
+        raise StaError(status, what)
+
+
+def _geom(latent, tile) -> _Geom:
+    return _Geom(int(latent[0]), int(latent[1]), int(latent[2]),
+                 int(tile[0]), int(tile[1]), int(tile[2]))
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _windows(heads: int, windows) -> ctypes.Array:
+    w = torch.as_tensor(windows, dtype=torch.int32).reshape(-1, 3)
+    if w.shape[0] == 1 and heads > 1:
+        w = w.expand(heads, 3)
+    if w.shape[0] != heads:
+        raise ValueError(f"expected {heads} windows, got {w.shape[0]}")
+    flat = w.contiguous().flatten().tolist()
+    return (ctypes.c_int32 * len(flat))(*flat)
+
+
+class Plan:
+    """Owner of a ``sta_plan_t`` handle (freed on ``destroy`` / garbage collection)."""
+
+    def __init__(self, handle: int, latent, tile, batch: int, heads: int, windows):
+        self._h = ctypes.c_void_p(handle)
+        self.latent = tuple(int(x) for x in latent)
+        self.tile = tuple(int(x) for x in tile)
+        self.batch = int(batch)
+        self.heads = int(heads)
+        self.windows = torch.as_tensor(windows, dtype=torch.int32).reshape(-1, 3)
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if not self._h:
+            raise ValueError("plan already destroyed")
+        return self._h
+
+    @property
+    def tokens(self) -> int:
+        return self.latent[0] * self.latent[1] * self.latent[2]
+
+    @property
+    def tiles_per_head(self) -> int:
+        return self.tokens // (self.tile[0] * self.tile[1] * self.tile[2])
+
+    def query(self, head: int, q_tile: int) -> list:
+        """Ascending key-tile ids attended by query tile ``q_tile`` of ``head``."""
+        count = ctypes.c_int32(0)
+        _check(_lib.sta_plan_query(self.handle, head, q_tile, None, 0, ctypes.byref(count)),
+               "sta_plan_query")
+        buf = (ctypes.c_int32 * max(count.value, 1))()
+        _check(_lib.sta_plan_query(self.handle, head, q_tile, buf, count.value, ctypes.byref(count)),
+               "sta_plan_query")
+        return list(buf[:count.value])
+
+    def stats(self) -> tuple:
+        """(computed query-tile/key-tile pairs over all b, h; work items)."""
+        pairs, items = ctypes.c_int64(0), ctypes.c_int64(0)
+        _check(_lib.sta_plan_stats(self.handle, ctypes.byref(pairs), ctypes.byref(items)),
+               "sta_plan_stats")
+        return pairs.value, items.value
+
+    def work_items(self):
+        """Work list as a list of (bh, first row block, second row block or -1, window id)."""
+        count = ctypes.c_int64(0)
+        _check(_lib.sta_plan_work_items(self.handle, None, 0, ctypes.byref(count)), "sta_plan_work_items")
+        buf = (ctypes.c_int32 * max(4 * count.value, 4))()
+        _check(_lib.sta_plan_work_items(self.handle, buf, count.value, ctypes.byref(count)),
+               "sta_plan_work_items")
+        flat = list(buf[:4 * count.value])
+        return [tuple(flat[4 * i:4 * i + 4]) for i in range(count.value)]
+
+    def flops(self, head_dim: int) -> float:
+        """Attention FLOPs over computed tiles: pairs * 4 * |tile|^2 * d."""
+        vol = self.tile[0] * self.tile[1] * self.tile[2]
+        return float(self.stats()[0]) * 4.0 * vol * vol * head_dim
+
+    def destroy(self) -> None:
+        if self._h:
+            _check(_lib.sta_plan_destroy(self._h), "sta_plan_destroy")
+            self._h = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            if self._h:
+                _lib.sta_plan_destroy(self._h)
+                self._h = ctypes.c_void_p(0)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.destroy()
+
+
+def sta_plan(latent, tile, batch: int, heads: int, windows, stream=None) -> Plan:
+    """Build a plan on the current CUDA device (windows: ``[heads, 3]`` tokens)."""
+    h = ctypes.c_void_p(0)
+    g = _geom(latent, tile)
+    _check(_lib.sta_plan(ctypes.byref(g), int(batch), int(heads), _windows(heads, windows),
+                         _stream(stream), ctypes.byref(h)), "sta_plan")
+    return Plan(h.value, latent, tile, batch, heads, windows)
+
+
+def sta_plan_host(latent, tile, batch: int, heads: int, windows) -> Plan:
+    """Host-only plan (no device memory): for ``query`` / ``stats`` without a GPU."""
+    h = ctypes.c_void_p(0)
+    g = _geom(latent, tile)
+    _check(_lib.sta_plan_host(ctypes.byref(g), int(batch), int(heads), _windows(heads, windows),
+                              ctypes.byref(h)), "sta_plan_host")
+    return Plan(h.value, latent, tile, batch, heads, windows)
+
+
+def _perm_args(src: torch.Tensor, dst: torch.Tensor, tokens: int, token_dim: int):
+    if not (src.is_cuda and dst.is_cuda):
+        raise ValueError("sta_tile_reorder/unreorder need CUDA tensors")
+    if src.shape != dst.shape or src.dtype != dst.dtype:
+        raise ValueError("src and dst must have the same shape and dtype")
+    if not (src.is_contiguous() and dst.is_contiguous()):
+        raise ValueError("src and dst must be contiguous")
+    td = token_dim % src.dim()
+    if src.shape[td] != tokens:
+        raise ValueError(f"dimension {td} has {src.shape[td]} tokens, geometry has {tokens}")
+    outer = math.prod(src.shape[:td]) if td > 0 else 1
+    row_bytes = math.prod(src.shape[td + 1:]) * src.element_size()
+    return outer, row_bytes
+
+
+def sta_tile_reorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_dim: int = 2,
+                     stream=None) -> torch.Tensor:
+    """dst = src with the token dimension permuted raster -> tile-major."""
+    outer, row_bytes = _perm_args(src, dst, latent[0] * latent[1] * latent[2], token_dim)
+    g = _geom(latent, tile)
+    _check(_lib.sta_tile_reorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
+                                 outer, row_bytes, ctypes.byref(g), _stream(stream)),
+           "sta_tile_reorder")
+    return dst
+
+
+def sta_tile_unreorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_dim: int = 2,
+                       stream=None) -> torch.Tensor:
+    """dst = src with the token dimension permuted tile-major -> raster."""
+    outer, row_bytes = _perm_args(src, dst, latent[0] * latent[1] * latent[2], token_dim)
+    g = _geom(latent, tile)
+    _check(_lib.sta_tile_unreorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
+                                   outer, row_bytes, ctypes.byref(g), _stream(stream)),
+           "sta_tile_unreorder")
+    return dst
+
+
+def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
+    """STA forward on tile-major ``[B, H, N, d]`` bf16 tensors; writes ``o`` and ``lse``."""
+    B, H, N = plan.batch, plan.heads, plan.tokens
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+        if t.dim() != 4 or tuple(t.shape[:3]) != (B, H, N):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, plan expects [{B}, {H}, {N}, d]")
+    d = q.shape[3]
+    if k.shape[3] != d or v.shape[3] != d or o.shape[3] != d:
+        raise ValueError("q, k, v, o must share the head dimension")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() \
+            or tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape [{B}, {H}, {N}]")
+    _check(_lib.sta_forward(plan.handle, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                            ctypes.c_void_p(lse.data_ptr()), int(d), float(softmax_scale),
+                            _stream(stream)), "sta_forward")
+    return o, lse
+
+
+def sta_last_device_status(plan: Plan, stream=None) -> int:
+    """Synchronise and return (clearing it) the plan's device status code."""
+    return int(_lib.sta_last_device_status(plan.handle, _stream(stream)))
+
+
+def sta_debug_inject_timeout(enable: bool, limit_ms: int = 50) -> None:
+    _check(_lib.sta_debug_inject_timeout(1 if enable else 0, int(limit_ms)), "sta_debug_inject_timeout")
+
+
+def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
+                  softmax_scale: float | None = None, stream=None):
+    """STA attention on raster-order ``[B, H, N, d]`` bf16 tensors.
+
+    Permutes Q, K, V to tile-major order, runs the forward kernel, and permutes
+    O and LSE back.  Returns ``(O bf16 [B, H, N, d], LSE fp32 [B, H, N])``.
+    """
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(q.shape[-1])
+    lat, tile = plan.latent, plan.tile
+    qt, kt, vt = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    sta_tile_reorder(q, qt, lat, tile, stream=stream)
+    sta_tile_reorder(k, kt, lat, tile, stream=stream)
+    sta_tile_reorder(v, vt, lat, tile, stream=stream)
+    ot = torch.empty_like(q)
+    lset = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    sta_forward(plan, qt, kt, vt, ot, lset, softmax_scale, stream=stream)
+    o = torch.empty_like(q)
+    lse = torch.empty_like(lset)
+    sta_tile_unreorder(ot, o, lat, tile, stream=stream)
+    sta_tile_unreorder(lset, lse, lat, tile, stream=stream)
+    return o, lse

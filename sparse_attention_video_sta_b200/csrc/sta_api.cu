@@ -1,0 +1,347 @@
+// sta_api.cu -- host side of the libsta C ABI: argument checks, the plan
+// builder, and the launch / status plumbing around the kernels.
+//
+// The plan follows "Fast Video Generation with Sliding Tile Attention": every
+// query tile attends the key tiles of a window of tiles centred on it, shifted
+// to stay inside the volume, with one window per head (podcast transcript at
+// hotaipapers.com, segments on tiles and on head specialisation; dianyo.github.io
+// ICML-2025 post, STA section "Observation & Proposed Method").
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <new>
+#include <tuple>
+#include <vector>
+
+#include "sta.h"
+#include "sta_internal.h"
+
+namespace {
+
+using sta::PlanHost;
+using sta::WorkItem;
+
+std::atomic<int> g_inject_timeout{0};
+std::atomic<int> g_inject_limit_ms{50};
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+
+bool geom_valid(const sta_geom* g) {
+    if (g == nullptr) return false;
+    const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
+    const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
+    for (int d = 0; d < 3; ++d) {
+        if (L[d] <= 0 || T[d] <= 0 || L[d] % T[d] != 0) return false;
+    }
+    const int64_t n = int64_t(L[0]) * L[1] * L[2];
+    return n <= INT32_MAX;
+}
+
+// Window start in tiles along one axis: centred on q, extent e, inside [0, n).
+int32_t window_start(int32_t q, int32_t e, int32_t n) {
+    return std::min(std::max(q - e / 2, 0), n - e);
+}
+
+sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
+                           const int32_t* window_thw, PlanHost& P) {
+    if (!geom_valid(g) || batch < 1 || heads < 1 || window_thw == nullptr)
+        return STA_ERR_INVALID_ARG;
+    const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
+    const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
+    for (int32_t h = 0; h < heads; ++h)
+        for (int d = 0; d < 3; ++d) {
+            const int32_t w = window_thw[3 * h + d];
+            if (w <= 0 || w % T[d] != 0) return STA_ERR_INVALID_ARG;
+        }
+    P.g = *g;
+    P.batch = batch;
+    P.heads = heads;
+    for (int d = 0; d < 3; ++d) P.n_tiles[d] = L[d] / T[d];
+    P.tiles_per_head = P.n_tiles[0] * P.n_tiles[1] * P.n_tiles[2];
+    P.tile_tokens = T[0] * T[1] * T[2];
+    if (P.tile_tokens % sta::kSubRows != 0) return STA_ERR_UNSUPPORTED;
+    P.sub_per_tile = P.tile_tokens / sta::kSubRows;
+    const int64_t n_tok = int64_t(P.tiles_per_head) * P.tile_tokens;
+    // Row coordinates of the kernel's tensor maps are int32.
+    if (int64_t(batch) * heads * n_tok > INT32_MAX) return STA_ERR_UNSUPPORTED;
+
+    // Distinct clamped windows.
+    std::map<std::tuple<int32_t, int32_t, int32_t>, int32_t> ids;
+    P.head_win.assign(heads, 0);
+    P.win_ext.clear();
+    for (int32_t h = 0; h < heads; ++h) {
+        int32_t e[3];
+        for (int d = 0; d < 3; ++d) e[d] = std::min(window_thw[3 * h + d] / T[d], P.n_tiles[d]);
+        auto key = std::make_tuple(e[0], e[1], e[2]);
+        auto it = ids.find(key);
+        if (it == ids.end()) {
+            const int32_t id = int32_t(ids.size());
+            ids.emplace(key, id);
+            P.win_ext.insert(P.win_ext.end(), {e[0], e[1], e[2]});
+            P.head_win[h] = id;
+        } else {
+            P.head_win[h] = it->second;
+        }
+    }
+    const int32_t n_win = int32_t(ids.size());
+
+    // Key-tile lists (CSR), ascending linear tile id.
+    const int32_t nt = P.n_tiles[0], nh = P.n_tiles[1], nw = P.n_tiles[2];
+    P.csr_off.assign(size_t(n_win) * (P.tiles_per_head + 1), 0);
+    P.csr_ids.clear();
+    std::vector<int32_t> list_len(n_win, 0);
+    for (int32_t w = 0; w < n_win; ++w) {
+        const int32_t* e = &P.win_ext[3 * w];
+        list_len[w] = e[0] * e[1] * e[2];
+        int32_t* off = &P.csr_off[size_t(w) * (P.tiles_per_head + 1)];
+        for (int32_t qt = 0; qt < nt; ++qt)
+            for (int32_t qh = 0; qh < nh; ++qh)
+                for (int32_t qw = 0; qw < nw; ++qw) {
+                    const int32_t q = (qt * nh + qh) * nw + qw;
+                    off[q] = int32_t(P.csr_ids.size());
+                    const int32_t st = window_start(qt, e[0], nt);
+                    const int32_t sh = window_start(qh, e[1], nh);
+                    const int32_t sw = window_start(qw, e[2], nw);
+                    for (int32_t kt = st; kt < st + e[0]; ++kt)
+                        for (int32_t kh = sh; kh < sh + e[1]; ++kh)
+                            for (int32_t kw = sw; kw < sw + e[2]; ++kw)
+                                P.csr_ids.push_back((kt * nh + kh) * nw + kw);
+                }
+        off[P.tiles_per_head] = int32_t(P.csr_ids.size());
+    }
+
+    // Work items.  Row blocks of one tile are paired so the pair shares K/V
+    // loads; with an odd count per tile, the last block of consecutive tiles
+    // are paired instead (each with its own list, same length).
+    const int32_t S = P.sub_per_tile;
+    P.items.clear();
+    P.computed_pairs = 0;
+    for (int32_t b = 0; b < batch; ++b)
+        for (int32_t h = 0; h < heads; ++h) {
+            const int32_t bh = b * heads + h, win = P.head_win[h];
+            P.computed_pairs += int64_t(P.tiles_per_head) * list_len[win];
+            int32_t pending = -1;
+            for (int32_t t = 0; t < P.tiles_per_head; ++t) {
+                for (int32_t s = 0; s + 1 < S; s += 2)
+                    P.items.push_back(WorkItem{bh, t * S + s, t * S + s + 1, win});
+                if (S % 2 == 1) {
+                    const int32_t blk = t * S + S - 1;
+                    if (pending < 0) {
+                        pending = blk;
+                    } else {
+                        P.items.push_back(WorkItem{bh, pending, blk, win});
+                        pending = -1;
+                    }
+                }
+            }
+            if (pending >= 0) P.items.push_back(WorkItem{bh, pending, -1, win});
+        }
+    // Longest lists first (stable: neighbouring tiles stay together for L2 reuse).
+    std::stable_sort(P.items.begin(), P.items.end(), [&](const WorkItem& a, const WorkItem& b) {
+        return list_len[a.win] > list_len[b.win];
+    });
+    return STA_OK;
+}
+
+void free_device(sta_plan_s* p) {
+    if (p->d_off) cudaFree(p->d_off);
+    if (p->d_ids) cudaFree(p->d_ids);
+    if (p->d_items) cudaFree(p->d_items);
+    if (p->d_status) cudaFree(p->d_status);
+    p->d_off = nullptr;
+    p->d_ids = nullptr;
+    p->d_items = nullptr;
+    p->d_status = nullptr;
+    p->on_device = false;
+}
+
+template <class T>
+cudaError_t upload(T** dst, const std::vector<T>& src, cudaStream_t stream) {
+    const size_t bytes = std::max<size_t>(src.size(), 1) * sizeof(T);
+    cudaError_t e = cudaMalloc(reinterpret_cast<void**>(dst), bytes);
+    if (e != cudaSuccess) return e;
+    if (!src.empty()) e = cudaMemcpyAsync(*dst, src.data(), src.size() * sizeof(T),
+                                          cudaMemcpyHostToDevice, stream);
+    return e;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row_bytes,
+                          const sta_geom* g, void* stream, bool inverse) {
+    if (src == nullptr || dst == nullptr || !geom_valid(g) || outer < 1 || row_bytes <= 0)
+        return STA_ERR_INVALID_ARG;
+    const int64_t n_tok = int64_t(g->lat_t) * g->lat_h * g->lat_w;
+    const int64_t bytes = outer * n_tok * int64_t(row_bytes);
+    const uintptr_t s = reinterpret_cast<uintptr_t>(src), d = reinterpret_cast<uintptr_t>(dst);
+    if (s < d + uint64_t(bytes) && d < s + uint64_t(bytes)) return STA_ERR_INVALID_ARG;  // overlap
+    cudaError_t e = sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sta_status_string(sta_status s) {
+    switch (s) {
+        case STA_OK: return "STA_OK";
+        case STA_ERR_INVALID_ARG: return "STA_ERR_INVALID_ARG";
+        case STA_ERR_UNSUPPORTED: return "STA_ERR_UNSUPPORTED";
+        case STA_ERR_CUDA: return "STA_ERR_CUDA";
+        case STA_ERR_TIMEOUT: return "STA_ERR_TIMEOUT";
+        case STA_ERR_OOM: return "STA_ERR_OOM";
+    }
+    return "STA_ERR_UNKNOWN";
+}
+
+sta_status sta_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
+                         const int32_t* window_thw, sta_plan_t* out) {
+    if (out == nullptr) return STA_ERR_INVALID_ARG;
+    *out = nullptr;
+    sta_plan_s* p = new (std::nothrow) sta_plan_s();
+    if (p == nullptr) return STA_ERR_OOM;
+    sta_status st;
+    try {
+        st = build_plan_host(g, batch, heads, window_thw, p->h);
+    } catch (const std::bad_alloc&) {
+        st = STA_ERR_OOM;
+    }
+    if (st != STA_OK) {
+        delete p;
+        return st;
+    }
+    *out = p;
+    return STA_OK;
+}
+
+sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
+                    const int32_t* window_thw, void* stream, sta_plan_t* out) {
+    sta_status st = sta_plan_host(g, batch, heads, window_thw, out);
+    if (st != STA_OK) return st;
+    sta_plan_s* p = *out;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaGetDevice(&p->device);
+    if (e == cudaSuccess) e = upload(&p->d_off, p->h.csr_off, s);
+    if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
+    if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
+    if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&p->d_status), sizeof(uint32_t));
+    if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) {
+        const bool oom = (e == cudaErrorMemoryAllocation);
+        cudaGetLastError();
+        free_device(p);
+        delete p;
+        *out = nullptr;
+        return oom ? STA_ERR_OOM : STA_ERR_CUDA;
+    }
+    p->on_device = true;
+    return STA_OK;
+}
+
+sta_status sta_plan_destroy(sta_plan_t p) {
+    if (p == nullptr) return STA_OK;
+    sta_status st = STA_OK;
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status) {
+        if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
+        free_device(p);
+    }
+    delete p;
+    return st;
+}
+
+sta_status sta_plan_query(sta_plan_t p, int32_t head, int32_t q_tile, int32_t* kv_ids,
+                          int32_t cap, int32_t* count) {
+    if (p == nullptr || count == nullptr || cap < 0 || (cap > 0 && kv_ids == nullptr))
+        return STA_ERR_INVALID_ARG;
+    const PlanHost& P = p->h;
+    if (head < 0 || head >= P.heads || q_tile < 0 || q_tile >= P.tiles_per_head)
+        return STA_ERR_INVALID_ARG;
+    const int32_t* off = &P.csr_off[size_t(P.head_win[head]) * (P.tiles_per_head + 1)];
+    const int32_t n = off[q_tile + 1] - off[q_tile];
+    *count = n;
+    for (int32_t i = 0; i < std::min(n, cap); ++i) kv_ids[i] = P.csr_ids[off[q_tile] + i];
+    return STA_OK;
+}
+
+sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, int64_t* work_items) {
+    if (p == nullptr) return STA_ERR_INVALID_ARG;
+    if (computed_tile_pairs) *computed_tile_pairs = p->h.computed_pairs;
+    if (work_items) *work_items = int64_t(p->h.items.size());
+    return STA_OK;
+}
+
+sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count) {
+    if (p == nullptr || count == nullptr || cap < 0 || (cap > 0 && items4 == nullptr))
+        return STA_ERR_INVALID_ARG;
+    const auto& it = p->h.items;
+    *count = int64_t(it.size());
+    const int64_t n = std::min<int64_t>(cap, int64_t(it.size()));
+    for (int64_t i = 0; i < n; ++i) {
+        items4[4 * i + 0] = it[i].bh;
+        items4[4 * i + 1] = it[i].qa;
+        items4[4 * i + 2] = it[i].qb;
+        items4[4 * i + 3] = it[i].win;
+    }
+    return STA_OK;
+}
+
+sta_status sta_tile_reorder(const void* src, void* dst, int64_t outer, int32_t row_bytes,
+                            const sta_geom* g, void* stream) {
+    return permute_common(src, dst, outer, row_bytes, g, stream, false);
+}
+
+sta_status sta_tile_unreorder(const void* src, void* dst, int64_t outer, int32_t row_bytes,
+                              const sta_geom* g, void* stream) {
+    return permute_common(src, dst, outer, row_bytes, g, stream, true);
+}
+
+sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v, void* o,
+                       float* lse, int32_t head_dim, float softmax_scale, void* stream) {
+    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
+        return STA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return STA_ERR_CUDA;
+    if (dev != p->device) return STA_ERR_INVALID_ARG;
+    const int inject = g_inject_timeout.load();
+    const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
+                                  : kDefaultTimeoutNs;
+    cudaError_t e = sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
+                                        static_cast<cudaStream_t>(stream), inject, limit);
+    return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+}
+
+sta_status sta_last_device_status(sta_plan_t p, void* stream) {
+    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return STA_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return STA_ERR_CUDA;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, p->d_status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return STA_ERR_CUDA;
+    if (word != 0 && cudaMemset(p->d_status, 0, sizeof word) != cudaSuccess) return STA_ERR_CUDA;
+    if (word & sta::kDevTimeout) return STA_ERR_TIMEOUT;
+    return STA_OK;
+}
+
+sta_status sta_debug_inject_timeout(int32_t enable, int32_t limit_ms) {
+    if (limit_ms < 1 || limit_ms > 10000) return STA_ERR_INVALID_ARG;
+    g_inject_timeout.store(enable ? 1 : 0);
+    g_inject_limit_ms.store(limit_ms);
+    return STA_OK;
+}
+
+}  // extern "C"

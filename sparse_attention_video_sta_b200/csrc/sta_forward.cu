@@ -1,0 +1,502 @@
+// sta_forward.cu -- Sliding Tile Attention forward for sm_100a (B200).
+//
+// Method ("Fast Video Generation with Sliding Tile Attention"): each query tile
+// attends, with exact softmax, to the key tiles listed by the plan (a window of
+// tiles centred on it); because the window slides tile by tile, every computed
+// (query tile, key tile) block is dense and needs no mask (podcast transcript at
+// hotaipapers.com, segments on tiles and on dense / empty / mixed blocks).  The
+// pages' own kernel splits a thread block into data warpgroups that load K/V and
+// manage the sparse tile list, and compute warpgroups doing dense attention math
+// (same transcript, segment on ThunderKittens); the design below keeps that
+// split but is built for Blackwell:
+//
+//   warp 8 (load)    : TMA loads of the query blocks and of 128-key K / V chunks
+//                      of the listed key tiles into a ring of shared-memory stages
+//   warp 9 (MMA)     : one thread issues tcgen05.mma: S = Q K^T into TMEM, then
+//                      O += P V with P read straight from TMEM
+//   warps 0-3, 4-7   : softmax for query slot 0 / 1: tcgen05.ld of S, online
+//                      softmax (fp32 running max / sum, exp2 with the scale folded
+//                      in, lazy rescale of O), bf16 P written back into TMEM over
+//                      S, and the epilogue O / l -> bf16, LSE
+//
+// A work item is up to two 128-row query blocks (slots) of one (b, h).  Blocks of
+// the same tile share every K/V chunk; the two slots ping-pong so the tensor core
+// computes one slot's S while the other slot's softmax runs.  TMEM (512 columns):
+// S0 | S1 | O0 | O1.  The kernel is persistent (one CTA per SM) over the plan's
+// work list, longest key lists first.  Every mbarrier wait has a time limit; on
+// expiry the kernel records STA timeout status, drains its copies and MMAs, frees
+// TMEM and exits.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "sta_internal.h"
+#include "sta_ptx.cuh"
+
+namespace sta {
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+template <int D>
+struct Cfg {
+    static constexpr int kColBlocks = D / 64;             // 128-byte swizzle columns per row
+    static constexpr int kBoxBytes = 128 * 128;           // one TMA box: 128 rows x 128 bytes
+    static constexpr int kQBytes = kSubRows * D * 2;      // one 128-row query block
+    static constexpr int kKVBytes = kChunkKeys * D * 2;   // one 128-key K or V chunk
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kQOff = 0;
+    static constexpr int kRingOff = 2 * kQBytes;
+    static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
+    // barriers: full[S], empty[S], q_full, q_empty, s_full[2], p_full[2], o_full[2],
+    // o_empty[2], dead, drain
+    static constexpr int kNumBars = 2 * kStages + 12;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot + abort flag
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+    // TMEM columns: S0 | S1 | O0 | O1
+    __host__ __device__ static constexpr uint32_t col_s(int slot) { return uint32_t(slot) * 128u; }
+    __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256u + uint32_t(slot) * D; }
+    static_assert(256 + 2 * D <= int(kTmemCols), "TMEM budget");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+struct FwdParams {
+    const WorkItem* items;
+    int32_t n_items;
+    const int32_t* off;  // CSR offsets [n_win][tiles + 1]
+    const int32_t* ids;  // CSR key-tile ids
+    int32_t tiles_per_head;
+    int32_t sub_per_tile;  // 128-row blocks (= 128-key chunks) per tile
+    int32_t tile_tokens;
+    int32_t tokens;  // N per (b, h)
+    __nv_bfloat16* o;
+    float* lse;
+    float scale_log2;  // softmax_scale * log2(e)
+    float scale;
+    uint32_t* status;
+    uint64_t timeout_ns;
+    int32_t inject;
+};
+
+// Bounded mbarrier wait.  Returns false when the CTA is aborting (another role
+// gave up) or when this wait ran past the time limit (then it starts the abort).
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         const FwdParams& p) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (true) {
+        for (int i = 0; i < 32; ++i)
+            if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
+            *abort_flag = 1;
+            atomicOr(p.status, kDevTimeout);
+            return false;
+        }
+    }
+}
+
+// Drain wait used on the way out: bounded, never starts an abort.
+__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+        if (ptx::globaltimer_ns() - t0 > limit_ns) return;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = ptx::smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const uint32_t bar0 = base + C::kBarOff;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+    const uint32_t bar_q_full = bar0 + 8u * (2 * C::kStages + 0);
+    const uint32_t bar_q_empty = bar0 + 8u * (2 * C::kStages + 1);
+    auto bar_s_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 2 + j); };
+    auto bar_p_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 4 + j); };
+    auto bar_o_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 6 + j); };
+    auto bar_o_empty = [&](int j) { return bar0 + 8u * (2 * C::kStages + 8 + j); };
+    const uint32_t bar_dead = bar0 + 8u * (2 * C::kStages + 10);
+    const uint32_t bar_drain = bar0 + 8u * (2 * C::kStages + 11);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            ptx::mbar_init(bar_full(s), 1);
+            ptx::mbar_init(bar_empty(s), 1);
+        }
+        ptx::mbar_init(bar_q_full, 1);
+        ptx::mbar_init(bar_q_empty, 1);
+        for (int j = 0; j < 2; ++j) {
+            ptx::mbar_init(bar_s_full(j), 1);
+            ptx::mbar_init(bar_p_full(j), 128);
+            ptx::mbar_init(bar_o_full(j), 1);
+            ptx::mbar_init(bar_o_empty(j), 128);
+        }
+        ptx::mbar_init(bar_dead, 1);
+        ptx::mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        ptx::fence_barrier_init();
+        ptx::fence_proxy_async_smem();
+    }
+    if (warp == kLoadWarp && lane == 0) {
+        ptx::prefetch_tensormap(&tm_q);
+        ptx::prefetch_tensormap(&tm_k);
+        ptx::prefetch_tensormap(&tm_v);
+    }
+    if (warp == kMmaWarp) {
+        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int32_t SPT = p.sub_per_tile;
+
+    if (warp == kLoadWarp) {
+        if (lane == 0) {
+            // ------------------------------------------------------------ load
+            uint32_t item = 0, unit_n = 0;
+            bool ok = true;
+            if (p.inject) {
+                // Debug: wait on a barrier nothing arrives at; the limit runs out.
+                ok = wait_bar(bar_dead, 0, abort_flag, p);
+            }
+            auto issue = [&](const CUtensorMap* m, int32_t row) -> bool {
+                const int slot = int(item % C::kStages);
+                const uint32_t phase = item / C::kStages;
+                if (!wait_bar(bar_empty(slot), (phase & 1u) ^ 1u, abort_flag, p)) return false;
+                const uint32_t dst = base + C::kRingOff + slot * C::kKVBytes;
+                ptx::mbar_arrive_expect_tx(bar_full(slot), C::kKVBytes);
+#pragma unroll
+                for (int cb = 0; cb < C::kColBlocks; ++cb)
+                    ptx::tma_load_2d(dst + cb * C::kBoxBytes, m, bar_full(slot), cb * 64, row);
+                ++item;
+                return true;
+            };
+            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x, ++unit_n) {
+                const WorkItem w = p.items[u];
+                const bool has_b = w.qb >= 0;
+                const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
+                const bool split = has_b && tile_a != tile_b;
+                const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
+                const int32_t* list_a = p.ids + off[tile_a];
+                const int32_t* list_b = p.ids + off[tile_b];
+                const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
+                const int32_t head_row = w.bh * p.tokens;
+                // query blocks
+                if (!wait_bar(bar_q_empty, (unit_n & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
+                ptx::mbar_arrive_expect_tx(bar_q_full, (has_b ? 2 : 1) * C::kQBytes);
+#pragma unroll
+                for (int cb = 0; cb < C::kColBlocks; ++cb)
+                    ptx::tma_load_2d(base + C::kQOff + cb * C::kBoxBytes, &tm_q, bar_q_full, cb * 64,
+                                     head_row + w.qa * kSubRows);
+                if (has_b) {
+#pragma unroll
+                    for (int cb = 0; cb < C::kColBlocks; ++cb)
+                        ptx::tma_load_2d(base + C::kQOff + C::kQBytes + cb * C::kBoxBytes, &tm_q,
+                                         bar_q_full, cb * 64, head_row + w.qb * kSubRows);
+                }
+                // K / V chunks in the order the MMA warp consumes them
+                for (int32_t i = 0; ok && i < n_chunks; ++i) {
+                    const int32_t kt = i / SPT, kc = i - kt * SPT;
+                    const int32_t row_a = head_row + list_a[kt] * p.tile_tokens + kc * kChunkKeys;
+                    const int32_t row_b = head_row + list_b[kt] * p.tile_tokens + kc * kChunkKeys;
+                    ok = issue(&tm_k, row_a);
+                    if (ok && split) ok = issue(&tm_k, row_b);
+                    if (ok) ok = issue(&tm_v, row_a);
+                    if (ok && split) ok = issue(&tm_v, row_b);
+                }
+            }
+            // Drain: the copies issued last into each stage, and the last query load.
+            const uint32_t first = item > uint32_t(C::kStages) ? item - C::kStages : 0u;
+            for (uint32_t it = first; it < item; ++it)
+                drain_bar(bar_full(int(it % C::kStages)), (it / C::kStages) & 1u, p.timeout_ns);
+            if (unit_n > 0) drain_bar(bar_q_full, (unit_n - 1) & 1u, p.timeout_ns);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            // ------------------------------------------------------------- MMA
+            constexpr uint32_t idesc_qk = ptx::idesc_bf16(128, kChunkKeys, false);
+            constexpr uint32_t idesc_pv = ptx::idesc_bf16(128, D, true);
+            uint32_t item = 0, unit_n = 0;
+            uint32_t pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+            bool ok = true;
+            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x, ++unit_n) {
+                const WorkItem w = p.items[u];
+                const bool has_b = w.qb >= 0;
+                const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
+                const bool split = has_b && tile_a != tile_b;
+                const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
+                const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
+                const uint32_t width = split ? 4u : 2u;
+                const int n_slots = has_b ? 2 : 1;
+                const uint32_t ubase = item;
+                if (!wait_bar(bar_q_full, unit_n & 1u, abort_flag, p)) { ok = false; break; }
+                ptx::tc_fence_after();
+                for (int32_t i = 0; ok && i <= n_chunks; ++i) {
+                    for (int s = 0; ok && s < n_slots; ++s) {
+                        const bool last_slot = (s == n_slots - 1);
+                        const uint32_t k_it = ubase + uint32_t(i) * width + (split ? uint32_t(s) : 0u);
+                        const uint32_t v_it =
+                            ubase + uint32_t(i - 1) * width + (split ? 2u + uint32_t(s) : 1u);
+                        if (i >= 1) {
+                            // O_s += P_s(i-1) V(i-1)
+                            if (!wait_bar(bar_p_full(s), pcnt[s] & 1u, abort_flag, p)) { ok = false; break; }
+                            ++pcnt[s];
+                            if (!wait_bar(bar_full(int(v_it % C::kStages)), (v_it / C::kStages) & 1u,
+                                          abort_flag, p)) { ok = false; break; }
+                            if (i == 1 && !wait_bar(bar_o_empty(s), (ocnt[s] & 1u) ^ 1u, abort_flag, p)) {
+                                ok = false;
+                                break;
+                            }
+                            ptx::tc_fence_after();
+                            const uint32_t vaddr = base + C::kRingOff + (v_it % C::kStages) * C::kKVBytes;
+#pragma unroll
+                            for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
+                                const uint64_t bdesc = ptx::desc_mn_sw128(vaddr + kk * 16 * 128, C::kBoxBytes);
+                                ptx::mma_ts(tmem + C::col_o(s), tmem + C::col_s(s) + kk * 8, bdesc, idesc_pv,
+                                            (i > 1 || kk > 0) ? 1u : 0u);
+                            }
+                        }
+                        if (i < n_chunks) {
+                            // S_s(i) = Q_s K(i)^T
+                            if (!wait_bar(bar_full(int(k_it % C::kStages)), (k_it / C::kStages) & 1u,
+                                          abort_flag, p)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            const uint32_t qaddr = base + C::kQOff + s * C::kQBytes;
+                            const uint32_t kaddr = base + C::kRingOff + (k_it % C::kStages) * C::kKVBytes;
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t coff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+                                ptx::mma_ss(tmem + C::col_s(s), ptx::desc_k_sw128(qaddr + coff),
+                                            ptx::desc_k_sw128(kaddr + coff), idesc_qk, kk > 0 ? 1u : 0u);
+                            }
+                            ptx::mma_commit(bar_s_full(s));
+                        } else {
+                            ptx::mma_commit(bar_o_full(s));
+                            ++ocnt[s];
+                        }
+                        if (i >= 1 && (split || last_slot)) ptx::mma_commit(bar_empty(int(v_it % C::kStages)));
+                        if (i < n_chunks && (split || last_slot))
+                            ptx::mma_commit(bar_empty(int(k_it % C::kStages)));
+                    }
+                }
+                if (!ok) break;
+                ptx::mma_commit(bar_q_empty);
+                item = ubase + uint32_t(n_chunks) * width;
+            }
+            // Drain: every MMA issued so far completes before TMEM is freed.
+            ptx::mma_commit(bar_drain);
+            drain_bar(bar_drain, 0, p.timeout_ns);
+        }
+    } else {
+        // ------------------------------------------------------------- softmax
+        const int slot = warp >> 2;
+        const int row = threadIdx.x & 127;
+        const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_addr + C::col_s(slot);
+        const uint32_t tO = tmem + lane_addr + C::col_o(slot);
+        const float c = p.scale_log2;
+        uint32_t scnt = 0, ocnt = 0;
+        bool ok = true;
+        for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            const WorkItem w = p.items[u];
+            if (slot == 1 && w.qb < 0) continue;
+            const int32_t tile_a = w.qa / SPT;
+            const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
+            const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
+            const int32_t q_blk = slot == 0 ? w.qa : w.qb;
+            float m_used = 0.0f, l = 0.0f;
+            for (int32_t i = 0; i < n_chunks; ++i) {
+                if (!__all_sync(0xffffffffu, wait_bar(bar_s_full(slot), scnt & 1u, abort_flag, p))) {
+                    ok = false;
+                    break;
+                }
+                ++scnt;
+                ptx::tc_fence_after();
+                uint32_t sr[128];
+                ptx::tmem_ld128(tS, sr);
+                float mx = __uint_as_float(sr[0]);
+#pragma unroll
+                for (int j = 1; j < 128; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+                if (i == 0) {
+                    m_used = mx;
+                } else {
+                    const bool need = (mx - m_used) * c > kRescaleThreshold;
+                    if (__any_sync(0xffffffffu, need)) {
+                        const float m_new = need ? mx : m_used;
+                        const float alpha = ptx::ex2((m_used - m_new) * c);
+#pragma unroll 1
+                        for (int cb = 0; cb < D / 32; ++cb) {
+                            uint32_t orr[32];
+                            ptx::tmem_ld32(tO + cb * 32, orr);
+#pragma unroll
+                            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
+                            ptx::tmem_st32(tO + cb * 32, orr);
+                        }
+                        ptx::tmem_wait_st();
+                        l *= alpha;
+                        m_used = m_new;
+                    }
+                }
+                const float mc = m_used * c;
+                float rowsum = 0.0f;
+                uint32_t pk[64];
+#pragma unroll
+                for (int j = 0; j < 64; ++j) {
+                    const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * j]), c, -mc));
+                    const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -mc));
+                    rowsum += p0 + p1;
+                    pk[j] = ptx::pack_bf16x2(p0, p1);
+                }
+                ptx::tmem_st64(tS, pk);
+                ptx::tmem_wait_st();
+                l += rowsum;
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(bar_p_full(slot));
+            }
+            if (!ok) break;
+            // epilogue: O / l -> bf16, LSE
+            if (!__all_sync(0xffffffffu, wait_bar(bar_o_full(slot), ocnt & 1u, abort_flag, p))) {
+                ok = false;
+                break;
+            }
+            ++ocnt;
+            ptx::tc_fence_after();
+            const float inv_l = 1.0f / l;
+            const int64_t grow = int64_t(w.bh) * p.tokens + int64_t(q_blk) * kSubRows + row;
+            uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D);
+#pragma unroll 1
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t orr[32];
+                ptx::tmem_ld32(tO + cb * 32, orr);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 v;
+                    v.x = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 0]) * inv_l, __uint_as_float(orr[8 * j + 1]) * inv_l);
+                    v.y = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv_l, __uint_as_float(orr[8 * j + 3]) * inv_l);
+                    v.z = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv_l, __uint_as_float(orr[8 * j + 5]) * inv_l);
+                    v.w = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv_l, __uint_as_float(orr[8 * j + 7]) * inv_l);
+                    dst[cb * 4 + j] = v;
+                }
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(bar_o_empty(slot));
+            p.lse[grow] = m_used * p.scale + logf(l);
+        }
+    }
+
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        __syncwarp();
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+struct EncodeFn {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    cudaError_t err = cudaSuccess;
+};
+
+const EncodeFn& encode_fn() {
+    static EncodeFn e;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        e.err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+        if (e.err == cudaSuccess && q != cudaDriverEntryPointSuccess) e.err = cudaErrorNotSupported;
+        e.fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return e;
+}
+
+// 2D map over a [rows, d] bf16 matrix: box of 64 elements (128 bytes) x 128 rows,
+// 128-byte swizzle (the layout the tcgen05 shared-memory descriptors expect).
+cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) {
+    const EncodeFn& e = encode_fn();
+    if (e.err != cudaSuccess) return e.err;
+    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = e.fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const void* v, void* o,
+                     float* lse, float scale, cudaStream_t stream, int inject, uint64_t timeout_ns) {
+    const PlanHost& P = pl->h;
+    const int64_t rows = int64_t(P.batch) * P.heads * P.tiles_per_head * P.tile_tokens;
+    CUtensorMap mq, mk, mv;
+    cudaError_t e = make_map(&mq, q, rows, D);
+    if (e == cudaSuccess) e = make_map(&mk, k, rows, D);
+    if (e == cudaSuccess) e = make_map(&mv, v, rows, D);
+    if (e != cudaSuccess) return e;
+    FwdParams fp;
+    fp.items = pl->d_items;
+    fp.n_items = int32_t(P.items.size());
+    fp.off = pl->d_off;
+    fp.ids = pl->d_ids;
+    fp.tiles_per_head = P.tiles_per_head;
+    fp.sub_per_tile = P.sub_per_tile;
+    fp.tile_tokens = P.tile_tokens;
+    fp.tokens = P.tiles_per_head * P.tile_tokens;
+    fp.o = static_cast<__nv_bfloat16*>(o);
+    fp.lse = lse;
+    fp.scale = scale;
+    fp.scale_log2 = scale * 1.4426950408889634f;
+    fp.status = pl->d_status;
+    fp.timeout_ns = timeout_ns;
+    fp.inject = inject;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(sta_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int grid = fp.n_items < sms ? fp.n_items : sms;
+    if (grid <= 0) return cudaSuccess;
+    sta_fwd_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, const void* v, void* o,
+                           float* lse, int head_dim, float softmax_scale, cudaStream_t stream,
+                           int inject_timeout, uint64_t timeout_ns) {
+    if (head_dim == 128)
+        return launch_d<128>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns);
+    return launch_d<64>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns);
+}
+
+}  // namespace sta

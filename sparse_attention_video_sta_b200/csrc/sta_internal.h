@@ -1,0 +1,69 @@
+// sta_internal.h -- internal types shared by the libsta translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "sta.h"
+
+namespace sta {
+
+// Query rows per MMA slot (tcgen05 M for cta_group::1) and keys per K/V chunk.
+constexpr int kSubRows = 128;
+constexpr int kChunkKeys = 128;
+
+// Device status bits written by kernels (OR-ed).
+constexpr uint32_t kDevTimeout = 1u;
+
+// One work item of the forward kernel: up to two 128-row query blocks of the
+// same (b, h), each with its own key-tile list.  qb < 0 means one block only.
+// When both blocks belong to the same tile they share every K/V load.
+struct WorkItem {
+    int32_t bh;   // b * heads + h
+    int32_t qa;   // query row block within the head: tile * sub_per_tile + sub
+    int32_t qb;   // second row block or -1
+    int32_t win;  // distinct-window id of head h
+};
+static_assert(sizeof(WorkItem) == 16, "WorkItem is loaded as one int4");
+
+struct PlanHost {
+    sta_geom g;
+    int32_t batch = 0, heads = 0;
+    int32_t n_tiles[3] = {0, 0, 0};
+    int32_t tiles_per_head = 0;
+    int32_t tile_tokens = 0;
+    int32_t sub_per_tile = 0;                // tile_tokens / kSubRows
+    std::vector<int32_t> head_win;           // [heads] distinct-window id
+    std::vector<int32_t> win_ext;            // [n_win][3] clamped extents in tiles
+    std::vector<int32_t> csr_off;            // [n_win][tiles_per_head + 1], global offsets
+    std::vector<int32_t> csr_ids;            // key-tile ids, ascending per list
+    std::vector<WorkItem> items;             // work list
+    int64_t computed_pairs = 0;              // B * sum_h sum_q |list|
+};
+
+}  // namespace sta
+
+struct sta_plan_s {
+    sta::PlanHost h;
+    bool on_device = false;
+    int device = -1;
+    int32_t* d_off = nullptr;
+    int32_t* d_ids = nullptr;
+    sta::WorkItem* d_items = nullptr;
+    uint32_t* d_status = nullptr;
+};
+
+namespace sta {
+
+// Forward kernel launch (sta_forward.cu).  Returns a CUDA error code.
+cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, const void* v,
+                           void* o, float* lse, int head_dim, float softmax_scale,
+                           cudaStream_t stream, int inject_timeout, uint64_t timeout_ns);
+
+// Permutation launch (sta_permute.cu).  inverse = false: raster -> tile-major.
+cudaError_t launch_permute(const void* src, void* dst, int64_t outer, int32_t row_bytes,
+                           const sta_geom& g, bool inverse, cudaStream_t stream);
+
+}  // namespace sta

@@ -11,14 +11,18 @@ five configurations below.  Values are i.i.d. N(0, 1) drawn in fp32 and rounded
 to bf16 (round to nearest even), optionally multiplied per head by a factor
 f_h ~ U[0.5, 2] before the rounding (configuration 5).
 
-Every (configuration, tensor, batch, head) slice has its own seed, so any
-slice can be regenerated alone: the oracle only draws the heads it samples.
+Every (configuration, tensor, batch, head) slice has its own seed (numpy
+PCG64 stream), so any slice can be regenerated alone: the oracle only draws the
+heads it samples.  Slices are drawn on a thread pool.
 """
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 TILE = (6, 8, 8)
@@ -71,8 +75,7 @@ def windows(w: Workload) -> torch.Tensor:
     """``[heads, 3]`` int32 window per head, in tokens."""
     if w.window is not None:
         return torch.tensor([list(w.window)] * w.heads, dtype=torch.int32)
-    g = torch.Generator().manual_seed(w.seed)
-    idx = torch.randint(0, len(MIXED_CHOICES), (w.heads,), generator=g)
+    idx = np.random.default_rng(w.seed).integers(0, len(MIXED_CHOICES), size=w.heads)
     return torch.tensor([list(MIXED_CHOICES[i]) for i in idx.tolist()], dtype=torch.int32)
 
 
@@ -80,8 +83,8 @@ def head_factors(w: Workload) -> torch.Tensor | None:
     """Per-head factor f_h ~ U[0.5, 2] (fp32) or None."""
     if not w.head_factors:
         return None
-    g = torch.Generator().manual_seed(w.seed * 7 + 1)
-    return 0.5 + 1.5 * torch.rand(w.heads, generator=g, dtype=torch.float32)
+    f = np.random.default_rng(w.seed * 7 + 1).uniform(0.5, 2.0, size=w.heads)
+    return torch.from_numpy(f.astype(np.float32))
 
 
 def slice_seed(w: Workload, which: int, b: int, h: int) -> int:
@@ -91,8 +94,8 @@ def slice_seed(w: Workload, which: int, b: int, h: int) -> int:
 
 def make_slice(w: Workload, which: int, b: int, h: int) -> torch.Tensor:
     """One ``[N, d]`` bf16 slice (CPU), raster token order."""
-    g = torch.Generator().manual_seed(slice_seed(w, which, b, h))
-    x = torch.randn(w.tokens, w.head_dim, generator=g, dtype=torch.float32)
+    rng = np.random.default_rng(slice_seed(w, which, b, h))
+    x = torch.from_numpy(rng.standard_normal((w.tokens, w.head_dim), dtype=np.float32))
     f = head_factors(w)
     if f is not None:
         x.mul_(float(f[h]))
@@ -109,8 +112,12 @@ def make_qkv(w: Workload, device="cpu", heads=None, batches=None):
     out = [torch.zeros(shape, dtype=torch.bfloat16, device=device) for _ in range(3)]
     hs = range(w.heads) if heads is None else heads
     bs = range(w.batch) if batches is None else batches
-    for which in range(3):
-        for b in bs:
-            for h in hs:
-                out[which][b, h].copy_(make_slice(w, which, b, h))
+    jobs = [(which, b, h) for which in range(3) for b in bs for h in hs]
+
+    def one(job):
+        which, b, h = job
+        out[which][b, h].copy_(make_slice(w, which, b, h))
+
+    with ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1))) as ex:
+        list(ex.map(one, jobs))
     return tuple(out)

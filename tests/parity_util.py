@@ -1,0 +1,86 @@
+"""Shared helpers of the GPU parity tests: sampling, oracle rows, tolerances.
+
+Tolerances (CUDA path vs the fp64 oracle on the same bf16 inputs):
+  O   : |delta| <= 2e-2 + 2^-9 |O_ref| element-wise, and mean |delta| <= 2e-3
+  LSE : |delta| <= 1e-3 * max(|LSE_ref|, 1)
+Plan and permutation results are compared bit-exactly.
+
+The 2e-2 / 2e-3 budget is the stated one.  The outputs are bf16 by
+specification, and rounding an exact value to bf16 alone moves it by up to half
+an ulp, 2^-9 |O|: more than 2e-2 once |O| >= 8 (possible on the workload whose
+heads are scaled by up to 2).  That unavoidable rounding is allowed on top of
+the budget; for |O| < 1 the bound stays within 2.2e-2.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+O_MAX_TOL = 2e-2
+BF16_HALF_ULP_REL = 2.0 ** -9
+O_MEAN_TOL = 2e-3
+LSE_REL_TOL = 1e-3
+
+
+def grid(latent, tile):
+    return [latent[i] // tile[i] for i in range(3)]
+
+
+def sample_tiles(latent, tile, n_random: int, seed: int):
+    """The 8 corner tiles, the centre tile and ``n_random`` seeded random tiles."""
+    n = grid(latent, tile)
+    out = []
+    for a in (0, n[0] - 1):
+        for b in (0, n[1] - 1):
+            for c in (0, n[2] - 1):
+                out.append((a * n[1] + b) * n[2] + c)
+    out.append(((n[0] // 2) * n[1] + n[1] // 2) * n[2] + n[2] // 2)
+    rng = np.random.default_rng(seed)
+    out += rng.integers(0, n[0] * n[1] * n[2], n_random).tolist()
+    return sorted(set(out))
+
+
+def tile_rows(latent, tile, tiles, rows_per_tile: int | None, seed: int):
+    """Raster query tokens of the given tiles; all of them, or a seeded subset
+    that always holds the first and last token of each 128-row block."""
+    vol = tile[0] * tile[1] * tile[2]
+    rng = np.random.default_rng(seed)
+    out = []
+    for t in tiles:
+        toks = oracle.tile_tokens(latent, tile, t)  # raster order == tile-major order
+        if rows_per_tile is None or rows_per_tile >= vol:
+            out.append(toks)
+            continue
+        keep = set()
+        for blk in range(0, vol, 128):
+            keep.update([blk, min(blk + 127, vol - 1)])
+        extra = rng.choice(vol, size=max(0, rows_per_tile - len(keep)), replace=False)
+        keep.update(extra.tolist())
+        out.append(toks[sorted(keep)])
+    return np.concatenate(out)
+
+
+def compare(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: np.ndarray, lse_ref: np.ndarray,
+            what: str = ""):
+    """Assert the tolerances; return (max |dO|, mean |dO|, max relative dLSE)."""
+    o = o_gpu.detach().cpu().to(torch.float64).numpy()
+    lse = lse_gpu.detach().cpu().to(torch.float64).numpy()
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), what
+    do = np.abs(o - o_ref)
+    bound = O_MAX_TOL + BF16_HALF_ULP_REL * np.abs(o_ref)
+    dl = np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1.0)
+    stats = (float(do.max()), float(do.mean()), float(dl.max()))
+    worst = np.unravel_index(int(np.argmax(do - bound)), do.shape)
+    assert np.all(do <= bound), (what, stats, "worst", worst, float(o_ref[worst]), float(o[worst]))
+    assert stats[1] <= O_MEAN_TOL, (what, stats)
+    assert stats[2] <= LSE_REL_TOL, (what, stats)
+    return stats
+
+
+def oracle_rows(q, k, v, latent, tile, windows, scale, bhs, tokens):
+    """Oracle on the cartesian product of (b * H + h) ids and raster tokens."""
+    rows = np.array([(bh, t) for bh in bhs for t in tokens], dtype=np.int64)
+    o, lse = oracle.sta_attention(q, k, v, latent, tile, windows, scale, rows=rows)
+    return rows, o, lse

@@ -1,0 +1,163 @@
+"""Host-side checks of the C-ABI library (no GPU, no compute call).
+
+- the library loads and exports every function ``include/sta.h`` declares;
+- argument validation happens before any launch;
+- the plan's key-tile lists equal the sets derived from the oracle's
+  token-level mask (bit-exact), for every workload geometry and window;
+- the work list covers every (b, h, 128-row block) exactly once.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import sta_inputs
+import sparse_attention_video_sta_b200 as sta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "sta.h")).read()
+    return sorted(set(re.findall(r"^STA_API\s+[\w\s\*]+?\b(sta_\w+)\s*\(", src, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert len(names) >= 10
+    lib = ctypes.CDLL(sta.library_path())
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(sta.EXPORTED_SYMBOLS)
+
+
+def test_status_strings():
+    assert sta.sta_status_string(0) == "STA_OK"
+    assert sta.sta_status_string(4) == "STA_ERR_TIMEOUT"
+    assert sta.sta_status_string(99) == "STA_ERR_UNKNOWN"
+
+
+def _raw_plan_host(latent, tile, batch, heads, windows):
+    lib = sta._lib
+    g = sta._geom(latent, tile)
+    h = ctypes.c_void_p(0)
+    w = (ctypes.c_int32 * (3 * heads))(*[int(x) for win in windows for x in win])
+    st = lib.sta_plan_host(ctypes.byref(g), batch, heads, w, ctypes.byref(h))
+    return st, h
+
+
+def test_plan_argument_validation():
+    INV, UNS = sta.STA_ERR_INVALID_ARG, sta.STA_ERR_UNSUPPORTED
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == 0
+    assert _raw_plan_host((30, 48, 81), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == INV  # latent % tile
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(18, 24, 20)])[0] == INV  # window % tile
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(0, 24, 24)])[0] == INV
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 0, 1, [(18, 24, 24)])[0] == INV
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 0, [])[0] == INV
+    assert _raw_plan_host((30, 48, 80), (3, 8, 8), 1, 1, [(18, 24, 24)])[0] == UNS  # 192 tokens
+    # int32 row-coordinate limit of the kernel's tensor maps
+    assert _raw_plan_host((96, 512, 512), (6, 8, 8), 2, 48, [(18, 24, 24)] * 48)[0] == UNS
+    lib = sta._lib
+    assert lib.sta_plan_host(None, 1, 1, None, None) == INV
+    assert lib.sta_plan_destroy(None) == 0
+
+
+def test_calls_rejected_before_launch():
+    INV = sta.STA_ERR_INVALID_ARG
+    lib = sta._lib
+    g = sta._geom((18, 24, 24), (6, 8, 8))
+    bad = sta._geom((18, 24, 25), (6, 8, 8))
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.sta_tile_reorder(None, p, 1, 128, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_reorder(p, None, 1, 128, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_reorder(p, ctypes.c_void_p((1 << 20) + 64), 1, 128, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_reorder(p, ctypes.c_void_p(1 << 34), 0, 128, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_reorder(p, ctypes.c_void_p(1 << 34), 1, 0, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_unreorder(p, ctypes.c_void_p(1 << 34), 1, 128, ctypes.byref(bad), None) == INV
+    # forward: host-only plan, null / misaligned pointers, bad scale, bad head_dim
+    hp = sta.sta_plan_host((18, 24, 24), (6, 8, 8), 1, 2, [(12, 16, 16)] * 2)
+    a = ctypes.c_void_p(1 << 30)
+    assert lib.sta_forward(hp.handle, a, a, a, a, a, 64, 0.125, None) == INV
+    assert lib.sta_forward(None, a, a, a, a, a, 64, 0.125, None) == INV
+    assert lib.sta_last_device_status(hp.handle, None) == INV
+    assert lib.sta_debug_inject_timeout(1, 0) == INV
+    assert lib.sta_plan_query(hp.handle, 2, 0, None, 0, ctypes.byref(ctypes.c_int32())) == INV
+    assert lib.sta_plan_query(hp.handle, 0, 27, None, 0, ctypes.byref(ctypes.c_int32())) == INV
+    hp.destroy()
+
+
+def oracle_tile_set(latent, tile, window, q_tile):
+    """Key tiles attended by query tile q_tile, read off the oracle's token mask."""
+    toks = oracle.tile_tokens(latent, tile, q_tile)
+    row = oracle.mask_row(latent, tile, window, int(toks[0]))
+    n_tiles = oracle.num_tokens(latent) // (tile[0] * tile[1] * tile[2])
+    out = []
+    for t in range(n_tiles):
+        kt = oracle.tile_tokens(latent, tile, t)
+        blk = row[kt]
+        assert blk.all() or not blk.any()
+        if blk.all():
+            out.append(t)
+    return out
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
+def test_plan_lists_match_oracle_mask(idx):
+    w = sta_inputs.WORKLOADS[idx]
+    wins = sta_inputs.windows(w).tolist()
+    p = sta.sta_plan_host(w.latent, w.tile, w.batch, w.heads, wins)
+    n_tiles = p.tiles_per_head
+    rng = np.random.default_rng(idx)
+    distinct = {}
+    for h, win in enumerate(wins):
+        distinct.setdefault(tuple(win), h)
+    for win, h in distinct.items():
+        tiles = sorted(set([0, n_tiles - 1, n_tiles // 2] + rng.integers(0, n_tiles, 6).tolist()))
+        if n_tiles <= 30:
+            tiles = range(n_tiles)
+        for q in tiles:
+            assert p.query(h, q) == oracle_tile_set(w.latent, w.tile, win, q), (idx, win, q)
+    pairs, items = p.stats()
+    expect = 0
+    vol = w.tile[0] * w.tile[1] * w.tile[2]
+    for win in wins:
+        e = [min(win[i] // w.tile[i], w.latent[i] // w.tile[i]) for i in range(3)]
+        expect += n_tiles * e[0] * e[1] * e[2]
+    assert pairs == expect * w.batch
+    # the pages' 91% sparsity for w=(18,24,24) on the 720p latent
+    if idx == 2:
+        assert pairs == 300 * 27 * 24
+        assert abs(1 - pairs / (24 * 300 * 300) - 0.91) < 1e-12
+    assert items >= w.batch * w.heads * n_tiles * (vol // 128) // 2
+
+
+def test_work_list_covers_every_row_block_once():
+    for latent, tile, heads, batch in [((18, 24, 24), (6, 8, 8), 2, 1), ((12, 16, 16), (4, 8, 8), 3, 2),
+                                       ((6, 16, 16), (2, 8, 8), 1, 1), ((30, 48, 80), (6, 8, 8), 24, 1),
+                                       ((18, 24, 16), (6, 8, 8), 2, 2)]:
+        wins = [tuple(3 * t for t in tile)] * (heads - 1) + [tile]
+        p = sta.sta_plan_host(latent, tile, batch, heads, wins)
+        items = p.work_items()
+        S = (tile[0] * tile[1] * tile[2]) // 128
+        n_tiles = p.tiles_per_head
+        seen = {}
+        lens = []
+        for bh, qa, qb, win in items:
+            h = bh % heads
+            blocks = [qa] + ([qb] if qb >= 0 else [])
+            for r in blocks:
+                assert 0 <= r < n_tiles * S
+                seen[(bh, r)] = seen.get((bh, r), 0) + 1
+            if qb >= 0 and S % 2 == 0:
+                assert qa // S == qb // S  # paired blocks of one tile share K/V
+            lens.append(len(p.query(h, qa // S)))
+            if qb >= 0:
+                assert len(p.query(h, qb // S)) == lens[-1]
+        assert len(seen) == batch * heads * n_tiles * S
+        assert all(c == 1 for c in seen.values())
+        assert lens == sorted(lens, reverse=True)  # longest lists first
+        pairs, n_items = p.stats()
+        assert n_items == len(items)
