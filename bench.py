@@ -52,6 +52,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sta", choices=["sta", "reference"])
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override the head count (small cases for profiling only)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip e2e, full-window, permutation and CPU-baseline legs")
     return ap.parse_args()
@@ -180,7 +182,7 @@ def run_reference(args, w):
     n_grid = [w.latent[i] // w.tile[i] for i in range(3)]
     n_tiles = n_grid[0] * n_grid[1] * n_grid[2]
     vol = w.tile[0] * w.tile[1] * w.tile[2]
-    rows_per_step = 128
+    rows_per_step = w.tile[0] * w.tile[1] * w.tile[2]
     cores = os.cpu_count() or 1
 
     def step(i):
@@ -215,6 +217,9 @@ def run_reference(args, w):
 def main():
     args = parse()
     w = sta_inputs.WORKLOADS[args.workload]
+    if args.heads > 0:
+        import dataclasses
+        w = dataclasses.replace(w, heads=args.heads, name=f"{w.name}_heads{args.heads}")
     if args.impl == "reference":
         return run_reference(args, w)
 
@@ -383,7 +388,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
-        cpu = cpu_baseline(w, n_tiles=2, heads=[0])
+        cpu = cpu_baseline(w, n_tiles=32, heads=[0, 1])
 
     if rank == 0:
         line = {
