@@ -137,6 +137,43 @@ STA_API sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const
                        void* o, float* lse, int32_t head_dim, float softmax_scale,
                        void* stream);
 
+/* STA forward that allocates nothing (this call has no counterpart in the
+ * paper; it exists for deployment).
+ *
+ * sta_plan puts the plan in device memory it allocates with cudaMalloc.  Some
+ * callers cannot do that: a process whose device memory belongs to another
+ * allocator or pool that forbids outside cudaMalloc calls; a service that
+ * reserves all its memory at start-up and allows no allocation, and none of
+ * the device synchronisation cudaMalloc may cause, while it serves; a plugin
+ * host that only hands a library the buffers it is meant to touch.  This call
+ * takes the geometry, batch, heads and per-head windows of sta_plan and the
+ * tensors of sta_forward (same layouts and rules), builds the plan on the host
+ * without heap use, and keeps it in a fixed scratch array compiled into the
+ * library: 4 MiB of device memory on every GPU that loads the library, held
+ * until the process exits.
+ *
+ * Limits: heads <= 1024, and the plan must fit the scratch:
+ *   256 + 16 * work_items + 4 * (n_windows * (tiles + 1) + sum over distinct
+ *   windows of tiles * window_tiles) <= 4 MiB
+ * (the 720p and 42x64x112 workloads of this library use 0.7 and 1.3 MiB).
+ * Larger problems, or heads > 1024, return STA_ERR_UNSUPPORTED before any work.
+ *
+ * Behaviour: the first call on a device looks up the scratch's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any stream
+ * capture.  Each call copies the plan from a static host buffer into the
+ * scratch on `stream` (this also clears the status word) and launches the
+ * forward kernel.  Every call shares the one scratch array: calls whose work
+ * overlaps on the GPU (different streams, or threads enqueueing concurrently)
+ * race and must be serialised by the caller, e.g. by using one stream.  Host
+ * threads are serialised inside the call.  A device-side timeout ends the
+ * kernel cleanly but is not reported by this call (use sta_forward with a plan
+ * and sta_last_device_status to observe it).  Errors: as sta_plan and
+ * sta_forward, UNSUPPORTED beyond the limits, CUDA on a failed copy or launch. */
+STA_API sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int32_t heads,
+                                       const int32_t* window_thw, const void* q, const void* k,
+                                       const void* v, void* o, float* lse, int32_t head_dim,
+                                       float softmax_scale, void* stream);
+
 /* Synchronise `stream`, then report (and clear) the first asynchronous error
  * of work enqueued with this plan: CUDA for a launch or execution fault,
  * TIMEOUT when a device-side wait gave up. */

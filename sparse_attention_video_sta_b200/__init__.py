@@ -25,8 +25,8 @@ import torch
 
 __all__ = [
     "StaError", "Plan", "sta_plan", "sta_plan_host", "sta_tile_reorder", "sta_tile_unreorder",
-    "sta_forward", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
-    "sta_attention", "library_path", "EXPORTED_SYMBOLS",
+    "sta_forward", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string",
+    "sta_debug_inject_timeout", "sta_attention", "library_path", "EXPORTED_SYMBOLS",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -41,8 +41,8 @@ STA_ERR_OOM = 5
 
 EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
-    "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward", "sta_last_device_status",
-    "sta_status_string", "sta_debug_inject_timeout",
+    "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
+    "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
 )
 
 
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "sta_tile_reorder": [vp, vp, i64, i32, G, vp],
         "sta_tile_unreorder": [vp, vp, i64, i32, G, vp],
         "sta_forward": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
+        "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
     }
@@ -278,6 +279,31 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                             ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
                             ctypes.c_void_p(lse.data_ptr()), int(d), float(softmax_scale),
                             _stream(stream)), "sta_forward")
+    return o, lse
+
+
+def sta_forward_noalloc(latent, tile, batch: int, heads: int, windows, q: torch.Tensor,
+                        k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+                        softmax_scale: float, stream=None):
+    """STA forward without any device allocation by the library: the plan is
+    kept in the library's fixed scratch array (see ``include/sta.h``).  Same
+    tile-major tensors as ``sta_forward``; calls must not overlap on the GPU."""
+    B, H = int(batch), int(heads)
+    N = int(latent[0]) * int(latent[1]) * int(latent[2])
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
+        if t.dim() != 4 or tuple(t.shape[:3]) != (B, H, N) or t.shape[3] != q.shape[3]:
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected [{B}, {H}, {N}, d]")
+    if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() \
+            or tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape [{B}, {H}, {N}]")
+    g = _geom(latent, tile)
+    _check(_lib.sta_forward_noalloc(ctypes.byref(g), B, H, _windows(H, windows),
+                                    ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                    ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                    ctypes.c_void_p(lse.data_ptr()), int(q.shape[3]),
+                                    float(softmax_scale), _stream(stream)), "sta_forward_noalloc")
     return o, lse
 
 

@@ -499,4 +499,49 @@ cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, co
     return launch_d<64>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns);
 }
 
+cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void* k, const void* v,
+                               void* o, float* lse, int head_dim, float softmax_scale,
+                               cudaStream_t stream) {
+    const int64_t rows = int64_t(pv.batch) * pv.heads * pv.tiles_per_head * pv.tile_tokens;
+    CUtensorMap mq, mk, mv;
+    cudaError_t e = make_map(&mq, q, rows, head_dim);
+    if (e == cudaSuccess) e = make_map(&mk, k, rows, head_dim);
+    if (e == cudaSuccess) e = make_map(&mv, v, rows, head_dim);
+    if (e != cudaSuccess) return e;
+    FwdParams fp;
+    fp.items = pv.items;
+    fp.n_items = pv.n_items;
+    fp.off = pv.off;
+    fp.ids = pv.ids;
+    fp.tiles_per_head = pv.tiles_per_head;
+    fp.sub_per_tile = pv.sub_per_tile;
+    fp.tile_tokens = pv.tile_tokens;
+    fp.tokens = pv.tiles_per_head * pv.tile_tokens;
+    fp.o = static_cast<__nv_bfloat16*>(o);
+    fp.lse = lse;
+    fp.scale = softmax_scale;
+    fp.scale_log2 = softmax_scale * 1.4426950408889634f;
+    fp.status = pv.status;
+    fp.timeout_ns = pv.timeout_ns;
+    fp.inject = 0;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const int grid = fp.n_items < sms ? fp.n_items : sms;
+    if (grid <= 0) return cudaSuccess;
+    if (head_dim == 128) {
+        e = cudaFuncSetAttribute(sta_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        sta_fwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    } else {
+        e = cudaFuncSetAttribute(sta_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<64>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        sta_fwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace sta

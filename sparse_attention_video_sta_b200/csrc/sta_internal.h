@@ -62,6 +62,23 @@ cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, co
                            void* o, float* lse, int head_dim, float softmax_scale,
                            cudaStream_t stream, int inject_timeout, uint64_t timeout_ns);
 
+// Device-side view of a plan whose arrays live in memory the caller provides
+// (used by the no-allocation entry point, sta_noalloc.cu).
+struct RawPlanView {
+    int32_t batch, heads, tiles_per_head, tile_tokens, sub_per_tile;
+    const WorkItem* items;
+    int32_t n_items;
+    const int32_t* off;
+    const int32_t* ids;
+    uint32_t* status;
+    uint64_t timeout_ns;
+};
+
+// Forward launch from a RawPlanView (sta_forward.cu).  Returns a CUDA error code.
+cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void* k, const void* v,
+                               void* o, float* lse, int head_dim, float softmax_scale,
+                               cudaStream_t stream);
+
 // Permutation launch (sta_permute.cu).  inverse = false: raster -> tile-major.
 cudaError_t launch_permute(const void* src, void* dst, int64_t outer, int32_t row_bytes,
                            const sta_geom& g, bool inverse, cudaStream_t stream);
