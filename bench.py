@@ -147,6 +147,31 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+def workload_config(w, wins, world: int) -> dict:
+    """The ``config`` object both arms print."""
+    return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
+            "latent": list(w.latent), "tile": list(w.tile),
+            "window": list(wins[0]) if w.window else "per-head", "tokens": w.tokens,
+            "parallelism": f"replicas{world}",
+            "l2": "inputs larger than L2 (3 x %.1f MB per step), no flush"
+                  % (w.batch * w.heads * w.tokens * w.head_dim * 2 / 1e6),
+            "step": "reorder Q,K,V + sta_forward + unreorder O,LSE; plan built once"}
+
+
+def max_over_ranks(dist, x: float, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Whole-job throughput: every rank ran flops_per_rank in at most ms."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 def cpu_baseline(w, n_tiles: int, heads):
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
     import oracle
@@ -206,8 +231,7 @@ def run_reference(args, w):
             "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
-                       "latent": list(w.latent), "tile": list(w.tile)},
+            "config": workload_config(w, wins, int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -242,12 +266,8 @@ def main():
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def reduce_max(x: float) -> float:
+        return max_over_ranks(dist, x, dev)
 
     # ---------------------------------------------------------------- inputs
     B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
@@ -310,13 +330,13 @@ def main():
     clocks = sampler.stop() if sampler else None
     ms_local = start.elapsed_time(stop) / args.steps
     fwd_ms_local = statistics.mean(a.elapsed_time(b) for a, b in ev_fwd)
-    ms = max_over_ranks(ms_local)
-    fwd_ms = max_over_ranks(fwd_ms_local)
+    ms = reduce_max(ms_local)
+    fwd_ms = reduce_max(fwd_ms_local)
     status = sta.sta_last_device_status(plan)
     if status != 0:
         raise RuntimeError(f"device status {sta.sta_status_string(status)} after timing")
 
-    value = world * flops / (ms * 1e-3) / 1e12
+    value = weak_scaling_tflops(world, flops, ms)
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -336,7 +356,7 @@ def main():
             sta.sta_forward(full, qt, kt, vt, ot, lset, scale)
         e1.record()
         torch.cuda.synchronize()
-        full_ms = max_over_ranks(e0.elapsed_time(e1) / reps)
+        full_ms = reduce_max(e0.elapsed_time(e1) / reps)
         ideal = full.stats()[0] / plan.stats()[0]
         extras["full_window"] = {"ms": full_ms, "tflops": full.flops(d) / (full_ms * 1e-3) / 1e12,
                                  "speedup": full_ms / fwd_ms, "ideal_speedup": ideal,
@@ -381,8 +401,8 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps)
+        e2e = {"value": weak_scaling_tflops(world, flops, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * nbytes,
                "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size()}
 
@@ -395,11 +415,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": B, "heads": H, "head_dim": d, "latent": list(L),
-                       "tile": list(T), "window": wins[0] if w.window else "per-head",
-                       "tokens": N, "parallelism": f"replicas{world}",
-                       "l2": "inputs larger than L2 (3 x %.1f MB per step), no flush" % (q.numel() * 2 / 1e6),
-                       "step": "reorder Q,K,V + sta_forward + unreorder O,LSE; plan built once"},
+            "config": workload_config(w, wins, world),
             "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak, "traffic": measured_traffic(),

@@ -1,0 +1,65 @@
+"""Multi-process host logic of bench.py on CPU (gloo, world size 2).
+
+The STA path shards by (batch, head) with no data exchange, so the only
+cross-rank logic is the timing reduction (max over ranks) and the whole-job
+throughput of weak scaling; the reference arm runs on rank 0 only.
+"""
+import datetime
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, queue):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        ms = bench.max_over_ranks(dist, 10.0 + rank, torch.device("cpu"))
+        value = bench.weak_scaling_tflops(world, 1.0e12, ms)
+        dist.barrier()
+        queue.put((rank, ms, value))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_take_the_max_time_and_sum_the_work():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, queue)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(queue.get(timeout=10) for _ in range(2))
+    for rank, ms, value in got:
+        assert ms == 11.0
+        assert value == pytest.approx(2 * 1.0e12 / 0.011 / 1e12)
+
+
+def test_reference_arm_exits_quietly_on_other_ranks():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
