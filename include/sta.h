@@ -179,6 +179,11 @@ STA_API sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int32_t
  * TIMEOUT when a device-side wait gave up. */
 STA_API sta_status sta_last_device_status(sta_plan_t p, void* stream);
 
+/* Name and text of the last CUDA error met by a libsta call in the calling
+ * thread (e.g. "cudaErrorLaunchOutOfResources: ..."), or "no error".  The
+ * string stays valid until the thread's next failing call. */
+STA_API const char* sta_last_error_detail(void);
+
 /* Static string naming a status code. */
 STA_API const char* sta_status_string(sta_status s);
 

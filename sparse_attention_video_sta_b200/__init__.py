@@ -43,6 +43,7 @@ EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
     "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
+    "sta_last_error_detail",
 )
 
 
@@ -80,6 +81,8 @@ def _load() -> ctypes.CDLL:
         f.restype = ctypes.c_int
     L.sta_status_string.argtypes = [ctypes.c_int]
     L.sta_status_string.restype = ctypes.c_char_p
+    L.sta_last_error_detail.argtypes = []
+    L.sta_last_error_detail.restype = ctypes.c_char_p
     return L
 
 
@@ -94,10 +97,17 @@ def sta_status_string(status: int) -> str:
     return _lib.sta_status_string(int(status)).decode()
 
 
+def sta_last_error_detail() -> str:
+    return _lib.sta_last_error_detail().decode()
+
+
 class StaError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = int(status)
-        super().__init__(f"{what}: {sta_status_string(status)}")
+        msg = f"{what}: {sta_status_string(status)}"
+        if self.status in (STA_ERR_CUDA, STA_ERR_OOM):
+            msg += f" ({sta_last_error_detail()})"
+        super().__init__(msg)
 
 
 def _check(status: int, what: str) -> None:

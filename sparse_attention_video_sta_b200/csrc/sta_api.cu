@@ -12,6 +12,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <map>
 #include <new>
@@ -30,6 +31,15 @@ std::atomic<int> g_inject_timeout{0};
 std::atomic<int> g_inject_limit_ms{50};
 
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;  // 2 s per device-side wait
+
+// Name and text of the last CUDA error this library saw in the calling thread.
+thread_local char g_detail[256] = "no error";
+
+sta_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return STA_OK;
+    snprintf(g_detail, sizeof g_detail, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? STA_ERR_OOM : STA_ERR_CUDA;
+}
 
 bool geom_valid(const sta_geom* g) {
     if (g == nullptr) return false;
@@ -180,9 +190,8 @@ sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row
     const int64_t bytes = outer * n_tok * int64_t(row_bytes);
     const uintptr_t s = reinterpret_cast<uintptr_t>(src), d = reinterpret_cast<uintptr_t>(dst);
     if (s < d + uint64_t(bytes) && d < s + uint64_t(bytes)) return STA_ERR_INVALID_ARG;  // overlap
-    cudaError_t e = sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
-                                        static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+    return cuda_status(sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -235,12 +244,12 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) {
-        const bool oom = (e == cudaErrorMemoryAllocation);
+        const sta_status st = cuda_status(e);
         cudaGetLastError();
         free_device(p);
         delete p;
         *out = nullptr;
-        return oom ? STA_ERR_OOM : STA_ERR_CUDA;
+        return st;
     }
     p->on_device = true;
     return STA_OK;
@@ -314,28 +323,31 @@ sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v
     if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess) return STA_ERR_CUDA;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
     if (dev != p->device) return STA_ERR_INVALID_ARG;
     const int inject = g_inject_timeout.load();
     const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
                                   : kDefaultTimeoutNs;
-    cudaError_t e = sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
-                                        static_cast<cudaStream_t>(stream), inject, limit);
-    return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
+    return cuda_status(sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
+                                           static_cast<cudaStream_t>(stream), inject, limit));
 }
 
 sta_status sta_last_device_status(sta_plan_t p, void* stream) {
     if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return STA_ERR_CUDA;
-    if (cudaGetLastError() != cudaSuccess) return STA_ERR_CUDA;
+    if (cudaError_t e = cudaStreamSynchronize(s); e != cudaSuccess) return cuda_status(e);
+    if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_status(e);
     uint32_t word = 0;
-    if (cudaMemcpy(&word, p->d_status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
-        return STA_ERR_CUDA;
-    if (word != 0 && cudaMemset(p->d_status, 0, sizeof word) != cudaSuccess) return STA_ERR_CUDA;
+    if (cudaError_t e = cudaMemcpy(&word, p->d_status, sizeof word, cudaMemcpyDeviceToHost); e != cudaSuccess)
+        return cuda_status(e);
+    if (word != 0) {
+        if (cudaError_t e = cudaMemset(p->d_status, 0, sizeof word); e != cudaSuccess) return cuda_status(e);
+    }
     if (word & sta::kDevTimeout) return STA_ERR_TIMEOUT;
     return STA_OK;
 }
+
+const char* sta_last_error_detail(void) { return g_detail; }
 
 sta_status sta_debug_inject_timeout(int32_t enable, int32_t limit_ms) {
     if (limit_ms < 1 || limit_ms > 10000) return STA_ERR_INVALID_ARG;

@@ -10,22 +10,26 @@
 // (same transcript, segment on ThunderKittens); the design below keeps that
 // split but is built for Blackwell:
 //
-//   warp 8 (load)    : TMA loads of the query blocks and of 128-key K / V chunks
-//                      of the listed key tiles into a ring of shared-memory stages
-//   warp 9 (MMA)     : one thread issues tcgen05.mma: S = Q K^T into TMEM, then
-//                      O += P V with P read straight from TMEM
-//   warps 0-3, 4-7   : softmax for query slot 0 / 1: tcgen05.ld of S, online
-//                      softmax (fp32 running max / sum, exp2 with the scale folded
-//                      in, lazy rescale of O), bf16 P written back into TMEM over
-//                      S, and the epilogue O / l -> bf16, LSE
+//   warp 8 (load)      : TMA loads of the query blocks and of the 128-key K / V
+//                        chunks of the listed key tiles into a ring of stages
+//   warps 9, 10 (MMA)  : one thread each, for query slot 0 / 1, issues
+//                        tcgen05.mma: S = Q K^T into TMEM, then O += P V with P
+//                        read straight from TMEM.  A tcgen05.mma issue does not
+//                        return before the tensor pipe takes the instruction,
+//                        so a single issuing thread leaves the pipe idle
+//                        whenever it waits; two independent issuers keep it fed.
+//   warps 0-3, 4-7     : softmax for query slot 0 / 1 (one thread per row):
+//                        tcgen05.ld of S, online softmax (fp32 running max and
+//                        sum, exp2 with the scale folded in, lazy rescale of O),
+//                        bf16 P written back into TMEM over S, and the epilogue
+//                        O / l -> bf16, LSE
 //
 // A work item is up to two 128-row query blocks (slots) of one (b, h).  Blocks of
-// the same tile share every K/V chunk; the two slots ping-pong so the tensor core
-// computes one slot's S while the other slot's softmax runs.  TMEM (512 columns):
-// S0 | S1 | O0 | O1.  The kernel is persistent (one CTA per SM) over the plan's
-// work list, longest key lists first.  Every mbarrier wait has a time limit; on
-// expiry the kernel records STA timeout status, drains its copies and MMAs, frees
-// TMEM and exits.
+// the same tile share every K/V chunk load.  TMEM (512 columns): S0 | S1 | O0 |
+// O1.  The kernel is persistent (one CTA per SM) over the plan's work list,
+// longest key lists first.  Every mbarrier wait has a time limit; on expiry the
+// kernel records STA timeout status, drains its copies and MMAs, frees TMEM and
+// exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
@@ -40,11 +44,13 @@
 namespace sta {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp0 = 9;  // slot 0 issuer; also allocates TMEM.  Slot 1 issuer: warp 10.
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+constexpr int kStagesD128 = 5;  // K/V ring stages of 32 KB at d = 128 (8 of 16 KB at d = 64)
 
 template <int D>
 struct Cfg {
@@ -52,13 +58,13 @@ struct Cfg {
     static constexpr int kBoxBytes = 128 * 128;           // one TMA box: 128 rows x 128 bytes
     static constexpr int kQBytes = kSubRows * D * 2;      // one 128-row query block
     static constexpr int kKVBytes = kChunkKeys * D * 2;   // one 128-key K or V chunk
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kStages = (D == 128) ? kStagesD128 : 8;
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = 2 * kQBytes;
     static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
-    // barriers: full[S], empty[S], q_full, q_empty, s_full[2], p_full[2], o_full[2],
-    // o_empty[2], dead, drain
-    static constexpr int kNumBars = 2 * kStages + 12;
+    // barriers: full[S], empty[S][2], q_full[2], q_empty[2], s_full[2], p_full[2],
+    // o_full[2], o_empty[2], dead, drain[2], turn[2]
+    static constexpr int kNumBars = 3 * kStages + 17;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot + abort flag
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
     // TMEM columns: S0 | S1 | O0 | O1
@@ -66,6 +72,7 @@ struct Cfg {
     __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256u + uint32_t(slot) * D; }
     static_assert(256 + 2 * D <= int(kTmemCols), "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    static_assert(kStages <= 16, "ring bookkeeping uses 2 bits per stage in a uint32");
 };
 
 struct FwdParams {
@@ -112,6 +119,56 @@ __device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_
     }
 }
 
+// P = exp2(S * c - m * c) for one 128-score row, packed to bf16 pairs; returns
+// the fp32 row sum.  With kTrack it also returns the row max of S in `mx`.
+template <bool kTrack>
+__device__ __forceinline__ float softmax_exp(const uint32_t (&sr)[128], float c, float m,
+                                             uint32_t (&pk)[64], float& mx) {
+    const uint64_t c2 = ptx::f2(c, c);
+    const uint64_t nmc2 = ptx::f2(-m * c, -m * c);
+    uint64_t acc0 = ptx::f2(0.0f, 0.0f), acc1 = acc0;
+    float a0 = __int_as_float(0xff800000), a1 = a0;
+#pragma unroll
+    for (int j = 0; j < 64; ++j) {
+        const float s0 = __uint_as_float(sr[2 * j]), s1 = __uint_as_float(sr[2 * j + 1]);
+        if (kTrack) {
+            if (j & 1)
+                a1 = ptx::max3(a1, s0, s1);
+            else
+                a0 = ptx::max3(a0, s0, s1);
+        }
+        float x0, x1, p0, p1;
+        ptx::f2_split(ptx::f2_fma(ptx::f2(s0, s1), c2, nmc2), x0, x1);
+        p0 = ptx::ex2(x0);
+        p1 = ptx::ex2(x1);
+        if (j & 1)
+            acc1 = ptx::f2_add(acc1, ptx::f2(p0, p1));
+        else
+            acc0 = ptx::f2_add(acc0, ptx::f2(p0, p1));
+        pk[j] = ptx::pack_bf16x2(p0, p1);
+    }
+    if (kTrack) mx = fmaxf(a0, a1);
+    float r0, r1, r2, r3;
+    ptx::f2_split(acc0, r0, r1);
+    ptx::f2_split(acc1, r2, r3);
+    return (r0 + r1) + (r2 + r3);
+}
+
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[128]) {
+    float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
+    float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
+#pragma unroll
+    for (int j = 4; j < 124; j += 8) {
+        a0 = ptx::max3(a0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+        a1 = ptx::max3(a1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+        a2 = ptx::max3(a2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+        a3 = ptx::max3(a3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+    }
+    a0 = ptx::max3(a0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
+    a1 = ptx::max3(a1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
+    return ptx::max3(a0, a1, fmaxf(a2, a3));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -126,44 +183,50 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int lane = threadIdx.x & 31;
 
     const uint32_t bar0 = base + C::kBarOff;
-    auto bar_full = [&](int s) { return bar0 + 8u * s; };
-    auto bar_empty = [&](int s) { return bar0 + 8u * (C::kStages + s); };
-    const uint32_t bar_q_full = bar0 + 8u * (2 * C::kStages + 0);
-    const uint32_t bar_q_empty = bar0 + 8u * (2 * C::kStages + 1);
-    auto bar_s_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 2 + j); };
-    auto bar_p_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 4 + j); };
-    auto bar_o_full = [&](int j) { return bar0 + 8u * (2 * C::kStages + 6 + j); };
-    auto bar_o_empty = [&](int j) { return bar0 + 8u * (2 * C::kStages + 8 + j); };
-    const uint32_t bar_dead = bar0 + 8u * (2 * C::kStages + 10);
-    const uint32_t bar_drain = bar0 + 8u * (2 * C::kStages + 11);
+    constexpr int S = C::kStages;
+    auto bar_full = [&](int r) { return bar0 + 8u * r; };
+    auto bar_empty = [&](int r, int s) { return bar0 + 8u * (S + 2 * r + s); };
+    auto bar_q_full = [&](int s) { return bar0 + 8u * (3 * S + 0 + s); };
+    auto bar_q_empty = [&](int s) { return bar0 + 8u * (3 * S + 2 + s); };
+    auto bar_s_full = [&](int s) { return bar0 + 8u * (3 * S + 4 + s); };
+    auto bar_p_full = [&](int s) { return bar0 + 8u * (3 * S + 6 + s); };
+    auto bar_o_full = [&](int s) { return bar0 + 8u * (3 * S + 8 + s); };
+    auto bar_o_empty = [&](int s) { return bar0 + 8u * (3 * S + 10 + s); };
+    const uint32_t bar_dead = bar0 + 8u * (3 * S + 12);
+    auto bar_drain = [&](int s) { return bar0 + 8u * (3 * S + 13 + s); };
+    auto bar_turn = [&](int s) { return bar0 + 8u * (3 * S + 15 + s); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            ptx::mbar_init(bar_full(s), 1);
-            ptx::mbar_init(bar_empty(s), 1);
+        for (int r = 0; r < S; ++r) {
+            ptx::mbar_init(bar_full(r), 1);
+            ptx::mbar_init(bar_empty(r, 0), 1);
+            ptx::mbar_init(bar_empty(r, 1), 1);
         }
-        ptx::mbar_init(bar_q_full, 1);
-        ptx::mbar_init(bar_q_empty, 1);
-        for (int j = 0; j < 2; ++j) {
-            ptx::mbar_init(bar_s_full(j), 1);
-            ptx::mbar_init(bar_p_full(j), 128);
-            ptx::mbar_init(bar_o_full(j), 1);
-            ptx::mbar_init(bar_o_empty(j), 128);
+        for (int s = 0; s < 2; ++s) {
+            ptx::mbar_init(bar_q_full(s), 1);
+            ptx::mbar_init(bar_q_empty(s), 1);
+            ptx::mbar_init(bar_s_full(s), 1);
+            ptx::mbar_init(bar_p_full(s), 4);  // one arrival per softmax warp
+            ptx::mbar_init(bar_o_full(s), 1);
+            ptx::mbar_init(bar_o_empty(s), 4);
+            ptx::mbar_init(bar_drain(s), 1);
         }
         ptx::mbar_init(bar_dead, 1);
-        ptx::mbar_init(bar_drain, 1);
+        ptx::mbar_init(bar_turn(0), 1);
+        ptx::mbar_init(bar_turn(1), 1);
         *abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive(bar_turn(0));  // slot 0 issues first
     }
     if (warp == kLoadWarp && lane == 0) {
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
         ptx::prefetch_tensormap(&tm_v);
     }
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -177,25 +240,35 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (warp == kLoadWarp) {
         if (lane == 0) {
             // ------------------------------------------------------------ load
-            uint32_t item = 0, unit_n = 0;
+            // Ring stage r holds one K or V chunk.  `users` keeps, 2 bits per
+            // stage, which issuers read the chunk now in it; `upar` keeps, per
+            // (stage, issuer), the parity of that issuer's uses of the stage.
+            // Before refilling a stage the previous readers' release is awaited.
+            uint32_t item = 0, qc0 = 0, qc1 = 0, users = 0, upar = 0;
             bool ok = true;
             if (p.inject) {
                 // Debug: wait on a barrier nothing arrives at; the limit runs out.
                 ok = wait_bar(bar_dead, 0, abort_flag, p);
             }
-            auto issue = [&](const CUtensorMap* m, int32_t row) -> bool {
-                const int slot = int(item % C::kStages);
-                const uint32_t phase = item / C::kStages;
-                if (!wait_bar(bar_empty(slot), (phase & 1u) ^ 1u, abort_flag, p)) return false;
-                const uint32_t dst = base + C::kRingOff + slot * C::kKVBytes;
-                ptx::mbar_arrive_expect_tx(bar_full(slot), C::kKVBytes);
+            auto issue = [&](const CUtensorMap* m, int32_t row, uint32_t mask) -> bool {
+                const int r = int(item % S);
+                const uint32_t prev = (users >> (2 * r)) & 3u;
+#pragma unroll
+                for (int s = 0; s < 2; ++s)
+                    if ((prev >> s) & 1u)
+                        if (!wait_bar(bar_empty(r, s), ((upar >> (2 * r + s)) & 1u) ^ 1u, abort_flag, p))
+                            return false;
+                users = (users & ~(3u << (2 * r))) | (mask << (2 * r));
+                upar ^= mask << (2 * r);
+                const uint32_t dst = base + C::kRingOff + r * C::kKVBytes;
+                ptx::mbar_arrive_expect_tx(bar_full(r), C::kKVBytes);
 #pragma unroll
                 for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    ptx::tma_load_2d(dst + cb * C::kBoxBytes, m, bar_full(slot), cb * 64, row);
+                    ptx::tma_load_2d(dst + cb * C::kBoxBytes, m, bar_full(r), cb * 64, row);
                 ++item;
                 return true;
             };
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x, ++unit_n) {
+            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
                 const WorkItem w = p.items[u];
                 const bool has_b = w.qb >= 0;
                 const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
@@ -205,45 +278,55 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int32_t* list_b = p.ids + off[tile_b];
                 const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
                 const int32_t head_row = w.bh * p.tokens;
-                // query blocks
-                if (!wait_bar(bar_q_empty, (unit_n & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                ptx::mbar_arrive_expect_tx(bar_q_full, (has_b ? 2 : 1) * C::kQBytes);
+                // query blocks, one buffer per slot
+                if (!wait_bar(bar_q_empty(0), (qc0 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
+                ptx::mbar_arrive_expect_tx(bar_q_full(0), C::kQBytes);
 #pragma unroll
                 for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    ptx::tma_load_2d(base + C::kQOff + cb * C::kBoxBytes, &tm_q, bar_q_full, cb * 64,
+                    ptx::tma_load_2d(base + C::kQOff + cb * C::kBoxBytes, &tm_q, bar_q_full(0), cb * 64,
                                      head_row + w.qa * kSubRows);
+                ++qc0;
                 if (has_b) {
+                    if (!wait_bar(bar_q_empty(1), (qc1 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(bar_q_full(1), C::kQBytes);
 #pragma unroll
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         ptx::tma_load_2d(base + C::kQOff + C::kQBytes + cb * C::kBoxBytes, &tm_q,
-                                         bar_q_full, cb * 64, head_row + w.qb * kSubRows);
+                                         bar_q_full(1), cb * 64, head_row + w.qb * kSubRows);
+                    ++qc1;
                 }
-                // K / V chunks in the order the MMA warp consumes them
+                // K / V chunks in the order the issuers consume them
+                const uint32_t both = has_b ? 3u : 1u;
                 for (int32_t i = 0; ok && i < n_chunks; ++i) {
                     const int32_t kt = i / SPT, kc = i - kt * SPT;
                     const int32_t row_a = head_row + list_a[kt] * p.tile_tokens + kc * kChunkKeys;
                     const int32_t row_b = head_row + list_b[kt] * p.tile_tokens + kc * kChunkKeys;
-                    ok = issue(&tm_k, row_a);
-                    if (ok && split) ok = issue(&tm_k, row_b);
-                    if (ok) ok = issue(&tm_v, row_a);
-                    if (ok && split) ok = issue(&tm_v, row_b);
+                    if (split) {
+                        ok = issue(&tm_k, row_a, 1u) && issue(&tm_k, row_b, 2u) && issue(&tm_v, row_a, 1u) &&
+                             issue(&tm_v, row_b, 2u);
+                    } else {
+                        ok = issue(&tm_k, row_a, both) && issue(&tm_v, row_a, both);
+                    }
                 }
             }
-            // Drain: the copies issued last into each stage, and the last query load.
-            const uint32_t first = item > uint32_t(C::kStages) ? item - C::kStages : 0u;
+            // Drain: the copies issued last into each stage, and the last query loads.
+            const uint32_t first = item > uint32_t(S) ? item - S : 0u;
             for (uint32_t it = first; it < item; ++it)
-                drain_bar(bar_full(int(it % C::kStages)), (it / C::kStages) & 1u, p.timeout_ns);
-            if (unit_n > 0) drain_bar(bar_q_full, (unit_n - 1) & 1u, p.timeout_ns);
+                drain_bar(bar_full(int(it % S)), (it / S) & 1u, p.timeout_ns);
+            if (qc0 > 0) drain_bar(bar_q_full(0), (qc0 - 1) & 1u, p.timeout_ns);
+            if (qc1 > 0) drain_bar(bar_q_full(1), (qc1 - 1) & 1u, p.timeout_ns);
         }
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
         if (lane == 0) {
             // ------------------------------------------------------------- MMA
+            const int s = warp - kMmaWarp0;  // the query slot this thread serves
             constexpr uint32_t idesc_qk = ptx::idesc_bf16(128, kChunkKeys, false);
             constexpr uint32_t idesc_pv = ptx::idesc_bf16(128, D, true);
-            uint32_t item = 0, unit_n = 0;
-            uint32_t pcnt[2] = {0, 0}, ocnt[2] = {0, 0};
+            const uint32_t tS = tmem + C::col_s(s), tO = tmem + C::col_o(s);
+            const uint32_t qaddr = base + C::kQOff + s * C::kQBytes;
+            uint32_t item = 0, qc = 0, pc = 0, oc = 0, tc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x, ++unit_n) {
+            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
                 const WorkItem w = p.items[u];
                 const bool has_b = w.qb >= 0;
                 const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
@@ -251,65 +334,74 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
                 const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
                 const uint32_t width = split ? 4u : 2u;
-                const int n_slots = has_b ? 2 : 1;
                 const uint32_t ubase = item;
-                if (!wait_bar(bar_q_full, unit_n & 1u, abort_flag, p)) { ok = false; break; }
+                item += uint32_t(n_chunks) * width;
+                if (s == 1 && !has_b) continue;
+                // ring positions: step i holds [K, V] (shared) or [K_a, K_b, V_a, V_b]
+                const uint32_t k_off = split ? uint32_t(s) : 0u, v_off = split ? 2u + uint32_t(s) : 1u;
+                if (!wait_bar(bar_q_full(s), qc & 1u, abort_flag, p)) { ok = false; break; }
                 ptx::tc_fence_after();
+                // With both slots busy the issuers take turns, one step's batch
+                // [PV_s(i-1), S_s(i)] each: the tensor pipe then runs slot 1's
+                // batch while slot 0's softmax works and the other way round.
+                // Each issuer finishes its own waits before it waits for the turn.
+                const bool turns = has_b;
                 for (int32_t i = 0; ok && i <= n_chunks; ++i) {
-                    for (int s = 0; ok && s < n_slots; ++s) {
-                        const bool last_slot = (s == n_slots - 1);
-                        const uint32_t k_it = ubase + uint32_t(i) * width + (split ? uint32_t(s) : 0u);
-                        const uint32_t v_it =
-                            ubase + uint32_t(i - 1) * width + (split ? 2u + uint32_t(s) : 1u);
-                        if (i >= 1) {
-                            // O_s += P_s(i-1) V(i-1)
-                            if (!wait_bar(bar_p_full(s), pcnt[s] & 1u, abort_flag, p)) { ok = false; break; }
-                            ++pcnt[s];
-                            if (!wait_bar(bar_full(int(v_it % C::kStages)), (v_it / C::kStages) & 1u,
-                                          abort_flag, p)) { ok = false; break; }
-                            if (i == 1 && !wait_bar(bar_o_empty(s), (ocnt[s] & 1u) ^ 1u, abort_flag, p)) {
-                                ok = false;
-                                break;
-                            }
-                            ptx::tc_fence_after();
-                            const uint32_t vaddr = base + C::kRingOff + (v_it % C::kStages) * C::kKVBytes;
+                    const uint32_t v_it = ubase + uint32_t(i - 1) * width + v_off;
+                    const uint32_t k_it = ubase + uint32_t(i) * width + k_off;
+                    // Stage and O waits first: they are normally satisfied while this
+                    // slot's softmax still runs, so only the P wait gates the batch.
+                    if (i < n_chunks && !wait_bar(bar_full(int(k_it % S)), (k_it / S) & 1u, abort_flag, p)) {
+                        ok = false;
+                        break;
+                    }
+                    if (i >= 1) {
+                        if (!wait_bar(bar_full(int(v_it % S)), (v_it / S) & 1u, abort_flag, p)) { ok = false; break; }
+                        if (i == 1 && !wait_bar(bar_o_empty(s), (oc & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
+                        if (!wait_bar(bar_p_full(s), pc & 1u, abort_flag, p)) { ok = false; break; }
+                        ++pc;
+                    }
+                    if (turns) {
+                        if (!wait_bar(bar_turn(s), tc & 1u, abort_flag, p)) { ok = false; break; }
+                        ++tc;
+                    }
+                    ptx::tc_fence_after();
+                    if (i >= 1) {
+                        // O_s += P_s(i-1) V(i-1)
+                        const uint32_t vaddr = base + C::kRingOff + (v_it % S) * C::kKVBytes;
 #pragma unroll
-                            for (int kk = 0; kk < kChunkKeys / 16; ++kk) {
-                                const uint64_t bdesc = ptx::desc_mn_sw128(vaddr + kk * 16 * 128, C::kBoxBytes);
-                                ptx::mma_ts(tmem + C::col_o(s), tmem + C::col_s(s) + kk * 8, bdesc, idesc_pv,
-                                            (i > 1 || kk > 0) ? 1u : 0u);
-                            }
-                        }
-                        if (i < n_chunks) {
-                            // S_s(i) = Q_s K(i)^T
-                            if (!wait_bar(bar_full(int(k_it % C::kStages)), (k_it / C::kStages) & 1u,
-                                          abort_flag, p)) { ok = false; break; }
-                            ptx::tc_fence_after();
-                            const uint32_t qaddr = base + C::kQOff + s * C::kQBytes;
-                            const uint32_t kaddr = base + C::kRingOff + (k_it % C::kStages) * C::kKVBytes;
+                        for (int kk = 0; kk < kChunkKeys / 16; ++kk)
+                            ptx::mma_ts(tO, tS + kk * 8, ptx::desc_mn_sw128(vaddr + kk * 16 * 128, C::kBoxBytes),
+                                        idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
+                    }
+                    if (i < n_chunks) {
+                        // S_s(i) = Q_s K(i)^T; in issue order after PV_s(i-1), which
+                        // reads the P that this S overwrites
+                        const uint32_t kaddr = base + C::kRingOff + (k_it % S) * C::kKVBytes;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                const uint32_t coff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-                                ptx::mma_ss(tmem + C::col_s(s), ptx::desc_k_sw128(qaddr + coff),
-                                            ptx::desc_k_sw128(kaddr + coff), idesc_qk, kk > 0 ? 1u : 0u);
-                            }
-                            ptx::mma_commit(bar_s_full(s));
-                        } else {
-                            ptx::mma_commit(bar_o_full(s));
-                            ++ocnt[s];
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t coff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
+                            ptx::mma_ss(tS, ptx::desc_k_sw128(qaddr + coff), ptx::desc_k_sw128(kaddr + coff),
+                                        idesc_qk, kk > 0 ? 1u : 0u);
                         }
-                        if (i >= 1 && (split || last_slot)) ptx::mma_commit(bar_empty(int(v_it % C::kStages)));
-                        if (i < n_chunks && (split || last_slot))
-                            ptx::mma_commit(bar_empty(int(k_it % C::kStages)));
+                    }
+                    if (turns) ptx::mbar_arrive(bar_turn(1 - s));
+                    if (i < n_chunks) ptx::mma_commit(bar_s_full(s));
+                    if (i >= 1) ptx::mma_commit(bar_empty(int(v_it % S), s));
+                    if (i < n_chunks) {
+                        ptx::mma_commit(bar_empty(int(k_it % S), s));
+                    } else {
+                        ptx::mma_commit(bar_o_full(s));
+                        ++oc;
                     }
                 }
                 if (!ok) break;
-                ptx::mma_commit(bar_q_empty);
-                item = ubase + uint32_t(n_chunks) * width;
+                ptx::mma_commit(bar_q_empty(s));
+                ++qc;
             }
-            // Drain: every MMA issued so far completes before TMEM is freed.
-            ptx::mma_commit(bar_drain);
-            drain_bar(bar_drain, 0, p.timeout_ns);
+            // Drain: every MMA this thread issued completes before TMEM is freed.
+            ptx::mma_commit(bar_drain(s));
+            drain_bar(bar_drain(s), 0, p.timeout_ns);
         }
     } else {
         // ------------------------------------------------------------- softmax
@@ -336,46 +428,61 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 ++scnt;
                 ptx::tc_fence_after();
+                float rowsum;
+                bool rescale = false;
+                float alpha = 1.0f;
+                float mx;
                 uint32_t sr[128];
                 ptx::tmem_ld128(tS, sr);
-                float mx = __uint_as_float(sr[0]);
-#pragma unroll
-                for (int j = 1; j < 128; ++j) mx = fmaxf(mx, __uint_as_float(sr[j]));
+                uint32_t pk[64];
                 if (i == 0) {
-                    m_used = mx;
+                    m_used = row_max(sr);
+                    rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
                 } else {
+                    // Exponentiate against the running max while finding this
+                    // chunk's max; only a row whose max grew by more than 2^8 is
+                    // redone (rarely) against its new max (lazy rescale).
+                    rowsum = softmax_exp<true>(sr, c, m_used, pk, mx);
                     const bool need = (mx - m_used) * c > kRescaleThreshold;
-                    if (__any_sync(0xffffffffu, need)) {
-                        const float m_new = need ? mx : m_used;
-                        const float alpha = ptx::ex2((m_used - m_new) * c);
-#pragma unroll 1
-                        for (int cb = 0; cb < D / 32; ++cb) {
-                            uint32_t orr[32];
-                            ptx::tmem_ld32(tO + cb * 32, orr);
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) orr[j] = __float_as_uint(__uint_as_float(orr[j]) * alpha);
-                            ptx::tmem_st32(tO + cb * 32, orr);
+                    rescale = __any_sync(0xffffffffu, need);
+                    if (rescale) {
+                        if (need) {
+                            alpha = ptx::ex2((m_used - mx) * c);
+                            m_used = mx;
                         }
-                        ptx::tmem_wait_st();
-                        l *= alpha;
-                        m_used = m_new;
+                        // S is still in TMEM (P has not been written over it yet)
+                        ptx::tmem_ld128(tS, sr);
+                        rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
                     }
                 }
-                const float mc = m_used * c;
-                float rowsum = 0.0f;
-                uint32_t pk[64];
-#pragma unroll
-                for (int j = 0; j < 64; ++j) {
-                    const float p0 = ptx::ex2(fmaf(__uint_as_float(sr[2 * j]), c, -mc));
-                    const float p1 = ptx::ex2(fmaf(__uint_as_float(sr[2 * j + 1]), c, -mc));
-                    rowsum += p0 + p1;
-                    pk[j] = ptx::pack_bf16x2(p0, p1);
-                }
                 ptx::tmem_st64(tS, pk);
+                l = l * alpha + rowsum;
+                if (rescale) {
+                    // O_s holds P(0..i-1) V: PV_s(i-1) completed before S_s(i) was
+                    // signalled, and PV_s(i) waits for this warpgroup's P signal.
+                    const uint64_t alpha2 = ptx::f2(alpha, alpha);
+#pragma unroll 1
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        uint32_t orr[32];
+                        ptx::tmem_ld32(tO + cb * 32, orr);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            float o0, o1;
+                            ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(orr[2 * j]),
+                                                              __uint_as_float(orr[2 * j + 1])), alpha2),
+                                          o0, o1);
+                            orr[2 * j] = __float_as_uint(o0);
+                            orr[2 * j + 1] = __float_as_uint(o1);
+                        }
+                        ptx::tmem_st32(tO + cb * 32, orr);
+                    }
+                }
                 ptx::tmem_wait_st();
-                l += rowsum;
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(bar_p_full(slot));
+                // One arrival per warp: 128 arrivals on one barrier serialise
+                // for hundreds of cycles on the critical path.
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(bar_p_full(slot));
             }
             if (!ok) break;
             // epilogue: O / l -> bf16, LSE
@@ -403,14 +510,15 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(bar_o_empty(slot));
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_o_empty(slot));
             p.lse[grow] = m_used * p.scale + logf(l);
         }
     }
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);

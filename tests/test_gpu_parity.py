@@ -190,3 +190,50 @@ def test_shape_mismatch_rejected_before_launch(sta):
     with pytest.raises(sta.StaError) as e:
         sta.sta_forward(plan, q96, q96, q96, torch.empty_like(q96), lse, 0.1)
     assert e.value.status == sta.STA_ERR_UNSUPPORTED
+
+
+# ---------------------------------------------------------------- online-softmax rescale paths
+
+def test_forward_running_max_grows_every_chunk(sta):
+    # Scores rise by 12 log2-units from one 32-key chunk (in the kernel's visit
+    # order: ascending tile id, tile-major inside a tile) to the next, so the
+    # running max moves inside every row step and across steps: the P already
+    # written, the row sum and O are all rescaled many times.
+    latent, tile, d = (6, 16, 16), (6, 8, 8), 64
+    N = latent[0] * latent[1] * latent[2]
+    scale = 1.0 / math.sqrt(d)
+    c = scale * 1.4426950408889634
+    tm = oracle.tile_major_index(latent, tile, np.arange(N))   # visit position of each raster key
+    q = torch.zeros(1, 1, N, d)
+    q[..., 0] = 8.0
+    k = torch.zeros(1, 1, N, d)
+    k[0, 0, :, 0] = torch.from_numpy(12.0 * (tm // 32) / (c * 8.0)).float()
+    g = torch.Generator().manual_seed(5)
+    v = torch.randn(1, 1, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    windows = [latent]
+    plan = sta.sta_plan(latent, tile, 1, 1, windows)
+    o, lse = sta.sta_attention(q.cuda(), k.cuda(), v.cuda(), plan, scale)
+    assert sta.sta_last_device_status(plan) == 0
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, scale)
+    compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
+            what="rising max")
+
+
+@pytest.mark.parametrize("factor", [4.0, 6.0])
+def test_forward_sharp_softmax_random(sta, factor):
+    # Q and K scaled so logits have std ~factor^2: row maxima jump by far more
+    # than 2^8 between chunks early in a row.
+    latent, tile, B, H, d = (12, 16, 16), (6, 8, 8), 1, 2, 128
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator().manual_seed(int(factor * 10))
+    q, k = ((factor * torch.randn(B, H, N, d, generator=g)).to(torch.bfloat16) for _ in range(2))
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    windows = [(12, 16, 8), (12, 16, 16)]
+    scale = 1.0 / math.sqrt(d)
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    o, lse = sta.sta_attention(q.cuda(), k.cuda(), v.cuda(), plan, scale)
+    assert sta.sta_last_device_status(plan) == 0
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, scale)
+    compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
+            what=f"sharp x{factor}")
