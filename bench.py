@@ -2,10 +2,11 @@
 """Benchmark of the STA forward hot path on B200.
 
 One step = one pass of the whole path over one batch of synthetic input:
-    raster Q, K, V  --sta_tile_reorder x3-->  tile-major
-    sta_forward (plan built once per geometry / window set, outside the step)
-    tile-major O, LSE  --sta_tile_unreorder x2-->  raster
-on the 720p 5 s HunyuanVideo-shaped workload (B=1, 24 heads, d=128, latent
+raster Q, K, V -> STA forward -> raster O, LSE, done by sta_forward_raster (the
+tile permutation fused into the kernel's loads and stores; the plan is built
+once per geometry / window set, outside the step).  The unfused pipeline
+(sta_tile_reorder x3 -> sta_forward -> sta_tile_unreorder x2) is timed too
+and reported under "permuted_pipeline".  Workload: the 720p 5 s HunyuanVideo-shaped one (B=1, 24 heads, d=128, latent
 30x48x80, tile 6x8x8, window 18x24x24).  Inputs (3 x 707.8 MB) are larger than
 L2, so no flush is needed between steps.
 
@@ -155,7 +156,7 @@ def workload_config(w, wins, world: int) -> dict:
             "parallelism": f"replicas{world}",
             "l2": "inputs larger than L2 (3 x %.1f MB per step), no flush"
                   % (w.batch * w.heads * w.tokens * w.head_dim * 2 / 1e6),
-            "step": "reorder Q,K,V + sta_forward + unreorder O,LSE; plan built once"}
+            "step": "sta_forward_raster (permutation fused), raster in and out; plan built once"}
 
 
 def max_over_ranks(dist, x: float, device) -> float:
@@ -294,20 +295,23 @@ def main():
     ev_fwd = []
 
     def step(record=False):
-        sta.sta_tile_reorder(q, qt, L, T)
-        sta.sta_tile_reorder(k, kt, L, T)
-        sta.sta_tile_reorder(v, vt, L, T)
         if record:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-        sta.sta_forward(plan, qt, kt, vt, ot, lset, scale)
+        sta.sta_forward_raster(plan, q, k, v, o, lse, scale)
         if record:
             e1.record()
             ev_fwd.append((e0, e1))
+
+    def permuted_step():
+        sta.sta_tile_reorder(q, qt, L, T)
+        sta.sta_tile_reorder(k, kt, L, T)
+        sta.sta_tile_reorder(v, vt, L, T)
+        sta.sta_forward(plan, qt, kt, vt, ot, lset, scale)
         sta.sta_tile_unreorder(ot, o, L, T)
         sta.sta_tile_unreorder(lset, lse, L, T, token_dim=2)
 
-    launches_per_step = 6
+    launches_per_step = 1
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -347,13 +351,13 @@ def main():
         # ------------------------------------------- full-window denominator
         full = sta.sta_plan(L, T, B, H, [tuple(L)] * H)
         for _ in range(2):
-            sta.sta_forward(full, qt, kt, vt, ot, lset, scale)
+            sta.sta_forward_raster(full, q, k, v, o, lse, scale)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 3
         e0.record()
         for _ in range(reps):
-            sta.sta_forward(full, qt, kt, vt, ot, lset, scale)
+            sta.sta_forward_raster(full, q, k, v, o, lse, scale)
         e1.record()
         torch.cuda.synchronize()
         full_ms = reduce_max(e0.elapsed_time(e1) / reps)
@@ -364,6 +368,20 @@ def main():
         if sta.sta_last_device_status(full) != 0:
             raise RuntimeError("device status error in the full-window run")
         full.destroy()
+        # ------------------------------------------- unfused pipeline
+        for _ in range(2):
+            permuted_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 5
+        e0.record()
+        for _ in range(reps):
+            permuted_step()
+        e1.record()
+        torch.cuda.synchronize()
+        perm_pipe_ms = reduce_max(e0.elapsed_time(e1) / reps)
+        extras["permuted_pipeline"] = {"ms": perm_pipe_ms, "tflops": flops / (perm_pipe_ms * 1e-3) / 1e12,
+                                       "launches": 6}
         # ------------------------------------------- permutation bandwidth
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -419,7 +437,7 @@ def main():
             "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak, "traffic": measured_traffic(),
-                         "kernel": "sta_fwd_kernel<128>",
+                         "kernel": "sta_fwd_kernel<128, raster>",
                          "peak_source": f"bf16_tflops_sustained ({peak_kind})",
                          "frac_of_burst": fwd_tflops / float(peaks.get("bf16_tflops", 1590.0))},
             "gpu_launches": launches_per_step * args.steps,

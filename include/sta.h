@@ -137,6 +137,20 @@ STA_API sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const
                        void* o, float* lse, int32_t head_dim, float softmax_scale,
                        void* stream);
 
+/* STA forward on raster-order tensors, the token permutation fused into the
+ * kernel's loads and stores (no reorder / unreorder passes).
+ *   q, k, v : device bf16 [B, heads, N, d] in raster token order (t, h, w)
+ *   o       : device bf16 [B, heads, N, d], raster order (written)
+ *   lse     : device fp32 [B, heads, N], raster order (written)
+ * Same arithmetic and results as sta_tile_reorder -> sta_forward ->
+ * sta_tile_unreorder, bit for bit.  Each 128-row block of a tile must be a box
+ * of whole (h, w) slices (tile_h * tile_w divides 128) or a run of whole w rows
+ * of one slice (128 divides tile_h * tile_w and tile_w divides 128), else
+ * UNSUPPORTED; 6x8x8 tiles are two slices per block.  Other rules as sta_forward. */
+STA_API sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k, const void* v,
+                                      void* o, float* lse, int32_t head_dim, float softmax_scale,
+                                      void* stream);
+
 /* STA forward that allocates nothing (this call has no counterpart in the
  * paper; it exists for deployment).
  *

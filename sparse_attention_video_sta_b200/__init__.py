@@ -25,8 +25,8 @@ import torch
 
 __all__ = [
     "StaError", "Plan", "sta_plan", "sta_plan_host", "sta_tile_reorder", "sta_tile_unreorder",
-    "sta_forward", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string",
-    "sta_debug_inject_timeout", "sta_attention", "library_path", "EXPORTED_SYMBOLS",
+    "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
+    "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,7 @@ STA_ERR_OOM = 5
 EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
-    "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
+    "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail",
 )
 
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "sta_tile_reorder": [vp, vp, i64, i32, G, vp],
         "sta_tile_unreorder": [vp, vp, i64, i32, G, vp],
         "sta_forward": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
+        "sta_forward_raster": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
@@ -270,9 +271,7 @@ def sta_tile_unreorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token
     return dst
 
 
-def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
-                o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
-    """STA forward on tile-major ``[B, H, N, d]`` bf16 tensors; writes ``o`` and ``lse``."""
+def _forward_args(plan: Plan, q, k, v, o, lse):
     B, H, N = plan.batch, plan.heads, plan.tokens
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
@@ -285,11 +284,33 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if not lse.is_cuda or lse.dtype != torch.float32 or not lse.is_contiguous() \
             or tuple(lse.shape) != (B, H, N):
         raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape [{B}, {H}, {N}]")
-    _check(_lib.sta_forward(plan.handle, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
-                            ctypes.c_void_p(lse.data_ptr()), int(d), float(softmax_scale),
-                            _stream(stream)), "sta_forward")
+    return (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()), ctypes.c_void_p(v.data_ptr()),
+            ctypes.c_void_p(o.data_ptr()), ctypes.c_void_p(lse.data_ptr()), int(d))
+
+
+def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
+    """STA forward on tile-major ``[B, H, N, d]`` bf16 tensors; writes ``o`` and ``lse``."""
+    args = _forward_args(plan, q, k, v, o, lse)
+    _check(_lib.sta_forward(plan.handle, *args, float(softmax_scale), _stream(stream)), "sta_forward")
     return o, lse
+
+
+def sta_forward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                       o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
+    """STA forward on raster-order ``[B, H, N, d]`` bf16 tensors (permutation fused)."""
+    args = _forward_args(plan, q, k, v, o, lse)
+    _check(_lib.sta_forward_raster(plan.handle, *args, float(softmax_scale), _stream(stream)),
+           "sta_forward_raster")
+    return o, lse
+
+
+def raster_supported(tile) -> bool:
+    """Whether the fused raster path handles this tile shape (see sta.h)."""
+    hw = int(tile[1]) * int(tile[2])
+    if 128 % hw == 0:
+        return int(tile[0]) % (128 // hw) == 0 and int(tile[1]) <= 256 and int(tile[2]) <= 256
+    return hw % 128 == 0 and 128 % int(tile[2]) == 0
 
 
 def sta_forward_noalloc(latent, tile, batch: int, heads: int, windows, q: torch.Tensor,
@@ -327,15 +348,21 @@ def sta_debug_inject_timeout(enable: bool, limit_ms: int = 50) -> None:
 
 
 def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
-                  softmax_scale: float | None = None, stream=None):
+                  softmax_scale: float | None = None, stream=None, fused: bool = True):
     """STA attention on raster-order ``[B, H, N, d]`` bf16 tensors.
 
-    Permutes Q, K, V to tile-major order, runs the forward kernel, and permutes
-    O and LSE back.  Returns ``(O bf16 [B, H, N, d], LSE fp32 [B, H, N])``.
+    With ``fused`` (and a tile shape the fused kernel handles) one kernel reads
+    and writes raster order directly; otherwise Q, K, V are permuted to
+    tile-major order, the forward kernel runs, and O and LSE are permuted back.
+    Both give the same bits.  Returns ``(O bf16 [B, H, N, d], LSE fp32 [B, H, N])``.
     """
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(q.shape[-1])
     lat, tile = plan.latent, plan.tile
+    if fused and raster_supported(tile):
+        o = torch.empty_like(q)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+        return sta_forward_raster(plan, q, k, v, o, lse, softmax_scale, stream=stream)
     qt, kt, vt = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     sta_tile_reorder(q, qt, lat, tile, stream=stream)
     sta_tile_reorder(k, kt, lat, tile, stream=stream)

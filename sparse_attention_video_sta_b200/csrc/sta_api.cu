@@ -125,6 +125,17 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
         off[P.tiles_per_head] = int32_t(P.csr_ids.size());
     }
 
+    // Raster origin of every tile (token coordinates of its first token).
+    P.tile_origin.assign(size_t(P.tiles_per_head) * 4, 0);
+    for (int32_t qt = 0; qt < nt; ++qt)
+        for (int32_t qh = 0; qh < nh; ++qh)
+            for (int32_t qw = 0; qw < nw; ++qw) {
+                int32_t* o = &P.tile_origin[size_t((qt * nh + qh) * nw + qw) * 4];
+                o[0] = qw * T[2];
+                o[1] = qh * T[1];
+                o[2] = qt * T[0];
+            }
+
     // Work items.  Row blocks of one tile are paired so the pair shares K/V
     // loads; with an odd count per tile, the last block of consecutive tiles
     // are paired instead (each with its own list, same length).
@@ -163,10 +174,12 @@ void free_device(sta_plan_s* p) {
     if (p->d_ids) cudaFree(p->d_ids);
     if (p->d_items) cudaFree(p->d_items);
     if (p->d_status) cudaFree(p->d_status);
+    if (p->d_origin) cudaFree(p->d_origin);
     p->d_off = nullptr;
     p->d_ids = nullptr;
     p->d_items = nullptr;
     p->d_status = nullptr;
+    p->d_origin = nullptr;
     p->on_device = false;
 }
 
@@ -192,6 +205,27 @@ sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row
     if (s < d + uint64_t(bytes) && d < s + uint64_t(bytes)) return STA_ERR_INVALID_ARG;  // overlap
     return cuda_status(sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+sta_status forward_common(sta_plan_t p, const void* q, const void* k, const void* v, void* o, float* lse,
+                          int32_t head_dim, float softmax_scale, void* stream, bool raster) {
+    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
+        return STA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
+    if (dev != p->device) return STA_ERR_INVALID_ARG;
+    const int inject = g_inject_timeout.load();
+    const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
+                                  : kDefaultTimeoutNs;
+    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
+    return cuda_status(sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
+                                           static_cast<cudaStream_t>(stream), inject, limit, raster));
 }
 
 }  // namespace
@@ -240,6 +274,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = upload(&p->d_off, p->h.csr_off, s);
     if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
+    if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
     if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&p->d_status), sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -258,7 +293,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status) {
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
         free_device(p);
     }
@@ -314,22 +349,12 @@ sta_status sta_tile_unreorder(const void* src, void* dst, int64_t outer, int32_t
 
 sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v, void* o,
                        float* lse, int32_t head_dim, float softmax_scale, void* stream) {
-    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
-    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
-        return STA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
-        !aligned(lse, 4))
-        return STA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
-    int dev = -1;
-    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
-    if (dev != p->device) return STA_ERR_INVALID_ARG;
-    const int inject = g_inject_timeout.load();
-    const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
-                                  : kDefaultTimeoutNs;
-    return cuda_status(sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
-                                           static_cast<cudaStream_t>(stream), inject, limit));
+    return forward_common(p, q, k, v, o, lse, head_dim, softmax_scale, stream, false);
+}
+
+sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k, const void* v, void* o,
+                              float* lse, int32_t head_dim, float softmax_scale, void* stream) {
+    return forward_common(p, q, k, v, o, lse, head_dim, softmax_scale, stream, true);
 }
 
 sta_status sta_last_device_status(sta_plan_t p, void* stream) {

@@ -44,9 +44,17 @@
 namespace sta {
 namespace {
 
-constexpr int kThreads = 352;
+constexpr int kThreads = 384;  // 3 warpgroups: softmax slot 0, softmax slot 1, producers
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp0 = 9;  // slot 0 issuer; also allocates TMEM.  Slot 1 issuer: warp 10.
+// Registers per thread: launched at 168 (384 threads, 3 warps per SM
+// sub-partition); the producer warpgroup (warps 8-11, warp 11 idle) gives
+// registers to the two softmax warpgroups.  128 * (208 + 208 + 88) is within the
+// launch's 384 * 168, so the increase never waits on registers that are not there
+// (88 keeps the producer code free of spills).
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsProducer = 88;
+static_assert(128 * (2 * kRegsSoftmax + kRegsProducer) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
@@ -91,7 +99,50 @@ struct FwdParams {
     uint32_t* status;
     uint64_t timeout_ns;
     int32_t inject;
+    // Raster layout only: latent and tile extents, tiles along h and w, and the
+    // shape of one 128-row block as a box of whole (t, h) slices.
+    int32_t lat_h, lat_w;
+    int32_t tile_t, tile_h, tile_w;
+    int32_t n_h, n_w;
+    int32_t box_t, box_h, blocks_per_slice;
+    const int4* tile_origin;  // [tiles]: raster (w, h, t) origin of each tile
 };
+
+// Load 128-row block `sub` of tile `tile` of head bh.  Tile-major layout: one
+// 2D row coordinate.  Raster layout: the (w, h, t) origin of the block's box
+// inside the tile (tile origin from the plan's table), whose rows TMA lays out
+// in tile-major order.
+template <bool kRaster>
+__device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* m, uint32_t bar, const FwdParams& p,
+                                           int32_t bh, int32_t tile, int32_t sub, int col_blocks, int box_bytes) {
+    if (!kRaster) {
+        const int32_t row = bh * p.tokens + tile * p.tile_tokens + sub * kSubRows;
+        for (int cb = 0; cb < col_blocks; ++cb) ptx::tma_load_2d(dst + cb * box_bytes, m, bar, cb * 64, row);
+    } else {
+        const int4 org = p.tile_origin[tile];
+        int32_t t0 = org.z, h0 = org.y;
+        if (p.blocks_per_slice == 1) {
+            t0 += sub * p.box_t;
+        } else {
+            t0 += sub / p.blocks_per_slice;
+            h0 += (sub % p.blocks_per_slice) * p.box_h;
+        }
+        for (int cb = 0; cb < col_blocks; ++cb)
+            ptx::tma_load_5d(dst + cb * box_bytes, m, bar, cb * 64, org.x, h0, t0, bh);
+    }
+}
+
+// Row of the output tensors that holds row `r` of block `blk` of head bh.
+template <bool kRaster>
+__device__ __forceinline__ int64_t out_row(const FwdParams& p, int32_t bh, int32_t blk, int32_t r) {
+    if (!kRaster) return int64_t(bh) * p.tokens + int64_t(blk) * kSubRows + r;
+    const int32_t tile = blk / p.sub_per_tile, sub = blk - tile * p.sub_per_tile;
+    const int32_t it = tile / (p.n_h * p.n_w), ih = (tile / p.n_w) % p.n_h, iw = tile % p.n_w;
+    const int32_t l = sub * kSubRows + r;  // tile-local row, raster over the tile's (t, h, w)
+    const int32_t lw = l % p.tile_w, lh = (l / p.tile_w) % p.tile_h, lt = l / (p.tile_w * p.tile_h);
+    const int64_t token = (int64_t(it * p.tile_t + lt) * p.lat_h + ih * p.tile_h + lh) * p.lat_w + iw * p.tile_w + lw;
+    return int64_t(bh) * p.tokens + token;
+}
 
 // Bounded mbarrier wait.  Returns false when the CTA is aborting (another role
 // gave up) or when this wait ran past the time limit (then it starts the abort).
@@ -169,7 +220,7 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[128]) {
     return ptx::max3(a0, a1, fmaxf(a2, a3));
 }
 
-template <int D>
+template <int D, bool kRaster>
 __global__ void __launch_bounds__(kThreads, 1)
 sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -238,6 +289,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int32_t SPT = p.sub_per_tile;
 
     if (warp == kLoadWarp) {
+        ptx::regs_dec<kRegsProducer>();
         if (lane == 0) {
             // ------------------------------------------------------------ load
             // Ring stage r holds one K or V chunk.  `users` keeps, 2 bits per
@@ -250,7 +302,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // Debug: wait on a barrier nothing arrives at; the limit runs out.
                 ok = wait_bar(bar_dead, 0, abort_flag, p);
             }
-            auto issue = [&](const CUtensorMap* m, int32_t row, uint32_t mask) -> bool {
+            auto issue = [&](const CUtensorMap* m, int32_t bh, int32_t tile, int32_t sub, uint32_t mask) -> bool {
                 const int r = int(item % S);
                 const uint32_t prev = (users >> (2 * r)) & 3u;
 #pragma unroll
@@ -260,11 +312,9 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                             return false;
                 users = (users & ~(3u << (2 * r))) | (mask << (2 * r));
                 upar ^= mask << (2 * r);
-                const uint32_t dst = base + C::kRingOff + r * C::kKVBytes;
                 ptx::mbar_arrive_expect_tx(bar_full(r), C::kKVBytes);
-#pragma unroll
-                for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    ptx::tma_load_2d(dst + cb * C::kBoxBytes, m, bar_full(r), cb * 64, row);
+                load_block<kRaster>(base + C::kRingOff + r * C::kKVBytes, m, bar_full(r), p, bh, tile, sub,
+                                    C::kColBlocks, C::kBoxBytes);
                 ++item;
                 return true;
             };
@@ -277,36 +327,38 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 const int32_t* list_a = p.ids + off[tile_a];
                 const int32_t* list_b = p.ids + off[tile_b];
                 const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
-                const int32_t head_row = w.bh * p.tokens;
                 // query blocks, one buffer per slot
                 if (!wait_bar(bar_q_empty(0), (qc0 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
                 ptx::mbar_arrive_expect_tx(bar_q_full(0), C::kQBytes);
-#pragma unroll
-                for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    ptx::tma_load_2d(base + C::kQOff + cb * C::kBoxBytes, &tm_q, bar_q_full(0), cb * 64,
-                                     head_row + w.qa * kSubRows);
+                load_block<kRaster>(base + C::kQOff, &tm_q, bar_q_full(0), p, w.bh, tile_a, w.qa - tile_a * SPT,
+                                    C::kColBlocks, C::kBoxBytes);
                 ++qc0;
                 if (has_b) {
                     if (!wait_bar(bar_q_empty(1), (qc1 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(bar_q_full(1), C::kQBytes);
-#pragma unroll
-                    for (int cb = 0; cb < C::kColBlocks; ++cb)
-                        ptx::tma_load_2d(base + C::kQOff + C::kQBytes + cb * C::kBoxBytes, &tm_q,
-                                         bar_q_full(1), cb * 64, head_row + w.qb * kSubRows);
+                    load_block<kRaster>(base + C::kQOff + C::kQBytes, &tm_q, bar_q_full(1), p, w.bh, tile_b,
+                                        w.qb - tile_b * SPT, C::kColBlocks, C::kBoxBytes);
                     ++qc1;
                 }
-                // K / V chunks in the order the issuers consume them
+                // K / V chunks in the order the issuers consume them: chunk kc of
+                // key tile kt is one 128-row block.  The key-tile ids of the next
+                // tile are read one tile ahead so no TMA issue waits on them.
                 const uint32_t both = has_b ? 3u : 1u;
-                for (int32_t i = 0; ok && i < n_chunks; ++i) {
-                    const int32_t kt = i / SPT, kc = i - kt * SPT;
-                    const int32_t row_a = head_row + list_a[kt] * p.tile_tokens + kc * kChunkKeys;
-                    const int32_t row_b = head_row + list_b[kt] * p.tile_tokens + kc * kChunkKeys;
-                    if (split) {
-                        ok = issue(&tm_k, row_a, 1u) && issue(&tm_k, row_b, 2u) && issue(&tm_v, row_a, 1u) &&
-                             issue(&tm_v, row_b, 2u);
-                    } else {
-                        ok = issue(&tm_k, row_a, both) && issue(&tm_v, row_a, both);
+                const int32_t n_kt = n_chunks / SPT;
+                int32_t ta = __ldg(list_a), tb = __ldg(list_b);
+                for (int32_t kt = 0; ok && kt < n_kt; ++kt) {
+                    const int32_t nta = kt + 1 < n_kt ? __ldg(list_a + kt + 1) : 0;
+                    const int32_t ntb = kt + 1 < n_kt ? __ldg(list_b + kt + 1) : 0;
+                    for (int32_t kc = 0; ok && kc < SPT; ++kc) {
+                        if (split) {
+                            ok = issue(&tm_k, w.bh, ta, kc, 1u) && issue(&tm_k, w.bh, tb, kc, 2u) &&
+                                 issue(&tm_v, w.bh, ta, kc, 1u) && issue(&tm_v, w.bh, tb, kc, 2u);
+                        } else {
+                            ok = issue(&tm_k, w.bh, ta, kc, both) && issue(&tm_v, w.bh, ta, kc, both);
+                        }
                     }
+                    ta = nta;
+                    tb = ntb;
                 }
             }
             // Drain: the copies issued last into each stage, and the last query loads.
@@ -316,7 +368,11 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (qc0 > 0) drain_bar(bar_q_full(0), (qc0 - 1) & 1u, p.timeout_ns);
             if (qc1 > 0) drain_bar(bar_q_full(1), (qc1 - 1) & 1u, p.timeout_ns);
         }
+    } else if (warp == kMmaWarp0 + 2) {
+        // idle: completes the producer warpgroup for the register hand-over
+        ptx::regs_dec<kRegsProducer>();
     } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
+        ptx::regs_dec<kRegsProducer>();
         if (lane == 0) {
             // ------------------------------------------------------------- MMA
             const int s = warp - kMmaWarp0;  // the query slot this thread serves
@@ -405,6 +461,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------- softmax
+        ptx::regs_inc<kRegsSoftmax>();
         const int slot = warp >> 2;
         const int row = threadIdx.x & 127;
         const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
@@ -493,7 +550,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ++ocnt;
             ptx::tc_fence_after();
             const float inv_l = 1.0f / l;
-            const int64_t grow = int64_t(w.bh) * p.tokens + int64_t(q_blk) * kSubRows + row;
+            const int64_t grow = out_row<kRaster>(p, w.bh, q_blk, row);
             uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D);
 #pragma unroll 1
             for (int cb = 0; cb < D / 32; ++cb) {
@@ -558,15 +615,45 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) {
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 5D map over a raster [BH, L_t, L_h, L_w, d] bf16 tensor whose box is one
+// 128-row block of a tile: 64 elements x tile_w x box_h x box_t x 1, with the
+// same 128-byte swizzle; TMA writes the box's rows in tile-major order.
+cudaError_t make_map_raster(CUtensorMap* m, const void* ptr, const sta_geom& g, int64_t bh, int d,
+                            int box_t, int box_h) {
+    const EncodeFn& e = encode_fn();
+    if (e.err != cudaSuccess) return e.err;
+    const cuuint64_t row = cuuint64_t(d) * 2;
+    cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(g.lat_w), cuuint64_t(g.lat_h), cuuint64_t(g.lat_t),
+                          cuuint64_t(bh)};
+    cuuint64_t strides[4] = {row, row * g.lat_w, row * g.lat_w * g.lat_h, row * g.lat_w * g.lat_h * g.lat_t};
+    cuuint32_t box[5] = {64, cuuint32_t(g.tile_w), cuuint32_t(box_h), cuuint32_t(box_t), 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = e.fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int D>
 cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const void* v, void* o,
-                     float* lse, float scale, cudaStream_t stream, int inject, uint64_t timeout_ns) {
+                     float* lse, float scale, cudaStream_t stream, int inject, uint64_t timeout_ns,
+                     bool raster) {
     const PlanHost& P = pl->h;
-    const int64_t rows = int64_t(P.batch) * P.heads * P.tiles_per_head * P.tile_tokens;
+    const int64_t bh = int64_t(P.batch) * P.heads;
+    const int64_t rows = bh * P.tiles_per_head * P.tile_tokens;
+    const RasterBox rb = raster_box(P.g);
+    if (raster && !rb.ok) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
-    cudaError_t e = make_map(&mq, q, rows, D);
-    if (e == cudaSuccess) e = make_map(&mk, k, rows, D);
-    if (e == cudaSuccess) e = make_map(&mv, v, rows, D);
+    cudaError_t e;
+    if (raster) {
+        e = make_map_raster(&mq, q, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_map_raster(&mk, k, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_map_raster(&mv, v, P.g, bh, D, rb.box_t, rb.box_h);
+    } else {
+        e = make_map(&mq, q, rows, D);
+        if (e == cudaSuccess) e = make_map(&mk, k, rows, D);
+        if (e == cudaSuccess) e = make_map(&mv, v, rows, D);
+    }
     if (e != cudaSuccess) return e;
     FwdParams fp;
     fp.items = pl->d_items;
@@ -584,27 +671,63 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.status = pl->d_status;
     fp.timeout_ns = timeout_ns;
     fp.inject = inject;
+    fp.lat_h = P.g.lat_h;
+    fp.lat_w = P.g.lat_w;
+    fp.tile_t = P.g.tile_t;
+    fp.tile_h = P.g.tile_h;
+    fp.tile_w = P.g.tile_w;
+    fp.n_h = P.n_tiles[1];
+    fp.n_w = P.n_tiles[2];
+    fp.box_t = rb.box_t;
+    fp.box_h = rb.box_h;
+    fp.blocks_per_slice = rb.blocks_per_slice;
+    fp.tile_origin = reinterpret_cast<const int4*>(pl->d_origin);
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(sta_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg<D>::kSmemBytes);
-    if (e != cudaSuccess) return e;
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
-    sta_fwd_kernel<D><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    if (raster) {
+        e = cudaFuncSetAttribute(sta_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<D>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        sta_fwd_kernel<D, true><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    } else {
+        e = cudaFuncSetAttribute(sta_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<D>::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        sta_fwd_kernel<D, false><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    }
     return cudaGetLastError();
 }
 
 }  // namespace
 
+RasterBox raster_box(const sta_geom& g) {
+    RasterBox rb{0, 0, 0, false};
+    const int32_t hw = g.tile_h * g.tile_w;
+    if (hw <= 0 || g.tile_w > 256) return rb;
+    if (kSubRows % hw == 0) {  // a block is whole (h, w) slices: box_t of them
+        rb.box_t = kSubRows / hw;
+        rb.box_h = g.tile_h;
+        rb.blocks_per_slice = 1;
+        rb.ok = g.tile_h <= 256 && g.tile_t % rb.box_t == 0;
+    } else if (hw % kSubRows == 0 && kSubRows % g.tile_w == 0) {  // a block is part of one slice
+        rb.box_t = 1;
+        rb.box_h = kSubRows / g.tile_w;
+        rb.blocks_per_slice = hw / kSubRows;
+        rb.ok = true;
+    }
+    return rb;
+}
+
 cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, const void* v, void* o,
                            float* lse, int head_dim, float softmax_scale, cudaStream_t stream,
-                           int inject_timeout, uint64_t timeout_ns) {
+                           int inject_timeout, uint64_t timeout_ns, bool raster) {
     if (head_dim == 128)
-        return launch_d<128>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns);
-    return launch_d<64>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns);
+        return launch_d<128>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns, raster);
+    return launch_d<64>(p, q, k, v, o, lse, softmax_scale, stream, inject_timeout, timeout_ns, raster);
 }
 
 cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void* k, const void* v,
@@ -616,7 +739,7 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     if (e == cudaSuccess) e = make_map(&mk, k, rows, head_dim);
     if (e == cudaSuccess) e = make_map(&mv, v, rows, head_dim);
     if (e != cudaSuccess) return e;
-    FwdParams fp;
+    FwdParams fp{};
     fp.items = pv.items;
     fp.n_items = pv.n_items;
     fp.off = pv.off;
@@ -639,15 +762,15 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
     if (head_dim == 128) {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sta_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<128>::kSmemBytes);
         if (e != cudaSuccess) return e;
-        sta_fwd_kernel<128><<<grid, kThreads, Cfg<128>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+        sta_fwd_kernel<128, false><<<grid, kThreads, Cfg<128>::kSmemBytes, stream>>>(mq, mk, mv, fp);
     } else {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(sta_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<64>::kSmemBytes);
         if (e != cudaSuccess) return e;
-        sta_fwd_kernel<64><<<grid, kThreads, Cfg<64>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+        sta_fwd_kernel<64, false><<<grid, kThreads, Cfg<64>::kSmemBytes, stream>>>(mq, mk, mv, fp);
     }
     return cudaGetLastError();
 }

@@ -40,6 +40,7 @@ struct PlanHost {
     std::vector<int32_t> csr_off;            // [n_win][tiles_per_head + 1], global offsets
     std::vector<int32_t> csr_ids;            // key-tile ids, ascending per list
     std::vector<WorkItem> items;             // work list
+    std::vector<int32_t> tile_origin;        // [tiles_per_head][4]: raster (w, h, t) origin of each tile, 0
     int64_t computed_pairs = 0;              // B * sum_h sum_q |list|
 };
 
@@ -53,14 +54,27 @@ struct sta_plan_s {
     int32_t* d_ids = nullptr;
     sta::WorkItem* d_items = nullptr;
     uint32_t* d_status = nullptr;
+    int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
 };
 
 namespace sta {
 
-// Forward kernel launch (sta_forward.cu).  Returns a CUDA error code.
+// Shape of one 128-row block of a tile as a box of whole (t, h) slices, for
+// loading Q, K, V straight from raster layout: box_t slices of tile_h rows, or
+// box_h rows of one slice (blocks_per_slice blocks per slice).  ok = false when
+// a block is not such a box.
+struct RasterBox {
+    int32_t box_t, box_h, blocks_per_slice;
+    bool ok;
+};
+RasterBox raster_box(const sta_geom& g);
+
+// Forward kernel launch (sta_forward.cu): tile-major tensors, or raster tensors
+// with the permutation done by the kernel's loads and stores (`raster`).
+// Returns a CUDA error code.
 cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, const void* v,
                            void* o, float* lse, int head_dim, float softmax_scale,
-                           cudaStream_t stream, int inject_timeout, uint64_t timeout_ns);
+                           cudaStream_t stream, int inject_timeout, uint64_t timeout_ns, bool raster);
 
 // Device-side view of a plan whose arrays live in memory the caller provides
 // (used by the no-allocation entry point, sta_noalloc.cu).

@@ -98,12 +98,12 @@ def test_forward_small_geometries_all_rows(sta, latent, tile, B, H, d, windows):
     run_full_oracle(sta, latent, tile, B, H, d, windows, 1.0 / math.sqrt(d), seed=d + H)
 
 
-def sampled_parity(sta, idx, heads, n_random, rows_per_tile):
+def sampled_parity(sta, idx, heads, n_random, rows_per_tile, fused=True):
     w = sta_inputs.WORKLOADS[idx]
     wins = sta_inputs.windows(w).tolist()
     q, k, v = sta_inputs.make_qkv(w, heads=heads)
     plan = sta.sta_plan(w.latent, w.tile, w.batch, w.heads, wins)
-    o, lse = sta.sta_attention(q.cuda(), k.cuda(), v.cuda(), plan, w.softmax_scale)
+    o, lse = sta.sta_attention(q.cuda(), k.cuda(), v.cuda(), plan, w.softmax_scale, fused=fused)
     assert sta.sta_last_device_status(plan) == 0
     tiles = sample_tiles(w.latent, w.tile, n_random, seed=idx)
     toks = tile_rows(w.latent, w.tile, tiles, rows_per_tile, seed=idx)
@@ -114,8 +114,10 @@ def sampled_parity(sta, idx, heads, n_random, rows_per_tile):
     return w, plan, o, lse, stats
 
 
-def test_forward_720p_sampled(sta):
-    w, plan, o, lse, _ = sampled_parity(sta, 2, heads=[0, 7, 16, 23], n_random=3, rows_per_tile=None)
+@pytest.mark.parametrize("fused", [True, False])
+def test_forward_720p_sampled(sta, fused):
+    w, plan, o, lse, _ = sampled_parity(sta, 2, heads=[0, 7, 16, 23], n_random=3, rows_per_tile=None,
+                                        fused=fused)
     # heads that were not drawn hold zeros: every score is 0, so O = 0 exactly
     # and LSE = ln(27 * 384) (27 key tiles of 384 tokens)
     zero = [h for h in range(w.heads) if h not in (0, 7, 16, 23)]
@@ -237,3 +239,56 @@ def test_forward_sharp_softmax_random(sta, factor):
     o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, scale)
     compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
             what=f"sharp x{factor}")
+
+
+# ---------------------------------------------------------------- fused raster path
+
+@pytest.mark.parametrize("latent,tile,B,H,d,windows", [
+    ((18, 24, 24), (6, 8, 8), 1, 2, 64, [(12, 16, 16)] * 2),      # 2 (h, w) slices per block
+    ((30, 48, 80), (6, 8, 8), 1, 2, 128, [(18, 24, 24), (30, 40, 40)]),
+    ((8, 16, 24), (4, 8, 8), 2, 1, 128, [(8, 16, 16)]),            # 256-token tiles
+    ((4, 16, 32), (1, 8, 16), 1, 2, 64, [(2, 8, 32), (4, 16, 16)]),  # one slice per block
+    ((4, 32, 32), (2, 16, 16), 1, 1, 128, [(2, 32, 32)]),          # half a slice per block
+])
+def test_fused_raster_path_matches_permuted_path_bit_for_bit(sta, latent, tile, B, H, d, windows):
+    assert sta.raster_supported(tile)
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator(device="cuda").manual_seed(N + d)
+    q, k, v = (torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    o1, l1 = sta.sta_attention(q, k, v, plan, 1.0 / math.sqrt(d), fused=True)
+    o2, l2 = sta.sta_attention(q, k, v, plan, 1.0 / math.sqrt(d), fused=False)
+    assert sta.sta_last_device_status(plan) == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fused_raster_path_matches_oracle(sta):
+    latent, tile, B, H, d = (4, 32, 32), (2, 16, 16), 1, 2, 64
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator().manual_seed(77)
+    q, k, v = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    windows = [(2, 16, 32), (4, 32, 16)]
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    o = torch.empty(B, H, N, d, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    sta.sta_forward_raster(plan, q.cuda(), k.cuda(), v.cuda(), o, lse, 0.125)
+    assert sta.sta_last_device_status(plan) == 0
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, 0.125)
+    compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
+            what="raster")
+
+
+def test_fused_raster_rejects_unsupported_tiles(sta):
+    tile = (8, 4, 12)  # 384 tokens, but a 128-row block is not a box of whole rows / slices
+    assert not sta.raster_supported(tile)
+    latent = (8, 8, 24)
+    N = latent[0] * latent[1] * latent[2]
+    plan = sta.sta_plan(latent, tile, 1, 1, [tile])
+    x = torch.zeros(1, 1, N, 64, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(1, 1, N, dtype=torch.float32, device="cuda")
+    with pytest.raises(sta.StaError) as e:
+        sta.sta_forward_raster(plan, x, x, x, torch.empty_like(x), lse, 0.125)
+    assert e.value.status == sta.STA_ERR_UNSUPPORTED
+    o, l = sta.sta_attention(x, x, x, plan, 0.125)   # runs the reorder / forward / unreorder kernels
+    assert sta.sta_last_device_status(plan) == 0
+    assert torch.count_nonzero(o).item() == 0
