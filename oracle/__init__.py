@@ -67,6 +67,12 @@ def lib() -> ctypes.CDLL:
                 ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
                 ctypes.c_int32]
             L.ora_sta_attention.restype = ctypes.c_int
+            bw = [ctypes.c_void_p] * 4 + [G, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, i32p,
+                                          ctypes.c_float, ctypes.c_void_p, ctypes.c_int64]
+            L.ora_sta_backward_dq.argtypes = bw + [ctypes.c_void_p, ctypes.c_int32]
+            L.ora_sta_backward_dq.restype = ctypes.c_int
+            L.ora_sta_backward_dkdv.argtypes = bw + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+            L.ora_sta_backward_dkdv.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -184,3 +190,78 @@ def sta_attention(q, k, v, latent, tile, windows, softmax_scale: float,
     if full:
         return out_o.reshape(B, H, N, d), out_lse.reshape(B, H, N)
     return out_o, out_lse
+
+
+def _rows_or_all(rows, B, H, N):
+    if rows is None:
+        bh = np.repeat(np.arange(B * H, dtype=np.int64), N)
+        tok = np.tile(np.arange(N, dtype=np.int64), B * H)
+        return np.stack([bh, tok], axis=1), True
+    return np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 2)), False
+
+
+def _bw_args(q, k, v, dout, latent, windows):
+    qa, ka, va, da = _as_u16(q), _as_u16(k), _as_u16(v), _as_u16(dout)
+    if qa.ndim != 4 or any(x.shape != qa.shape for x in (ka, va, da)):
+        raise ValueError("oracle: q, k, v, dout must share a [B, H, N, d] shape")
+    B, H, N, d = qa.shape
+    if N != num_tokens(latent):
+        raise ValueError("oracle: N does not match the latent")
+    win = np.ascontiguousarray(np.asarray(windows, dtype=np.int32).reshape(H, 3))
+    return qa, ka, va, da, win, (B, H, N, d)
+
+
+def sta_backward_dq(q, k, v, dout, latent, tile, windows, softmax_scale: float,
+                    rows=None, nthreads: int | None = None):
+    """fp64 gradient of STA attention with respect to Q, for upstream gradient
+    ``dout`` (same shape as O).
+
+    rows : optional ``[R, 2]`` pairs ``(b * H + h, raster query token)``;
+           default every row, returned as ``[B, H, N, d]``, else ``[R, d]``.
+    """
+    qa, ka, va, da, win, (B, H, N, d) = _bw_args(q, k, v, dout, latent, windows)
+    rows_a, full = _rows_or_all(rows, B, H, N)
+    out = np.empty((rows_a.shape[0], d), dtype=np.float64)
+    r = lib().ora_sta_backward_dq(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data,
+        ctypes.byref(_geom(latent, tile)), B, H, d,
+        win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), float(softmax_scale),
+        rows_a.ctypes.data, rows_a.shape[0], out.ctypes.data,
+        int(nthreads or max(1, os.cpu_count() or 1)))
+    if r != 0:
+        raise ValueError(f"oracle: ora_sta_backward_dq failed with status {r}")
+    return out.reshape(B, H, N, d) if full else out
+
+
+def sta_backward_dkdv(q, k, v, dout, latent, tile, windows, softmax_scale: float,
+                      keys=None, nthreads: int | None = None):
+    """fp64 gradients of STA attention with respect to K and V.
+
+    keys : optional ``[R, 2]`` pairs ``(b * H + h, raster key token)``;
+           default every key.  Returns ``(dK, dV)``, ``[B, H, N, d]`` each for
+           all keys, else ``[R, d]`` each.
+    """
+    qa, ka, va, da, win, (B, H, N, d) = _bw_args(q, k, v, dout, latent, windows)
+    keys_a, full = _rows_or_all(keys, B, H, N)
+    R = keys_a.shape[0]
+    dk = np.empty((R, d), dtype=np.float64)
+    dv = np.empty((R, d), dtype=np.float64)
+    r = lib().ora_sta_backward_dkdv(
+        qa.ctypes.data, ka.ctypes.data, va.ctypes.data, da.ctypes.data,
+        ctypes.byref(_geom(latent, tile)), B, H, d,
+        win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), float(softmax_scale),
+        keys_a.ctypes.data, R, dk.ctypes.data, dv.ctypes.data,
+        int(nthreads or max(1, os.cpu_count() or 1)))
+    if r != 0:
+        raise ValueError(f"oracle: ora_sta_backward_dkdv failed with status {r}")
+    if full:
+        return dk.reshape(B, H, N, d), dv.reshape(B, H, N, d)
+    return dk, dv
+
+
+def sta_backward(q, k, v, dout, latent, tile, windows, softmax_scale: float,
+                 nthreads: int | None = None):
+    """All three fp64 gradients ``(dQ, dK, dV)``, each ``[B, H, N, d]``."""
+    dq = sta_backward_dq(q, k, v, dout, latent, tile, windows, softmax_scale, nthreads=nthreads)
+    dk, dv = sta_backward_dkdv(q, k, v, dout, latent, tile, windows, softmax_scale, nthreads=nthreads)
+    return dq, dk, dv

@@ -88,7 +88,7 @@ def head_factors(w: Workload) -> torch.Tensor | None:
 
 
 def slice_seed(w: Workload, which: int, b: int, h: int) -> int:
-    """Seed of one [N, d] slice; which = 0 (Q), 1 (K), 2 (V)."""
+    """Seed of one [N, d] slice; which = 0 (Q), 1 (K), 2 (V), 3 (dO)."""
     return ((w.seed * 4 + which) * 1024 + b) * 1024 + h
 
 
@@ -97,7 +97,7 @@ def make_slice(w: Workload, which: int, b: int, h: int) -> torch.Tensor:
     rng = np.random.default_rng(slice_seed(w, which, b, h))
     x = torch.from_numpy(rng.standard_normal((w.tokens, w.head_dim), dtype=np.float32))
     f = head_factors(w)
-    if f is not None:
+    if f is not None and which < 3:
         x.mul_(float(f[h]))
     return x.to(torch.bfloat16)
 
@@ -121,3 +121,20 @@ def make_qkv(w: Workload, device="cpu", heads=None, batches=None):
     with ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1))) as ex:
         list(ex.map(one, jobs))
     return tuple(out)
+
+
+def make_dout(w: Workload, device="cpu", heads=None, batches=None) -> torch.Tensor:
+    """Upstream gradient dO for the backward pass: ``[B, H, N, d]`` bf16, raster
+    order, i.i.d. N(0, 1) rounded to bf16 (no head factor), same slice seeding."""
+    out = torch.zeros((w.batch, w.heads, w.tokens, w.head_dim), dtype=torch.bfloat16, device=device)
+    hs = range(w.heads) if heads is None else heads
+    bs = range(w.batch) if batches is None else batches
+    jobs = [(b, h) for b in bs for h in hs]
+
+    def one(job):
+        b, h = job
+        out[b, h].copy_(make_slice(w, 3, b, h))
+
+    with ThreadPoolExecutor(max_workers=max(1, min(16, os.cpu_count() or 1))) as ex:
+        list(ex.map(one, jobs))
+    return out
