@@ -395,6 +395,36 @@ def main():
                                  "peak_gbs": float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])),
                                  "bytes_per_launch": 2 * nbytes}
         extras["permutation"]["frac"] = extras["permutation"]["gbs"] / extras["permutation"]["peak_gbs"]
+        # ------------------------------------------- backward (tile-major, 3 launches)
+        permuted_step()
+        dout = torch.empty_like(q)
+        for b in range(B):
+            for h in range(H):
+                dout[b, h].copy_(torch.randn((N, d), generator=gen, device=dev, dtype=torch.float32))
+        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+        ws = torch.empty(2 * B * H * N, dtype=torch.float32, device=dev)
+
+        def bwd_step():
+            sta.sta_backward(plan, qt, kt, vt, ot, lset, dout, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+        for _ in range(2):
+            bwd_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record()
+        for _ in range(reps):
+            bwd_step()
+        e1.record()
+        torch.cuda.synchronize()
+        bwd_ms = reduce_max(e0.elapsed_time(e1) / reps)
+        if sta.sta_last_device_status(plan) != 0:
+            raise RuntimeError("device status error in the backward run")
+        # algorithmic work: five tile-pair products (S, dP, dV, dK, dQ) against the forward's two
+        bwd_flops = 2.5 * flops
+        extras["backward"] = {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12, "flops": bwd_flops,
+                              "launches": 3, "layout": "tile-major"}
+        del dout, dq, dk, dv, ws
         # ------------------------------------------- end to end from pinned host memory
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()

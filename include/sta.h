@@ -1,5 +1,6 @@
 /*
- * sta.h -- C ABI of the Sliding Tile Attention (STA) forward library (libsta).
+ * sta.h -- C ABI of the Sliding Tile Attention (STA) library (libsta): forward
+ * and backward passes.
  *
  * The method: "Fast Video Generation with Sliding Tile Attention".  A video
  * latent of L_t x L_h x L_w tokens is cut into tiles, contiguous cubes of
@@ -98,6 +99,13 @@ STA_API sta_status sta_plan_destroy(sta_plan_t p);
 STA_API sta_status sta_plan_query(sta_plan_t p, int32_t head, int32_t q_tile,
                           int32_t* kv_ids, int32_t cap, int32_t* count);
 
+/* Transposed list of key tile `k_tile` for head `head`: the query tiles whose
+ * window holds it, ascending.  Writes min(count, cap) ids to q_ids (host) and
+ * the full length to *count.  The backward's dK / dV kernel walks these lists.
+ * INVALID_ARG on a bad head / tile / pointer. */
+STA_API sta_status sta_plan_key_query(sta_plan_t p, int32_t head, int32_t k_tile,
+                                      int32_t* q_ids, int32_t cap, int32_t* count);
+
 /* Plan totals: computed (query tile, key tile) pairs over all batches and
  * heads, and number of work items.  Either pointer may be NULL. */
 STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, int64_t* work_items);
@@ -150,6 +158,37 @@ STA_API sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const
 STA_API sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k, const void* v,
                                       void* o, float* lse, int32_t head_dim, float softmax_scale,
                                       void* stream);
+
+/* STA backward on tile-major tensors: gradients of the forward's output with
+ * respect to q, k and v.  The pages use STA in fine-tuning ("Fast Video
+ * Generation with Sliding Tile Attention": podcast transcript at
+ * hotaipapers.com, fine-tuning segment; dianyo.github.io ICML-2025 post, STA
+ * section, last paragraph), which needs these gradients; they give no backward
+ * kernel.  This call computes the exact gradient of the forward's function with
+ * the tile window held fixed (the mask has no gradient):
+ *   P_ij = exp(scale q_i . k_j - lse_i) over the plan's key tiles of i's tile,
+ *   D_i = dout_i . o_i,  dS_ij = P_ij (dout_i . v_j - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j = sum_i P_ij dout_i.
+ *   q, k, v, o : device bf16 [B, heads, N, d], tile-major; o and lse as
+ *                written by sta_forward for the same q, k, v and plan
+ *   dout       : device bf16 [B, heads, N, d], tile-major: gradient w.r.t. o
+ *   lse        : device fp32 [B, heads, N], tile-major
+ *   dq, dk, dv : device bf16 [B, heads, N, d], tile-major (written; distinct
+ *                from every input)
+ *   workspace  : device fp32, 2 * B * heads * N floats, 16-byte aligned,
+ *                caller-owned; on return plane 0 holds -D_i and plane 1
+ *                -lse_i * log2(e) (row order of lse)
+ *   head_dim, softmax_scale: as sta_forward
+ * P and dS enter the tensor-core products as bf16 with fp32 accumulation;
+ * dq, dk, dv are rounded to bf16.  No atomics: results are deterministic.
+ * Allocates nothing; enqueues three kernels on `stream`.  Errors: INVALID_ARG
+ * (null or misaligned pointer, bad scale, plan not on the current device),
+ * UNSUPPORTED (head_dim), CUDA. */
+STA_API sta_status sta_backward(sta_plan_t p, const void* q, const void* k, const void* v,
+                                const void* o, const void* dout, const float* lse, void* dq,
+                                void* dk, void* dv, float* workspace, int32_t head_dim,
+                                float softmax_scale, void* stream);
 
 /* STA forward that allocates nothing (this call has no counterpart in the
  * paper; it exists for deployment).

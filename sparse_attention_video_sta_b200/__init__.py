@@ -1,4 +1,4 @@
-"""Sliding Tile Attention (STA) forward for NVIDIA B200 (sm_100a).
+"""Sliding Tile Attention (STA) forward and backward for NVIDIA B200 (sm_100a).
 
 Thin ctypes binding of the C-ABI library ``libsta.so`` (declared in
 ``include/sta.h``).  This module only marshals arguments -- tensor pointers,
@@ -11,9 +11,12 @@ The functions carry the C names:
     sta_plan / sta_plan_host -> Plan  (per-head key-tile lists + work list)
     sta_tile_reorder / sta_tile_unreorder  (raster <-> tile-major tokens)
     sta_forward                             (STA attention on tile-major tensors)
+    sta_forward_raster                      (same, raster tensors, permutation fused)
+    sta_backward                            (dQ, dK, dV on tile-major tensors)
     sta_last_device_status, sta_status_string, sta_debug_inject_timeout
 
-and ``sta_attention`` chains them for raster-order tensors.
+``sta_attention`` / ``sta_attention_backward`` chain them for raster-order
+tensors, and ``StaAttention`` wraps both as a ``torch.autograd.Function``.
 """
 from __future__ import annotations
 
@@ -27,6 +30,7 @@ __all__ = [
     "StaError", "Plan", "sta_plan", "sta_plan_host", "sta_tile_reorder", "sta_tile_unreorder",
     "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
     "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
+    "sta_backward", "sta_attention_backward", "StaAttention",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +47,7 @@ EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
-    "sta_last_error_detail",
+    "sta_last_error_detail", "sta_plan_key_query", "sta_backward",
 )
 
 
@@ -66,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "sta_plan_host": [G, i32, i32, i32p, ctypes.POINTER(vp)],
         "sta_plan_destroy": [vp],
         "sta_plan_query": [vp, i32, i32, i32p, i32, i32p],
+        "sta_plan_key_query": [vp, i32, i32, i32p, i32, i32p],
         "sta_plan_stats": [vp, i64p, i64p],
         "sta_plan_work_items": [vp, i32p, i64, i64p],
         "sta_tile_reorder": [vp, vp, i64, i32, G, vp],
@@ -73,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "sta_forward": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_forward_raster": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
+        "sta_backward": [vp] * 11 + [i32, ctypes.c_float, vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
     }
@@ -172,6 +178,16 @@ class Plan:
         buf = (ctypes.c_int32 * max(count.value, 1))()
         _check(_lib.sta_plan_query(self.handle, head, q_tile, buf, count.value, ctypes.byref(count)),
                "sta_plan_query")
+        return list(buf[:count.value])
+
+    def key_query(self, head: int, k_tile: int) -> list:
+        """Ascending query-tile ids whose window holds key tile ``k_tile`` of ``head``."""
+        count = ctypes.c_int32(0)
+        _check(_lib.sta_plan_key_query(self.handle, head, k_tile, None, 0, ctypes.byref(count)),
+               "sta_plan_key_query")
+        buf = (ctypes.c_int32 * max(count.value, 1))()
+        _check(_lib.sta_plan_key_query(self.handle, head, k_tile, buf, count.value, ctypes.byref(count)),
+               "sta_plan_key_query")
         return list(buf[:count.value])
 
     def stats(self) -> tuple:
@@ -305,6 +321,33 @@ def sta_forward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Te
     return o, lse
 
 
+def sta_backward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                 lse: torch.Tensor, dout: torch.Tensor, softmax_scale: float, dq=None, dk=None, dv=None,
+                 workspace=None, stream=None):
+    """STA backward on tile-major ``[B, H, N, d]`` bf16 tensors (``o`` and ``lse``
+    from ``sta_forward``).  Returns ``(dq, dk, dv)``; outputs and the fp32
+    workspace (``2 * B * H * N`` floats) are allocated when not given."""
+    args = _forward_args(plan, q, k, v, o, lse)
+    B, H, N, d = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    if workspace is None:
+        workspace = torch.empty(2 * B * H * N, dtype=torch.float32, device=q.device)
+    if not workspace.is_cuda or workspace.dtype != torch.float32 or not workspace.is_contiguous() \
+            or workspace.numel() < 2 * B * H * N:
+        raise ValueError(f"workspace must be a contiguous CUDA fp32 tensor of {2 * B * H * N} floats")
+    qp, kp, vp_, op, lp, hd = args
+    _check(_lib.sta_backward(plan.handle, qp, kp, vp_, op, ctypes.c_void_p(dout.data_ptr()), lp,
+                             ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+                             ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(workspace.data_ptr()), hd,
+                             float(softmax_scale), _stream(stream)), "sta_backward")
+    return dq, dk, dv
+
+
 def raster_supported(tile) -> bool:
     """Whether the fused raster path handles this tile shape (see sta.h)."""
     hw = int(tile[1]) * int(tile[2])
@@ -375,3 +418,48 @@ def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
     sta_tile_unreorder(ot, o, lat, tile, stream=stream)
     sta_tile_unreorder(lset, lse, lat, tile, stream=stream)
     return o, lse
+
+
+def sta_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                           lse: torch.Tensor, dout: torch.Tensor, plan: Plan,
+                           softmax_scale: float | None = None, stream=None):
+    """Gradients ``(dq, dk, dv)`` of ``sta_attention`` on raster-order tensors:
+    the inputs are permuted to tile-major order, ``sta_backward`` runs, and the
+    gradients are permuted back."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(q.shape[-1])
+    lat, tile = plan.latent, plan.tile
+
+    def to_tiles(x):
+        y = torch.empty_like(x)
+        sta_tile_reorder(x, y, lat, tile, stream=stream)
+        return y
+
+    qt, kt, vt, ot, dot, lset = (to_tiles(x) for x in (q, k, v, o, dout, lse))
+    dqt, dkt, dvt = sta_backward(plan, qt, kt, vt, ot, lset, dot, softmax_scale, stream=stream)
+    out = []
+    for x in (dqt, dkt, dvt):
+        y = torch.empty_like(x)
+        sta_tile_unreorder(x, y, lat, tile, stream=stream)
+        out.append(y)
+    return tuple(out)
+
+
+class StaAttention(torch.autograd.Function):
+    """``O = StaAttention.apply(q, k, v, plan, softmax_scale)`` on raster-order
+    bf16 tensors, with gradients for q, k and v through ``sta_backward``."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, plan, softmax_scale=None):
+        scale = 1.0 / math.sqrt(q.shape[-1]) if softmax_scale is None else float(softmax_scale)
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = sta_attention(q, k, v, plan, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.plan, ctx.scale = plan, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = sta_attention_backward(q, k, v, o, lse, dout.contiguous(), ctx.plan, ctx.scale)
+        return dq, dk, dv, None, None

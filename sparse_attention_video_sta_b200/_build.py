@@ -11,8 +11,8 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libsta.so")
 
-SOURCES = ["sta_api.cu", "sta_permute.cu", "sta_forward.cu", "sta_noalloc.cu"]
-HEADERS = ["sta_internal.h", "sta_ptx.cuh"]
+SOURCES = ["sta_api.cu", "sta_permute.cu", "sta_forward.cu", "sta_backward.cu", "sta_noalloc.cu"]
+HEADERS = ["sta_internal.h", "sta_ptx.cuh", "sta_wait.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

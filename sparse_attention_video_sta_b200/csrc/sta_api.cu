@@ -166,6 +166,44 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
     std::stable_sort(P.items.begin(), P.items.end(), [&](const WorkItem& a, const WorkItem& b) {
         return list_len[a.win] > list_len[b.win];
     });
+
+    // Backward: transposed lists (query tiles ascending for each key tile).
+    const int32_t tph = P.tiles_per_head;
+    P.tcsr_off.assign(size_t(n_win) * (tph + 1), 0);
+    P.tcsr_ids.assign(P.csr_ids.size(), 0);
+    for (int32_t w = 0; w < n_win; ++w) {
+        const int32_t* off = &P.csr_off[size_t(w) * (tph + 1)];
+        int32_t* toff = &P.tcsr_off[size_t(w) * (tph + 1)];
+        std::vector<int32_t> cnt(tph, 0);
+        for (int32_t q = 0; q < tph; ++q)
+            for (int32_t i = off[q]; i < off[q + 1]; ++i) ++cnt[P.csr_ids[i]];
+        toff[0] = off[0];
+        for (int32_t kt = 0; kt < tph; ++kt) toff[kt + 1] = toff[kt] + cnt[kt];
+        std::vector<int32_t> fill(toff, toff + tph);
+        for (int32_t q = 0; q < tph; ++q)
+            for (int32_t i = off[q]; i < off[q + 1]; ++i) P.tcsr_ids[fill[P.csr_ids[i]]++] = q;
+    }
+    // One-block work lists, longest lists first.
+    P.bq_items.clear();
+    P.bkv_items.clear();
+    for (int32_t b = 0; b < batch; ++b)
+        for (int32_t h = 0; h < heads; ++h) {
+            const int32_t bh = b * heads + h, win = P.head_win[h];
+            for (int32_t blk = 0; blk < tph * S; ++blk) {
+                P.bq_items.push_back(WorkItem{bh, blk, -1, win});
+                P.bkv_items.push_back(WorkItem{bh, blk, -1, win});
+            }
+        }
+    std::stable_sort(P.bq_items.begin(), P.bq_items.end(), [&](const WorkItem& a, const WorkItem& b) {
+        return list_len[a.win] > list_len[b.win];
+    });
+    auto tlen = [&](const WorkItem& it) {
+        const int32_t* toff = &P.tcsr_off[size_t(it.win) * (tph + 1)];
+        const int32_t kt = it.qa / S;
+        return toff[kt + 1] - toff[kt];
+    };
+    std::stable_sort(P.bkv_items.begin(), P.bkv_items.end(),
+                     [&](const WorkItem& a, const WorkItem& b) { return tlen(a) > tlen(b); });
     return STA_OK;
 }
 
@@ -175,6 +213,14 @@ void free_device(sta_plan_s* p) {
     if (p->d_items) cudaFree(p->d_items);
     if (p->d_status) cudaFree(p->d_status);
     if (p->d_origin) cudaFree(p->d_origin);
+    if (p->d_toff) cudaFree(p->d_toff);
+    if (p->d_tids) cudaFree(p->d_tids);
+    if (p->d_bq_items) cudaFree(p->d_bq_items);
+    if (p->d_bkv_items) cudaFree(p->d_bkv_items);
+    p->d_toff = nullptr;
+    p->d_tids = nullptr;
+    p->d_bq_items = nullptr;
+    p->d_bkv_items = nullptr;
     p->d_off = nullptr;
     p->d_ids = nullptr;
     p->d_items = nullptr;
@@ -275,6 +321,10 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
     if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
+    if (e == cudaSuccess) e = upload(&p->d_toff, p->h.tcsr_off, s);
+    if (e == cudaSuccess) e = upload(&p->d_tids, p->h.tcsr_ids, s);
+    if (e == cudaSuccess) e = upload(&p->d_bq_items, p->h.bq_items, s);
+    if (e == cudaSuccess) e = upload(&p->d_bkv_items, p->h.bkv_items, s);
     if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&p->d_status), sizeof(uint32_t));
     if (e == cudaSuccess) e = cudaMemsetAsync(p->d_status, 0, sizeof(uint32_t), s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
@@ -293,7 +343,8 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin) {
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_toff ||
+        p->d_tids || p->d_bq_items || p->d_bkv_items) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
         free_device(p);
     }
@@ -312,6 +363,20 @@ sta_status sta_plan_query(sta_plan_t p, int32_t head, int32_t q_tile, int32_t* k
     const int32_t n = off[q_tile + 1] - off[q_tile];
     *count = n;
     for (int32_t i = 0; i < std::min(n, cap); ++i) kv_ids[i] = P.csr_ids[off[q_tile] + i];
+    return STA_OK;
+}
+
+sta_status sta_plan_key_query(sta_plan_t p, int32_t head, int32_t k_tile, int32_t* q_ids,
+                              int32_t cap, int32_t* count) {
+    if (p == nullptr || count == nullptr || cap < 0 || (cap > 0 && q_ids == nullptr))
+        return STA_ERR_INVALID_ARG;
+    const PlanHost& P = p->h;
+    if (head < 0 || head >= P.heads || k_tile < 0 || k_tile >= P.tiles_per_head)
+        return STA_ERR_INVALID_ARG;
+    const int32_t* off = &P.tcsr_off[size_t(P.head_win[head]) * (P.tiles_per_head + 1)];
+    const int32_t n = off[k_tile + 1] - off[k_tile];
+    *count = n;
+    for (int32_t i = 0; i < std::min(n, cap); ++i) q_ids[i] = P.tcsr_ids[off[k_tile] + i];
     return STA_OK;
 }
 
@@ -355,6 +420,24 @@ sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v
 sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k, const void* v, void* o,
                               float* lse, int32_t head_dim, float softmax_scale, void* stream) {
     return forward_common(p, q, k, v, o, lse, head_dim, softmax_scale, stream, true);
+}
+
+sta_status sta_backward(sta_plan_t p, const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        float* workspace, int32_t head_dim, float softmax_scale, void* stream) {
+    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    const void* in16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+    for (const void* x : in16)
+        if (x == nullptr || !aligned(x, 16)) return STA_ERR_INVALID_ARG;
+    if (lse == nullptr || !aligned(lse, 4)) return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
+    if (dev != p->device) return STA_ERR_INVALID_ARG;
+    return cuda_status(sta::launch_backward(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim,
+                                            softmax_scale, static_cast<cudaStream_t>(stream),
+                                            kDefaultTimeoutNs));
 }
 
 sta_status sta_last_device_status(sta_plan_t p, void* stream) {

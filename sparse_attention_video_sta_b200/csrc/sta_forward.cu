@@ -40,6 +40,7 @@
 
 #include "sta_internal.h"
 #include "sta_ptx.cuh"
+#include "sta_wait.cuh"
 
 namespace sta {
 namespace {
@@ -144,30 +145,10 @@ __device__ __forceinline__ int64_t out_row(const FwdParams& p, int32_t bh, int32
     return int64_t(bh) * p.tokens + token;
 }
 
-// Bounded mbarrier wait.  Returns false when the CTA is aborting (another role
-// gave up) or when this wait ran past the time limit (then it starts the abort).
+// Bounded wait with this launch's status word and time limit.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          const FwdParams& p) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = ptx::globaltimer_ns();
-    while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (ptx::mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (ptx::globaltimer_ns() - t0 > p.timeout_ns) {
-            *abort_flag = 1;
-            atomicOr(p.status, kDevTimeout);
-            return false;
-        }
-    }
-}
-
-// Drain wait used on the way out: bounded, never starts an abort.
-__device__ __forceinline__ void drain_bar(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
-    const uint64_t t0 = ptx::globaltimer_ns();
-    while (!ptx::mbar_try_wait(bar, parity)) {
-        if (ptx::globaltimer_ns() - t0 > limit_ns) return;
-    }
+    return wait_bar_limited(bar, parity, abort_flag, p.status, p.timeout_ns);
 }
 
 // P = exp2(S * c - m * c) for one 128-score row, packed to bf16 pairs; returns

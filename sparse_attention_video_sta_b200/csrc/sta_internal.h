@@ -39,7 +39,14 @@ struct PlanHost {
     std::vector<int32_t> win_ext;            // [n_win][3] clamped extents in tiles
     std::vector<int32_t> csr_off;            // [n_win][tiles_per_head + 1], global offsets
     std::vector<int32_t> csr_ids;            // key-tile ids, ascending per list
-    std::vector<WorkItem> items;             // work list
+    std::vector<WorkItem> items;             // forward work list
+    // Backward: for each key tile the query tiles whose window holds it
+    // (the forward lists transposed), and one-block work lists for the dQ
+    // kernel (qa = query block) and the dK/dV kernel (qa = key block).
+    std::vector<int32_t> tcsr_off;           // [n_win][tiles_per_head + 1], global offsets
+    std::vector<int32_t> tcsr_ids;           // query-tile ids, ascending per list
+    std::vector<WorkItem> bq_items;
+    std::vector<WorkItem> bkv_items;
     std::vector<int32_t> tile_origin;        // [tiles_per_head][4]: raster (w, h, t) origin of each tile, 0
     int64_t computed_pairs = 0;              // B * sum_h sum_q |list|
 };
@@ -55,6 +62,10 @@ struct sta_plan_s {
     sta::WorkItem* d_items = nullptr;
     uint32_t* d_status = nullptr;
     int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
+    int32_t* d_toff = nullptr;
+    int32_t* d_tids = nullptr;
+    sta::WorkItem* d_bq_items = nullptr;
+    sta::WorkItem* d_bkv_items = nullptr;
 };
 
 namespace sta {
@@ -92,6 +103,13 @@ struct RawPlanView {
 cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void* k, const void* v,
                                void* o, float* lse, int head_dim, float softmax_scale,
                                cudaStream_t stream);
+
+// Backward launches (sta_backward.cu): the D / log2-LSE pass, then the dQ and
+// dK / dV kernels, on tile-major tensors.  Returns a CUDA error code.
+cudaError_t launch_backward(const sta_plan_s* p, const void* q, const void* k, const void* v,
+                            const void* o, const void* dout, const float* lse, void* dq, void* dk,
+                            void* dv, float* workspace, int head_dim, float softmax_scale,
+                            cudaStream_t stream, uint64_t timeout_ns);
 
 // Permutation launch (sta_permute.cu).  inverse = false: raster -> tile-major.
 cudaError_t launch_permute(const void* src, void* dst, int64_t outer, int32_t row_bytes,

@@ -84,3 +84,37 @@ def oracle_rows(q, k, v, latent, tile, windows, scale, bhs, tokens):
     rows = np.array([(bh, t) for bh in bhs for t in tokens], dtype=np.int64)
     o, lse = oracle.sta_attention(q, k, v, latent, tile, windows, scale, rows=rows)
     return rows, o, lse
+
+
+# Gradients (dQ, dK, dV) of the backward pass, per (b, h) slice with rms the
+# root mean square of the reference slice:
+#   |delta| <= 3e-2 rms + 2^-8 |ref| element-wise, mean |delta| <= 3e-3 rms.
+# Derivation: P and dS enter the tensor-core products as bf16 (relative
+# rounding up to 2^-9 per term, errors of random sign that add up to about
+# 2^-9 / sqrt(3) of the rms), D uses the forward's bf16 output, and the
+# gradients are rounded to bf16 (up to 2^-9 |ref|).  A CPU emulation of that
+# arithmetic against the fp64 oracle on the tiny workload gives max
+# (|delta| - 2^-8 |ref|) / rms = 1.6e-2 and mean |delta| / rms = 1.8e-3.
+GRAD_RMS_TOL = 3e-2
+GRAD_REL = 2.0 ** -8
+GRAD_MEAN_TOL = 3e-3
+
+
+def compare_grad(got, ref: np.ndarray, bh: np.ndarray, what: str = ""):
+    """got, ref: [R, d] rows; bh: [R] slice id of each row.  Asserts the
+    gradient tolerances per slice; returns the worst (max/rms, mean/rms)."""
+    g = got.detach().cpu().to(torch.float64).numpy() if hasattr(got, "detach") else np.asarray(got)
+    assert np.all(np.isfinite(g)), what
+    worst = (0.0, 0.0)
+    for s in np.unique(bh):
+        sel = bh == s
+        r, a = ref[sel], g[sel]
+        rms = float(np.sqrt(np.mean(r * r)))
+        e = np.abs(a - r)
+        assert rms > 0, (what, int(s))
+        excess = float(np.max(e - GRAD_REL * np.abs(r))) / rms
+        mean = float(np.mean(e)) / rms
+        assert excess <= GRAD_RMS_TOL, (what, int(s), "max excess / rms", excess)
+        assert mean <= GRAD_MEAN_TOL, (what, int(s), "mean / rms", mean)
+        worst = (max(worst[0], excess), max(worst[1], mean))
+    return worst

@@ -161,3 +161,34 @@ def test_work_list_covers_every_row_block_once():
         assert lens == sorted(lens, reverse=True)  # longest lists first
         pairs, n_items = p.stats()
         assert n_items == len(items)
+
+
+@pytest.mark.parametrize("idx", [1, 2, 3])
+def test_key_lists_are_transposed_query_lists(idx):
+    """sta_plan_key_query(kt) lists exactly the query tiles whose oracle mask
+    attends tile kt (the backward's dK / dV kernel walks these lists)."""
+    w = sta_inputs.WORKLOADS[idx]
+    wins = sta_inputs.windows(w).tolist()
+    p = sta.sta_plan_host(w.latent, w.tile, w.batch, w.heads, wins)
+    n_tiles = p.tiles_per_head
+    distinct = {}
+    for h, win in enumerate(wins):
+        distinct.setdefault(tuple(win), h)
+    for win, h in distinct.items():
+        attends = [set(oracle_tile_set(w.latent, w.tile, win, q)) for q in range(n_tiles)]
+        for kt in range(n_tiles):
+            expect = [q for q in range(n_tiles) if kt in attends[q]]
+            assert p.key_query(h, kt) == expect, (idx, win, kt)
+
+
+def test_backward_rejected_before_launch():
+    INV = sta.STA_ERR_INVALID_ARG
+    lib = sta._lib
+    hp = sta.sta_plan_host((18, 24, 24), (6, 8, 8), 1, 2, [(12, 16, 16)] * 2)
+    a = ctypes.c_void_p(1 << 30)
+    args = [a] * 10
+    assert lib.sta_backward(hp.handle, *args, 64, 0.125, None) == INV  # host-only plan
+    assert lib.sta_backward(None, *args, 64, 0.125, None) == INV
+    assert lib.sta_plan_key_query(hp.handle, 0, 27, None, 0, ctypes.byref(ctypes.c_int32())) == INV
+    assert lib.sta_plan_key_query(hp.handle, 2, 0, None, 0, ctypes.byref(ctypes.c_int32())) == INV
+    hp.destroy()
