@@ -56,7 +56,9 @@ def parse():
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for profiling only)")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip e2e, full-window, permutation and CPU-baseline legs")
+                    help="skip e2e, full-window, permutation, backward and CPU-baseline legs")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward pass (for profiling) and print its figures")
     return ap.parse_args()
 
 
@@ -239,6 +241,39 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def time_backward(sta, plan, forward, qt, kt, vt, ot, lset, scale, gen, flops, warmup, reps, reduce_max):
+    """Time sta_backward on the tile-major tensors after one forward; returns
+    its figures.  Algorithmic work: five tile-pair products (S, dP, dV, dK, dQ)
+    against the forward's two."""
+    forward()
+    dout = torch.empty_like(qt)
+    B, H, N, d = qt.shape
+    for b in range(B):
+        for h in range(H):
+            dout[b, h].copy_(torch.randn((N, d), generator=gen, device=qt.device, dtype=torch.float32))
+    dq, dk, dv = (torch.empty_like(qt) for _ in range(3))
+    ws = torch.empty(2 * B * H * N, dtype=torch.float32, device=qt.device)
+
+    def bwd_step():
+        sta.sta_backward(plan, qt, kt, vt, ot, lset, dout, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(warmup):
+        bwd_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        bwd_step()
+    e1.record()
+    torch.cuda.synchronize()
+    bwd_ms = reduce_max(e0.elapsed_time(e1) / reps)
+    if sta.sta_last_device_status(plan) != 0:
+        raise RuntimeError("device status error in the backward run")
+    bwd_flops = 2.5 * flops
+    return {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12, "flops": bwd_flops,
+            "launches": 3, "layout": "tile-major"}
+
+
 def main():
     args = parse()
     w = sta_inputs.WORKLOADS[args.workload]
@@ -310,6 +345,13 @@ def main():
         sta.sta_forward(plan, qt, kt, vt, ot, lset, scale)
         sta.sta_tile_unreorder(ot, o, L, T)
         sta.sta_tile_unreorder(lset, lse, L, T, token_dim=2)
+
+    if args.backward_only:
+        res = time_backward(sta, plan, permuted_step, qt, kt, vt, ot, lset, scale, gen, flops,
+                            max(3, args.warmup), args.steps, reduce_max)
+        if rank == 0:
+            print(json.dumps({"workload": w.name, "backward": res}), flush=True)
+        return
 
     launches_per_step = 1
     for _ in range(max(3, args.warmup)):
@@ -396,35 +438,8 @@ def main():
                                  "bytes_per_launch": 2 * nbytes}
         extras["permutation"]["frac"] = extras["permutation"]["gbs"] / extras["permutation"]["peak_gbs"]
         # ------------------------------------------- backward (tile-major, 3 launches)
-        permuted_step()
-        dout = torch.empty_like(q)
-        for b in range(B):
-            for h in range(H):
-                dout[b, h].copy_(torch.randn((N, d), generator=gen, device=dev, dtype=torch.float32))
-        dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-        ws = torch.empty(2 * B * H * N, dtype=torch.float32, device=dev)
-
-        def bwd_step():
-            sta.sta_backward(plan, qt, kt, vt, ot, lset, dout, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
-
-        for _ in range(2):
-            bwd_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 3
-        e0.record()
-        for _ in range(reps):
-            bwd_step()
-        e1.record()
-        torch.cuda.synchronize()
-        bwd_ms = reduce_max(e0.elapsed_time(e1) / reps)
-        if sta.sta_last_device_status(plan) != 0:
-            raise RuntimeError("device status error in the backward run")
-        # algorithmic work: five tile-pair products (S, dP, dV, dK, dQ) against the forward's two
-        bwd_flops = 2.5 * flops
-        extras["backward"] = {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12, "flops": bwd_flops,
-                              "launches": 3, "layout": "tile-major"}
-        del dout, dq, dk, dv, ws
+        extras["backward"] = time_backward(sta, plan, permuted_step, qt, kt, vt, ot, lset, scale, gen,
+                                           flops, 2, 3, reduce_max)
         # ------------------------------------------- end to end from pinned host memory
         hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
         ho = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
