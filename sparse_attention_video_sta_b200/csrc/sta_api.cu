@@ -57,8 +57,36 @@ int32_t window_start(int32_t q, int32_t e, int32_t n) {
     return std::min(std::max(q - e / 2, 0), n - e);
 }
 
+// Order one-block work items for a persistent grid of `ctas` CTAs, CTA c
+// taking items c, c + ctas, c + 2 ctas, ...: the items stay in natural
+// (head, block) order round by round, so the CTAs work on neighbouring tiles
+// of one head at the same time and share their K/V (or Q/dO) tiles in L2;
+// inside each round the longest items go to the CTAs with the least work so
+// far, which keeps the CTAs' totals level when list lengths vary.
+template <class Len>
+void order_rounds(std::vector<WorkItem>& items, const Len& len, int32_t ctas) {
+    if (ctas < 1) ctas = 1;
+    std::vector<int64_t> load(size_t(ctas), 0);
+    std::vector<WorkItem> out(items.size());
+    for (size_t r0 = 0; r0 < items.size(); r0 += size_t(ctas)) {
+        const size_t n = std::min(size_t(ctas), items.size() - r0);
+        std::vector<size_t> idx(n), slot(n);
+        for (size_t i = 0; i < n; ++i) idx[i] = slot[i] = i;
+        std::stable_sort(idx.begin(), idx.end(),
+                         [&](size_t a, size_t b) { return len(items[r0 + a]) > len(items[r0 + b]); });
+        std::stable_sort(slot.begin(), slot.end(), [&](size_t a, size_t b) { return load[a] < load[b]; });
+        for (size_t i = 0; i < n; ++i) {
+            out[r0 + slot[i]] = items[r0 + idx[i]];
+            load[slot[i]] += len(items[r0 + idx[i]]);
+        }
+    }
+    items.swap(out);
+}
+
+// `ctas`: the persistent grid the backward work lists are ordered for (the
+// device's SM count; 148 for host-only plans).
 sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
-                           const int32_t* window_thw, PlanHost& P) {
+                           const int32_t* window_thw, int32_t ctas, PlanHost& P) {
     if (!geom_valid(g) || batch < 1 || heads < 1 || window_thw == nullptr)
         return STA_ERR_INVALID_ARG;
     const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
@@ -183,7 +211,7 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
         for (int32_t q = 0; q < tph; ++q)
             for (int32_t i = off[q]; i < off[q + 1]; ++i) P.tcsr_ids[fill[P.csr_ids[i]]++] = q;
     }
-    // One-block work lists, longest lists first.
+    // One-block work lists (ordered for the persistent grid below).
     P.bq_items.clear();
     P.bkv_items.clear();
     for (int32_t b = 0; b < batch; ++b)
@@ -194,16 +222,14 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
                 P.bkv_items.push_back(WorkItem{bh, blk, -1, win});
             }
         }
-    std::stable_sort(P.bq_items.begin(), P.bq_items.end(), [&](const WorkItem& a, const WorkItem& b) {
-        return list_len[a.win] > list_len[b.win];
-    });
+    auto qlen = [&](const WorkItem& it) { return int64_t(list_len[it.win]); };
     auto tlen = [&](const WorkItem& it) {
         const int32_t* toff = &P.tcsr_off[size_t(it.win) * (tph + 1)];
         const int32_t kt = it.qa / S;
-        return toff[kt + 1] - toff[kt];
+        return int64_t(toff[kt + 1] - toff[kt]);
     };
-    std::stable_sort(P.bkv_items.begin(), P.bkv_items.end(),
-                     [&](const WorkItem& a, const WorkItem& b) { return tlen(a) > tlen(b); });
+    order_rounds(P.bq_items, qlen, ctas);
+    order_rounds(P.bkv_items, tlen, ctas);
     return STA_OK;
 }
 
@@ -274,6 +300,28 @@ sta_status forward_common(sta_plan_t p, const void* q, const void* k, const void
                                            static_cast<cudaStream_t>(stream), inject, limit, raster));
 }
 
+constexpr int32_t kHostPlanCtas = 148;  // B200 SM count, for plans built without a device
+
+sta_status plan_host_for(const sta_geom* g, int32_t batch, int32_t heads, const int32_t* window_thw,
+                         int32_t ctas, sta_plan_t* out) {
+    if (out == nullptr) return STA_ERR_INVALID_ARG;
+    *out = nullptr;
+    sta_plan_s* p = new (std::nothrow) sta_plan_s();
+    if (p == nullptr) return STA_ERR_OOM;
+    sta_status st;
+    try {
+        st = build_plan_host(g, batch, heads, window_thw, ctas, p->h);
+    } catch (const std::bad_alloc&) {
+        st = STA_ERR_OOM;
+    }
+    if (st != STA_OK) {
+        delete p;
+        return st;
+    }
+    *out = p;
+    return STA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -292,27 +340,16 @@ const char* sta_status_string(sta_status s) {
 
 sta_status sta_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
                          const int32_t* window_thw, sta_plan_t* out) {
-    if (out == nullptr) return STA_ERR_INVALID_ARG;
-    *out = nullptr;
-    sta_plan_s* p = new (std::nothrow) sta_plan_s();
-    if (p == nullptr) return STA_ERR_OOM;
-    sta_status st;
-    try {
-        st = build_plan_host(g, batch, heads, window_thw, p->h);
-    } catch (const std::bad_alloc&) {
-        st = STA_ERR_OOM;
-    }
-    if (st != STA_OK) {
-        delete p;
-        return st;
-    }
-    *out = p;
-    return STA_OK;
+    return plan_host_for(g, batch, heads, window_thw, kHostPlanCtas, out);
 }
 
 sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
                     const int32_t* window_thw, void* stream, sta_plan_t* out) {
-    sta_status st = sta_plan_host(g, batch, heads, window_thw, out);
+    int dev = -1, sms = 0;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
+    if (cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess)
+        return cuda_status(e);
+    sta_status st = plan_host_for(g, batch, heads, window_thw, sms, out);
     if (st != STA_OK) return st;
     sta_plan_s* p = *out;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

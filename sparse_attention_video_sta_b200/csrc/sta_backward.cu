@@ -660,8 +660,9 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     break;
                 }
                 ptx::tc_fence_after();
-                const float2* cl = reinterpret_cast<const float2*>(smem + (stage(r) - base) + C::kStL) + 32 * h;
-                const float2* cd = reinterpret_cast<const float2*>(smem + (stage(r) - base) + C::kStD) + 32 * h;
+                // per-column constants, 16-byte broadcast loads
+                const float4* cl = reinterpret_cast<const float4*>(smem + (stage(r) - base) + C::kStL) + 16 * h;
+                const float4* cd = reinterpret_cast<const float4*>(smem + (stage(r) - base) + C::kStD) + 16 * h;
                 const uint32_t ts = tmem + lane_addr + C::kColS + 64u * h;
                 float pr[64];
                 uint32_t pk[32];
@@ -669,14 +670,19 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     uint32_t sr[64];
                     ptx::tmem_ld64(ts, sr);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float2 l = cl[i];
-                        float x0, x1;
-                        ptx::f2_split(ptx::f2_fma(ptx::f2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                    for (int i = 0; i < 16; ++i) {
+                        const float4 l = cl[i];
+                        float x0, x1, x2, x3;
+                        ptx::f2_split(ptx::f2_fma(ptx::f2(__uint_as_float(sr[4 * i]), __uint_as_float(sr[4 * i + 1])),
                                                   c2, ptx::f2(l.x, l.y)),
                                       x0, x1);
-                        pr[2 * i] = ptx::ex2(x0);
-                        pr[2 * i + 1] = ptx::ex2(x1);
+                        ptx::f2_split(ptx::f2_fma(ptx::f2(__uint_as_float(sr[4 * i + 2]), __uint_as_float(sr[4 * i + 3])),
+                                                  c2, ptx::f2(l.z, l.w)),
+                                      x2, x3);
+                        pr[4 * i] = ptx::ex2(x0);
+                        pr[4 * i + 1] = ptx::ex2(x1);
+                        pr[4 * i + 2] = ptx::ex2(x2);
+                        pr[4 * i + 3] = ptx::ex2(x3);
                     }
                 }
                 pack64(pr, pk);
@@ -695,15 +701,21 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     uint32_t dr[64];
                     ptx::tmem_ld64(tdp, dr);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float2 dd = cd[i];
-                        float t0, t1;
-                        ptx::f2_split(ptx::f2_mul(ptx::f2(pr[2 * i], pr[2 * i + 1]),
-                                                  ptx::f2_add(ptx::f2(__uint_as_float(dr[2 * i]),
-                                                                      __uint_as_float(dr[2 * i + 1])),
+                    for (int i = 0; i < 16; ++i) {
+                        const float4 dd = cd[i];
+                        float t0, t1, t2, t3;
+                        ptx::f2_split(ptx::f2_mul(ptx::f2(pr[4 * i], pr[4 * i + 1]),
+                                                  ptx::f2_add(ptx::f2(__uint_as_float(dr[4 * i]),
+                                                                      __uint_as_float(dr[4 * i + 1])),
                                                               ptx::f2(dd.x, dd.y))),
                                       t0, t1);
-                        pk[i] = ptx::pack_bf16x2(t0, t1);
+                        ptx::f2_split(ptx::f2_mul(ptx::f2(pr[4 * i + 2], pr[4 * i + 3]),
+                                                  ptx::f2_add(ptx::f2(__uint_as_float(dr[4 * i + 2]),
+                                                                      __uint_as_float(dr[4 * i + 3])),
+                                                              ptx::f2(dd.z, dd.w))),
+                                      t2, t3);
+                        pk[2 * i] = ptx::pack_bf16x2(t0, t1);
+                        pk[2 * i + 1] = ptx::pack_bf16x2(t2, t3);
                     }
                 }
                 ptx::tmem_st32(tdp, pk);
