@@ -391,6 +391,7 @@ def main():
     e2e = None
     if not args.no_extras:
         # ------------------------------------------- full-window denominator
+        o_win, lse_win = o.clone(), lse.clone()  # the timed step's output (the STA window)
         full = sta.sta_plan(L, T, B, H, [tuple(L)] * H)
         for _ in range(2):
             sta.sta_forward_raster(full, q, k, v, o, lse, scale)
@@ -410,6 +411,21 @@ def main():
         if sta.sta_last_device_status(full) != 0:
             raise RuntimeError("device status error in the full-window run")
         full.destroy()
+        # ------------------------------------------- window-search statistics (recall, output error)
+        sta.sta_window_stats(lse_win, lse, o_win, o)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            recall, err = sta.sta_window_stats(lse_win, lse, o_win, o)
+        e1.record()
+        torch.cuda.synchronize()
+        st_ms = e0.elapsed_time(e1) / 3
+        st_bytes = 2 * o.numel() * o.element_size() + 2 * lse.numel() * lse.element_size()
+        extras["window_stats"] = {"ms": st_ms, "gbs": st_bytes / (st_ms * 1e-3) / 1e9, "bytes": st_bytes,
+                                  "window": list(wins[0]), "recall_mean": float(recall.mean()),
+                                  "recall_min_head": float(recall.mean(dim=0).min()),
+                                  "mse_mean": float(err.mean())}
+        del o_win, lse_win
         # ------------------------------------------- unfused pipeline
         for _ in range(2):
             permuted_step()

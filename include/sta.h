@@ -190,6 +190,30 @@ STA_API sta_status sta_backward(sta_plan_t p, const void* q, const void* k, cons
                                 void* dk, void* dv, float* workspace, int32_t head_dim,
                                 float softmax_scale, void* stream);
 
+/* Per-(b, h) statistics of a candidate window against the full window, for
+ * choosing a window per head by profiling ("Fast Video Generation with Sliding
+ * Tile Attention": podcast transcript at hotaipapers.com, segments on the 3D
+ * locality pattern and on head specialisation; dianyo.github.io ICML-2025
+ * post, STA section, "Observation & Proposed Method").
+ *   lse_w, lse_full : device fp32 [slices, tokens]: the forward's LSE with the
+ *                     candidate window and with a window covering the volume
+ *   o_w, o_full     : device bf16 [slices, tokens, head_dim], the matching
+ *                     outputs, 16-byte aligned; any token order, the same in
+ *                     all four tensors
+ *   recall          : device fp64 [slices] (written): mean over rows of
+ *                     exp(lse_w - lse_full), the attention recall, i.e. the
+ *                     share of each row's full-attention softmax mass that the
+ *                     window keeps
+ *   mse             : device fp64 [slices] (written): mean of (o_w - o_full)^2
+ *                     over rows and channels (the mask-search loss, read here
+ *                     as the output's mean squared error against full attention)
+ * 1 <= slices (B * heads) <= 2^28, tokens >= 1, head_dim a positive multiple
+ * of 8, else INVALID_ARG.  One kernel (a cluster of 8 CTAs per slice),
+ * deterministic; allocates nothing. */
+STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, const void* o_w,
+                                    const void* o_full, int64_t slices, int64_t tokens, int32_t head_dim,
+                                    double* recall, double* mse, void* stream);
+
 /* STA forward that allocates nothing (this call has no counterpart in the
  * paper; it exists for deployment).
  *

@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
             L.ora_sta_backward_dq.restype = ctypes.c_int
             L.ora_sta_backward_dkdv.argtypes = bw + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
             L.ora_sta_backward_dkdv.restype = ctypes.c_int
+            L.ora_window_recall.argtypes = [ctypes.c_void_p, ctypes.c_void_p, G, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_int32, i32p, ctypes.c_float, ctypes.c_void_p,
+                                            ctypes.c_int64, ctypes.c_void_p, ctypes.c_int32]
+            L.ora_window_recall.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -265,3 +269,26 @@ def sta_backward(q, k, v, dout, latent, tile, windows, softmax_scale: float,
     dq = sta_backward_dq(q, k, v, dout, latent, tile, windows, softmax_scale, nthreads=nthreads)
     dk, dv = sta_backward_dkdv(q, k, v, dout, latent, tile, windows, softmax_scale, nthreads=nthreads)
     return dq, dk, dv
+
+
+def window_recall(q, k, latent, tile, windows, softmax_scale: float, rows=None,
+                  nthreads: int | None = None) -> np.ndarray:
+    """Attention recall of query rows: the share of each row's full-attention
+    softmax mass on the keys its STA window attends.  ``rows`` as in
+    ``sta_attention``; default every row, returned as ``[B, H, N]``."""
+    qa, ka = _as_u16(q), _as_u16(k)
+    if qa.ndim != 4 or qa.shape != ka.shape:
+        raise ValueError("oracle: q, k must share a [B, H, N, d] shape")
+    B, H, N, d = qa.shape
+    if N != num_tokens(latent):
+        raise ValueError("oracle: N does not match the latent")
+    win = np.ascontiguousarray(np.asarray(windows, dtype=np.int32).reshape(H, 3))
+    rows_a, full = _rows_or_all(rows, B, H, N)
+    out = np.empty((rows_a.shape[0],), dtype=np.float64)
+    r = lib().ora_window_recall(qa.ctypes.data, ka.ctypes.data, ctypes.byref(_geom(latent, tile)), B, H, d,
+                                win.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), float(softmax_scale),
+                                rows_a.ctypes.data, rows_a.shape[0], out.ctypes.data,
+                                int(nthreads or max(1, os.cpu_count() or 1)))
+    if r != 0:
+        raise ValueError(f"oracle: ora_window_recall failed with status {r}")
+    return out.reshape(B, H, N) if full else out

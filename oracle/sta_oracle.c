@@ -598,3 +598,70 @@ int ora_sta_backward_dkdv(const uint16_t* q, const uint16_t* k, const uint16_t* 
     free(stat);
     return st;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Attention recall                                                           */
+/* ------------------------------------------------------------------------ */
+/*
+ * "Attention recall" of a query row (page 1, the segment on the 3D locality
+ * pattern; page 4, "Observation & Proposed Method"): the share of the row's
+ * full-attention softmax mass that falls on the keys inside the local window.
+ * Written out: with s_j = scale q . k_j over all N keys,
+ *
+ *   recall_i = sum_{j in A_i} exp(s_j) / sum_{j} exp(s_j)
+ *
+ * where A_i is the STA key set of row i (the token mask above).
+ */
+static void* recall_worker(void* arg)
+{
+    ora_bjob* job = (ora_bjob*)arg;
+    const int64_t n_tok = ora_num_tokens(job->g);
+    const int32_t d = job->d;
+    double* score = (double*)malloc(sizeof(double) * (size_t)n_tok);
+    double* qrow = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!score || !qrow) {
+        bjob_fail(job, ORA_NO_MEM);
+        free(score); free(qrow);
+        return NULL;
+    }
+    for (;;) {
+        int64_t r = bjob_take(job);
+        if (r >= job->nitems) break;
+        int64_t bh = job->items[2 * r], qi = job->items[2 * r + 1];
+        const int32_t* win = job->win + 3 * (bh % job->heads);
+        load_row(job->q, bh, qi, n_tok, d, qrow);
+        const uint16_t* kbase = job->k + bh * n_tok * d;
+        double m = -INFINITY;
+        for (int64_t j = 0; j < n_tok; ++j) {
+            score[j] = job->scale * dot_bf16(qrow, kbase + j * d, d);
+            if (score[j] > m) m = score[j];
+        }
+        double all = 0.0, inside = 0.0;
+        for (int64_t j = 0; j < n_tok; ++j) {
+            double w = exp(score[j] - m);
+            all += w;
+            if (key_allowed(job->g, win, qi, j)) inside += w;
+        }
+        job->out_a[r] = inside / all;
+    }
+    free(score); free(qrow);
+    return NULL;
+}
+
+/* Attention recall of an explicit list of query rows (bh, raster token):
+ * out_recall[r] in (0, 1].  q and k as for ora_sta_attention. */
+int ora_window_recall(const uint16_t* q, const uint16_t* k, const ora_geom* g, int64_t batch, int64_t heads,
+                      int32_t d, const int32_t* win, float softmax_scale, const int64_t* rows, int64_t nrows,
+                      double* out_recall, int32_t nthreads)
+{
+    ora_bjob job;
+    /* v and dout are not used: pass q so the argument checks see non-null pointers */
+    int st = bjob_init(&job, q, k, q, q, g, batch, heads, d, win, softmax_scale, rows, nrows);
+    if (st != ORA_OK) return st;
+    if (!out_recall || nthreads <= 0) return ORA_BAD_ARG;
+    job.out_a = out_recall;
+    pthread_mutex_init(&job.lock, NULL);
+    st = run_bjob(&job, recall_worker, nthreads);
+    pthread_mutex_destroy(&job.lock);
+    return st;
+}

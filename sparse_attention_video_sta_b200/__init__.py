@@ -17,6 +17,8 @@ The functions carry the C names:
 
 ``sta_attention`` / ``sta_attention_backward`` chain them for raster-order
 tensors, and ``StaAttention`` wraps both as a ``torch.autograd.Function``.
+``sta_window_stats`` / ``sta_window_search`` profile candidate windows per head
+(attention recall and output error against full attention).
 """
 from __future__ import annotations
 
@@ -30,7 +32,7 @@ __all__ = [
     "StaError", "Plan", "sta_plan", "sta_plan_host", "sta_tile_reorder", "sta_tile_unreorder",
     "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
     "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
-    "sta_backward", "sta_attention_backward", "StaAttention",
+    "sta_backward", "sta_attention_backward", "StaAttention", "sta_window_stats", "sta_window_search",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -47,7 +49,7 @@ EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
-    "sta_last_error_detail", "sta_plan_key_query", "sta_backward",
+    "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
 )
 
 
@@ -79,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "sta_forward_raster": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_backward": [vp] * 11 + [i32, ctypes.c_float, vp],
+        "sta_window_stats": [vp, vp, vp, vp, i64, i64, i32, vp, vp, vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
     }
@@ -463,3 +466,70 @@ class StaAttention(torch.autograd.Function):
         q, k, v, o, lse = ctx.saved_tensors
         dq, dk, dv = sta_attention_backward(q, k, v, o, lse, dout.contiguous(), ctx.plan, ctx.scale)
         return dq, dk, dv, None, None
+
+
+def sta_window_stats(lse_w: torch.Tensor, lse_full: torch.Tensor, o_w: torch.Tensor, o_full: torch.Tensor,
+                     stream=None):
+    """Per-(b, h) attention recall (mean of exp(lse_w - lse_full)) and output
+    mean squared error of a candidate window against the full window.
+    Returns ``(recall, mse)``, fp64 CUDA tensors of shape ``[B, H]``."""
+    if o_w.shape != o_full.shape or lse_w.shape != lse_full.shape or tuple(lse_w.shape) != tuple(o_w.shape[:3]):
+        raise ValueError("o_w / o_full must be [B, H, N, d] and lse_w / lse_full [B, H, N], matching")
+    for name, t, dt in (("lse_w", lse_w, torch.float32), ("lse_full", lse_full, torch.float32),
+                        ("o_w", o_w, torch.bfloat16), ("o_full", o_full, torch.bfloat16)):
+        if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
+    B, H, N, d = o_w.shape
+    recall = torch.empty((B, H), dtype=torch.float64, device=o_w.device)
+    mse = torch.empty_like(recall)
+    _check(_lib.sta_window_stats(ctypes.c_void_p(lse_w.data_ptr()), ctypes.c_void_p(lse_full.data_ptr()),
+                                 ctypes.c_void_p(o_w.data_ptr()), ctypes.c_void_p(o_full.data_ptr()),
+                                 B * H, N, d, ctypes.c_void_p(recall.data_ptr()),
+                                 ctypes.c_void_p(mse.data_ptr()), _stream(stream)), "sta_window_stats")
+    return recall, mse
+
+
+def sta_window_search(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, latent, tile, candidates,
+                      softmax_scale: float | None = None, max_mse: float | None = None,
+                      min_recall: float | None = None, stream=None) -> dict:
+    """Profile candidate windows per head on raster-order inputs and pick one.
+
+    For every candidate (a window in tokens, used for all heads) the STA
+    forward runs once, and once with a window covering the volume;
+    ``sta_window_stats`` gives each (b, h) its recall and output error, which
+    are averaged over the batch (the inputs the search averages over).  Each
+    head gets the candidate with the fewest attended tiles that meets every
+    given bound (``max_mse``, ``min_recall``); the full window when none does.
+    Returns ``{"windows": [H][3], "recall": [C, H], "mse": [C, H],
+    "candidates": [C][3], "tiles": [C]}`` (host values, fp64)."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(q.shape[-1])
+    B, H = int(q.shape[0]), int(q.shape[1])
+    lat = tuple(int(x) for x in latent)
+    cands = [tuple(int(x) for x in c) for c in candidates]
+    full = sta_plan(lat, tile, B, H, [lat] * H, stream=stream)
+    o_full, lse_full = sta_attention(q, k, v, full, softmax_scale, stream=stream)
+    n = [lat[i] // int(tile[i]) for i in range(3)]
+    tiles, rec, err = [], [], []
+    for c in cands:
+        plan = sta_plan(lat, tile, B, H, [c] * H, stream=stream)
+        o_c, lse_c = sta_attention(q, k, v, plan, softmax_scale, stream=stream)
+        r, m = sta_window_stats(lse_c, lse_full, o_c, o_full, stream=stream)
+        rec.append(r.mean(dim=0))
+        err.append(m.mean(dim=0))
+        tiles.append(math.prod(min(c[i] // int(tile[i]), n[i]) for i in range(3)))
+        plan.destroy()
+    full.destroy()
+    recall = torch.stack(rec).cpu().numpy() if rec else None
+    mse = torch.stack(err).cpu().numpy() if err else None
+    order = sorted(range(len(cands)), key=lambda i: tiles[i])
+    chosen = []
+    for h in range(H):
+        pick = lat
+        for i in order:
+            if (max_mse is None or mse[i, h] <= max_mse) and (min_recall is None or recall[i, h] >= min_recall):
+                pick = cands[i]
+                break
+        chosen.append(list(pick))
+    return {"windows": chosen, "recall": recall, "mse": mse, "candidates": [list(c) for c in cands],
+            "tiles": tiles}

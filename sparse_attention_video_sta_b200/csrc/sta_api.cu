@@ -477,6 +477,22 @@ sta_status sta_backward(sta_plan_t p, const void* q, const void* k, const void* 
                                             kDefaultTimeoutNs));
 }
 
+sta_status sta_window_stats(const float* lse_w, const float* lse_full, const void* o_w, const void* o_full,
+                            int64_t slices, int64_t tokens, int32_t head_dim, double* recall, double* mse,
+                            void* stream) {
+    if (lse_w == nullptr || lse_full == nullptr || o_w == nullptr || o_full == nullptr || recall == nullptr ||
+        mse == nullptr)
+        return STA_ERR_INVALID_ARG;
+    if (!aligned(lse_w, 4) || !aligned(lse_full, 4) || !aligned(o_w, 16) || !aligned(o_full, 16) ||
+        !aligned(recall, 8) || !aligned(mse, 8))
+        return STA_ERR_INVALID_ARG;
+    // 8 CTAs per slice in the launch grid
+    if (slices < 1 || slices > (int64_t(1) << 28) || tokens < 1 || head_dim < 8 || head_dim % 8 != 0)
+        return STA_ERR_INVALID_ARG;
+    return cuda_status(sta::launch_window_stats(lse_w, lse_full, o_w, o_full, slices, tokens, head_dim, recall,
+                                                mse, static_cast<cudaStream_t>(stream)));
+}
+
 sta_status sta_last_device_status(sta_plan_t p, void* stream) {
     if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

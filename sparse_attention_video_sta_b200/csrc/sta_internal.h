@@ -111,6 +111,11 @@ cudaError_t launch_backward(const sta_plan_s* p, const void* q, const void* k, c
                             void* dv, float* workspace, int head_dim, float softmax_scale,
                             cudaStream_t stream, uint64_t timeout_ns);
 
+// Per-slice recall / loss reduction for the window search (sta_search.cu).
+cudaError_t launch_window_stats(const float* lse_w, const float* lse_full, const void* o_w, const void* o_full,
+                                int64_t slices, int64_t tokens, int head_dim, double* recall, double* mse,
+                                cudaStream_t stream);
+
 // Permutation launch (sta_permute.cu).  inverse = false: raster -> tile-major.
 cudaError_t launch_permute(const void* src, void* dst, int64_t outer, int32_t row_bytes,
                            const sta_geom& g, bool inverse, cudaStream_t stream);

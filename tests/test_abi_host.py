@@ -192,3 +192,15 @@ def test_backward_rejected_before_launch():
     assert lib.sta_plan_key_query(hp.handle, 0, 27, None, 0, ctypes.byref(ctypes.c_int32())) == INV
     assert lib.sta_plan_key_query(hp.handle, 2, 0, None, 0, ctypes.byref(ctypes.c_int32())) == INV
     hp.destroy()
+
+
+def test_window_stats_rejected_before_launch():
+    INV = sta.STA_ERR_INVALID_ARG
+    lib = sta._lib
+    a = ctypes.c_void_p(1 << 30)
+    odd = ctypes.c_void_p((1 << 30) + 8)
+    assert lib.sta_window_stats(None, a, a, a, 1, 128, 64, a, a, None) == INV
+    assert lib.sta_window_stats(a, a, odd, a, 1, 128, 64, a, a, None) == INV   # o not 16-byte aligned
+    assert lib.sta_window_stats(a, a, a, a, 0, 128, 64, a, a, None) == INV     # no slices
+    assert lib.sta_window_stats(a, a, a, a, 1, 0, 64, a, a, None) == INV       # no tokens
+    assert lib.sta_window_stats(a, a, a, a, 1, 128, 12, a, a, None) == INV     # head_dim not a multiple of 8
