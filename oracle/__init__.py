@@ -132,14 +132,16 @@ def tile_major_index(latent, tile, tokens) -> np.ndarray:
 
 
 def tile_tokens(latent, tile, tile_id: int) -> np.ndarray:
-    """Raster indices of the tokens of tile ``tile_id`` (tiles numbered in
-    raster order over the tile grid), in raster order."""
-    n = [latent[i] // tile[i] for i in range(3)]
+    """Raster indices of the real tokens of tile ``tile_id`` (tiles numbered in
+    raster order over the tile grid of ceil(L / T) tiles per axis), in raster
+    order; a tile at a padded edge holds fewer than a full tile."""
+    n = [-(-latent[i] // tile[i]) for i in range(3)]
     it, rem = divmod(int(tile_id), n[1] * n[2])
     ih, iw = divmod(rem, n[2])
     t = np.arange(tile[0]) + it * tile[0]
     h = np.arange(tile[1]) + ih * tile[1]
     w = np.arange(tile[2]) + iw * tile[2]
+    t, h, w = t[t < latent[0]], h[h < latent[1]], w[w < latent[2]]
     tt, hh, ww = np.meshgrid(t, h, w, indexing="ij")
     return ((tt * latent[1] + hh) * latent[2] + ww).ravel().astype(np.int64)
 

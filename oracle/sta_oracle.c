@@ -30,7 +30,14 @@
  *     its extra tile on the lower side;
  *   - LSE is the natural log of sum_j exp(scale * q . k_j) over attended keys;
  *   - scale is applied as the double value of the fp32 softmax scale;
- *   - inputs are bf16 values, widened exactly to double.
+ *   - inputs are bf16 values, widened exactly to double;
+ *   - a latent axis that is not a multiple of the tile is padded at its high
+ *     end to whole tiles: the tile grid has n_d = ceil(L_d / T_d) tiles, the
+ *     windows are placed on that grid by the rule above, and a query attends
+ *     the real tokens of its window's tiles (padding tokens are neither keys
+ *     nor queries).  The pages fix only divisible latents; this is the plain
+ *     extension that keeps every interior block dense and puts mixed blocks at
+ *     the padded edge only.
  *
  * The oracle never builds a tile list and never permutes tokens: it evaluates
  * the token-level mask straight from token coordinates, in raster order.
@@ -63,9 +70,14 @@ static int geom_ok(const ora_geom* g)
 {
     for (int d = 0; d < 3; ++d) {
         if (g->lat[d] <= 0 || g->tile[d] <= 0) return 0;
-        if (g->lat[d] % g->tile[d] != 0) return 0;
     }
     return 1;
+}
+
+/* Tiles along axis d: the latent padded up to whole tiles. */
+static int32_t tiles_along(const ora_geom* g, int d)
+{
+    return (g->lat[d] + g->tile[d] - 1) / g->tile[d];
 }
 
 static int window_ok(const ora_geom* g, const int32_t* win)
@@ -107,7 +119,7 @@ static int key_allowed(const ora_geom* g, const int32_t* win, int64_t qi, int64_
     unravel(g, qi, qc);
     unravel(g, kj, kc);
     for (int d = 0; d < 3; ++d) {
-        int32_t n = g->lat[d] / g->tile[d];
+        int32_t n = tiles_along(g, d);
         int32_t e = win[d] / g->tile[d];
         if (e > n) e = n;
         int32_t s = window_start(qc[d] / g->tile[d], e, n);
@@ -138,15 +150,17 @@ int ora_mask_row(const ora_geom* g, const int32_t* win, int64_t qi, uint8_t* out
 /* Position of raster token `token` in tile-major order: tiles in raster order
  * over the tile grid, tokens inside a tile in raster order over the tile's own
  * (t, h, w) offsets.  The pages only say a tile is a contiguous cube of tokens;
- * this fixed order is the reading every layout test uses. */
+ * this fixed order is the reading every layout test uses.  With a padded
+ * latent the tile-major layout holds every tile whole (padding rows included),
+ * so positions range over n_tiles * tile volume. */
 int64_t ora_tile_major_index(const ora_geom* g, int64_t token)
 {
     if (!geom_ok(g)) return -1;
     if (token < 0 || token >= ora_num_tokens(g)) return -1;
     int32_t c[3];
     unravel(g, token, c);
-    int64_t n_h = g->lat[1] / g->tile[1];
-    int64_t n_w = g->lat[2] / g->tile[2];
+    int64_t n_h = tiles_along(g, 1);
+    int64_t n_w = tiles_along(g, 2);
     int64_t tile_id = ((int64_t)(c[0] / g->tile[0]) * n_h + c[1] / g->tile[1]) * n_w + c[2] / g->tile[2];
     int64_t local = ((int64_t)(c[0] % g->tile[0]) * g->tile[1] + c[1] % g->tile[1]) * g->tile[2] + c[2] % g->tile[2];
     return tile_id * ((int64_t)g->tile[0] * g->tile[1] * g->tile[2]) + local;
