@@ -167,11 +167,19 @@ class Plan:
 
     @property
     def tokens(self) -> int:
+        """Raster tokens per head (the latent)."""
         return self.latent[0] * self.latent[1] * self.latent[2]
 
     @property
     def tiles_per_head(self) -> int:
-        return self.tokens // (self.tile[0] * self.tile[1] * self.tile[2])
+        """Tiles per head; an axis that is not a multiple of the tile is padded to whole tiles."""
+        return math.prod(-(-self.latent[i] // self.tile[i]) for i in range(3))
+
+    @property
+    def padded_tokens(self) -> int:
+        """Rows per head of the tile-major layout (whole tiles; equals ``tokens``
+        when every axis is a multiple of the tile)."""
+        return self.tiles_per_head * self.tile[0] * self.tile[1] * self.tile[2]
 
     def query(self, head: int, q_tile: int) -> list:
         """Ascending key-tile ids attended by query tile ``q_tile`` of ``head``."""
@@ -253,16 +261,31 @@ def sta_plan_host(latent, tile, batch: int, heads: int, windows) -> Plan:
     return Plan(h.value, latent, tile, batch, heads, windows)
 
 
-def _perm_args(src: torch.Tensor, dst: torch.Tensor, tokens: int, token_dim: int):
+def _padded_tokens(latent, tile) -> int:
+    return math.prod(-(-int(latent[i]) // int(tile[i])) * int(tile[i]) for i in range(3))
+
+
+def _tile_major_like(x: torch.Tensor, plan: Plan, token_dim: int = 2) -> torch.Tensor:
+    """Empty tensor shaped like raster ``x`` with the token dimension padded to whole tiles."""
+    shape = list(x.shape)
+    shape[token_dim] = plan.padded_tokens
+    return torch.empty(shape, dtype=x.dtype, device=x.device)
+
+
+def _perm_args(src: torch.Tensor, dst: torch.Tensor, tokens: int, token_dim: int,
+               src_tokens: int | None = None, dst_tokens: int | None = None):
     if not (src.is_cuda and dst.is_cuda):
         raise ValueError("sta_tile_reorder/unreorder need CUDA tensors")
-    if src.shape != dst.shape or src.dtype != dst.dtype:
-        raise ValueError("src and dst must have the same shape and dtype")
+    if src.dtype != dst.dtype or src.dim() != dst.dim():
+        raise ValueError("src and dst must have the same dtype and rank")
     if not (src.is_contiguous() and dst.is_contiguous()):
         raise ValueError("src and dst must be contiguous")
     td = token_dim % src.dim()
-    if src.shape[td] != tokens:
-        raise ValueError(f"dimension {td} has {src.shape[td]} tokens, geometry has {tokens}")
+    for name, t, n in (("src", src, src_tokens), ("dst", dst, dst_tokens)):
+        if t.shape[td] != n:
+            raise ValueError(f"{name} dimension {td} has {t.shape[td]} tokens, expected {n}")
+    if src.shape[:td] != dst.shape[:td] or src.shape[td + 1:] != dst.shape[td + 1:]:
+        raise ValueError("src and dst may differ only in the token dimension")
     outer = math.prod(src.shape[:td]) if td > 0 else 1
     row_bytes = math.prod(src.shape[td + 1:]) * src.element_size()
     return outer, row_bytes
@@ -270,8 +293,10 @@ def _perm_args(src: torch.Tensor, dst: torch.Tensor, tokens: int, token_dim: int
 
 def sta_tile_reorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_dim: int = 2,
                      stream=None) -> torch.Tensor:
-    """dst = src with the token dimension permuted raster -> tile-major."""
-    outer, row_bytes = _perm_args(src, dst, latent[0] * latent[1] * latent[2], token_dim)
+    """dst = src with the token dimension permuted raster -> tile-major (dst's
+    token dimension padded to whole tiles, padding rows zeroed)."""
+    N = latent[0] * latent[1] * latent[2]
+    outer, row_bytes = _perm_args(src, dst, N, token_dim, N, _padded_tokens(latent, tile))
     g = _geom(latent, tile)
     _check(_lib.sta_tile_reorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
                                  outer, row_bytes, ctypes.byref(g), _stream(stream)),
@@ -281,8 +306,10 @@ def sta_tile_reorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_d
 
 def sta_tile_unreorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_dim: int = 2,
                        stream=None) -> torch.Tensor:
-    """dst = src with the token dimension permuted tile-major -> raster."""
-    outer, row_bytes = _perm_args(src, dst, latent[0] * latent[1] * latent[2], token_dim)
+    """dst = src with the token dimension permuted tile-major -> raster (src's
+    padding rows are dropped)."""
+    N = latent[0] * latent[1] * latent[2]
+    outer, row_bytes = _perm_args(src, dst, N, token_dim, _padded_tokens(latent, tile), N)
     g = _geom(latent, tile)
     _check(_lib.sta_tile_unreorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
                                    outer, row_bytes, ctypes.byref(g), _stream(stream)),
@@ -290,8 +317,9 @@ def sta_tile_unreorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token
     return dst
 
 
-def _forward_args(plan: Plan, q, k, v, o, lse):
-    B, H, N = plan.batch, plan.heads, plan.tokens
+def _forward_args(plan: Plan, q, k, v, o, lse, raster: bool = False):
+    B, H = plan.batch, plan.heads
+    N = plan.tokens if raster else plan.padded_tokens
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor")
@@ -318,7 +346,7 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
 def sta_forward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                        o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
     """STA forward on raster-order ``[B, H, N, d]`` bf16 tensors (permutation fused)."""
-    args = _forward_args(plan, q, k, v, o, lse)
+    args = _forward_args(plan, q, k, v, o, lse, raster=True)
     _check(_lib.sta_forward_raster(plan.handle, *args, float(softmax_scale), _stream(stream)),
            "sta_forward_raster")
     return o, lse
@@ -351,12 +379,18 @@ def sta_backward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, 
     return dq, dk, dv
 
 
-def raster_supported(tile) -> bool:
-    """Whether the fused raster path handles this tile shape (see sta.h)."""
-    hw = int(tile[1]) * int(tile[2])
+def raster_supported(tile, latent=None) -> bool:
+    """Whether the fused raster path handles this tile shape (see sta.h); with
+    ``latent``, also that one block's box is no larger than the latent."""
+    T = [int(x) for x in tile]
+    L = [int(x) for x in latent] if latent is not None else [1 << 30] * 3
+    hw = T[1] * T[2]
+    if T[2] > 256 or T[2] > L[2]:
+        return False
     if 128 % hw == 0:
-        return int(tile[0]) % (128 // hw) == 0 and int(tile[1]) <= 256 and int(tile[2]) <= 256
-    return hw % 128 == 0 and 128 % int(tile[2]) == 0
+        box_t = 128 // hw
+        return T[0] % box_t == 0 and T[1] <= 256 and box_t <= L[0] and T[1] <= L[1]
+    return hw % 128 == 0 and 128 % T[2] == 0 and 128 // T[2] <= L[1]
 
 
 def sta_forward_noalloc(latent, tile, batch: int, heads: int, windows, q: torch.Tensor,
@@ -405,19 +439,19 @@ def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(q.shape[-1])
     lat, tile = plan.latent, plan.tile
-    if fused and raster_supported(tile):
+    if fused and raster_supported(tile, lat):
         o = torch.empty_like(q)
         lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
         return sta_forward_raster(plan, q, k, v, o, lse, softmax_scale, stream=stream)
-    qt, kt, vt = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    qt, kt, vt = (_tile_major_like(x, plan) for x in (q, k, v))
     sta_tile_reorder(q, qt, lat, tile, stream=stream)
     sta_tile_reorder(k, kt, lat, tile, stream=stream)
     sta_tile_reorder(v, vt, lat, tile, stream=stream)
-    ot = torch.empty_like(q)
-    lset = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    ot = torch.empty_like(qt)
+    lset = torch.empty(qt.shape[:3], dtype=torch.float32, device=q.device)
     sta_forward(plan, qt, kt, vt, ot, lset, softmax_scale, stream=stream)
     o = torch.empty_like(q)
-    lse = torch.empty_like(lset)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
     sta_tile_unreorder(ot, o, lat, tile, stream=stream)
     sta_tile_unreorder(lset, lse, lat, tile, stream=stream)
     return o, lse
@@ -434,15 +468,15 @@ def sta_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o:
     lat, tile = plan.latent, plan.tile
 
     def to_tiles(x):
-        y = torch.empty_like(x)
+        y = _tile_major_like(x, plan)
         sta_tile_reorder(x, y, lat, tile, stream=stream)
         return y
 
     qt, kt, vt, ot, dot, lset = (to_tiles(x) for x in (q, k, v, o, dout, lse))
     dqt, dkt, dvt = sta_backward(plan, qt, kt, vt, ot, lset, dot, softmax_scale, stream=stream)
     out = []
-    for x in (dqt, dkt, dvt):
-        y = torch.empty_like(x)
+    for x, like in ((dqt, q), (dkt, k), (dvt, v)):
+        y = torch.empty_like(like)
         sta_tile_unreorder(x, y, lat, tile, stream=stream)
         out.append(y)
     return tuple(out)

@@ -46,7 +46,7 @@ bool geom_valid(const sta_geom* g) {
     const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
     const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
     for (int d = 0; d < 3; ++d) {
-        if (L[d] <= 0 || T[d] <= 0 || L[d] % T[d] != 0) return false;
+        if (L[d] <= 0 || T[d] <= 0) return false;
     }
     const int64_t n = int64_t(L[0]) * L[1] * L[2];
     return n <= INT32_MAX;
@@ -99,7 +99,9 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
     P.g = *g;
     P.batch = batch;
     P.heads = heads;
-    for (int d = 0; d < 3; ++d) P.n_tiles[d] = L[d] / T[d];
+    // An axis that is not a multiple of the tile is padded at its high end to
+    // whole tiles (padding tokens are neither keys nor queries).
+    for (int d = 0; d < 3; ++d) P.n_tiles[d] = (L[d] + T[d] - 1) / T[d];
     P.tiles_per_head = P.n_tiles[0] * P.n_tiles[1] * P.n_tiles[2];
     P.tile_tokens = T[0] * T[1] * T[2];
     if (P.tile_tokens % sta::kSubRows != 0) return STA_ERR_UNSUPPORTED;
@@ -163,6 +165,27 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
                 o[1] = qh * T[1];
                 o[2] = qt * T[0];
             }
+
+    // Padded latents: which keys of each 128-key chunk of a tile are real
+    // tokens (bit j of word j / 32 for key j of the chunk).  Tiles at the
+    // padded edge are the only ones with clear bits.
+    P.padded = (L[0] % T[0]) != 0 || (L[1] % T[1]) != 0 || (L[2] % T[2]) != 0;
+    P.key_mask.clear();
+    if (P.padded) {
+        P.key_mask.assign(size_t(P.tiles_per_head) * P.sub_per_tile * 4, 0u);
+        for (int32_t tile = 0; tile < P.tiles_per_head; ++tile) {
+            const int32_t* o = &P.tile_origin[size_t(tile) * 4];
+            const int32_t vt = std::min(T[0], L[0] - o[2]), vh = std::min(T[1], L[1] - o[1]),
+                          vw = std::min(T[2], L[2] - o[0]);
+            for (int32_t l = 0; l < P.tile_tokens; ++l) {
+                const int32_t x = l % T[2], y = (l / T[2]) % T[1], t = l / (T[2] * T[1]);
+                if (t < vt && y < vh && x < vw) {
+                    const int32_t sub = l / sta::kChunkKeys, j = l % sta::kChunkKeys;
+                    P.key_mask[(size_t(tile) * P.sub_per_tile + sub) * 4 + j / 32] |= 1u << (j % 32);
+                }
+            }
+        }
+    }
 
     // Work items.  Row blocks of one tile are paired so the pair shares K/V
     // loads; with an odd count per tile, the last block of consecutive tiles
@@ -239,6 +262,8 @@ void free_device(sta_plan_s* p) {
     if (p->d_items) cudaFree(p->d_items);
     if (p->d_status) cudaFree(p->d_status);
     if (p->d_origin) cudaFree(p->d_origin);
+    if (p->d_kmask) cudaFree(p->d_kmask);
+    p->d_kmask = nullptr;
     if (p->d_toff) cudaFree(p->d_toff);
     if (p->d_tids) cudaFree(p->d_tids);
     if (p->d_bq_items) cudaFree(p->d_bq_items);
@@ -272,9 +297,13 @@ sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row
     if (src == nullptr || dst == nullptr || !geom_valid(g) || outer < 1 || row_bytes <= 0)
         return STA_ERR_INVALID_ARG;
     const int64_t n_tok = int64_t(g->lat_t) * g->lat_h * g->lat_w;
-    const int64_t bytes = outer * n_tok * int64_t(row_bytes);
+    int64_t n_pad = 1;  // tile-major rows per slice: whole tiles
+    const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w}, T[3] = {g->tile_t, g->tile_h, g->tile_w};
+    for (int d = 0; d < 3; ++d) n_pad *= int64_t((L[d] + T[d] - 1) / T[d]) * T[d];
+    const int64_t r_bytes = outer * n_tok * int64_t(row_bytes), t_bytes = outer * n_pad * int64_t(row_bytes);
+    const int64_t s_bytes = inverse ? t_bytes : r_bytes, d_bytes = inverse ? r_bytes : t_bytes;
     const uintptr_t s = reinterpret_cast<uintptr_t>(src), d = reinterpret_cast<uintptr_t>(dst);
-    if (s < d + uint64_t(bytes) && d < s + uint64_t(bytes)) return STA_ERR_INVALID_ARG;  // overlap
+    if (s < d + uint64_t(d_bytes) && d < s + uint64_t(s_bytes)) return STA_ERR_INVALID_ARG;  // overlap
     return cuda_status(sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
                                            static_cast<cudaStream_t>(stream)));
 }
@@ -358,6 +387,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
     if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
+    if (e == cudaSuccess && p->h.padded) e = upload(&p->d_kmask, p->h.key_mask, s);
     if (e == cudaSuccess) e = upload(&p->d_toff, p->h.tcsr_off, s);
     if (e == cudaSuccess) e = upload(&p->d_tids, p->h.tcsr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_bq_items, p->h.bq_items, s);
@@ -380,7 +410,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_toff ||
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_kmask || p->d_toff ||
         p->d_tids || p->d_bq_items || p->d_bkv_items) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
         free_device(p);

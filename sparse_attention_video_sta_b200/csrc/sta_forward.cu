@@ -92,7 +92,8 @@ struct FwdParams {
     int32_t tiles_per_head;
     int32_t sub_per_tile;  // 128-row blocks (= 128-key chunks) per tile
     int32_t tile_tokens;
-    int32_t tokens;  // N per (b, h)
+    int32_t tokens;  // tile-major rows per (b, h): whole tiles
+    int32_t tokens_raster;  // raster rows per (b, h): the latent's tokens
     __nv_bfloat16* o;
     float* lse;
     float scale_log2;  // softmax_scale * log2(e)
@@ -107,6 +108,10 @@ struct FwdParams {
     int32_t n_h, n_w;
     int32_t box_t, box_h, blocks_per_slice;
     const int4* tile_origin;  // [tiles]: raster (w, h, t) origin of each tile
+    // Padded latents (an axis not a multiple of the tile): real-key bits of
+    // every 128-key chunk, [tiles][sub_per_tile] x 4 words; null otherwise.
+    const uint4* key_mask;
+    int32_t lat_t;
 };
 
 // Load 128-row block `sub` of tile `tile` of head bh.  Tile-major layout: one
@@ -133,22 +138,34 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* m, u
     }
 }
 
-// Row of the output tensors that holds row `r` of block `blk` of head bh.
-template <bool kRaster>
+// Row of the output tensors that holds row `r` of block `blk` of head bh; -1
+// for a padding row of a raster output (a token past the latent; kPadded only).
+template <bool kRaster, bool kPadded>
 __device__ __forceinline__ int64_t out_row(const FwdParams& p, int32_t bh, int32_t blk, int32_t r) {
     if (!kRaster) return int64_t(bh) * p.tokens + int64_t(blk) * kSubRows + r;
     const int32_t tile = blk / p.sub_per_tile, sub = blk - tile * p.sub_per_tile;
     const int32_t it = tile / (p.n_h * p.n_w), ih = (tile / p.n_w) % p.n_h, iw = tile % p.n_w;
     const int32_t l = sub * kSubRows + r;  // tile-local row, raster over the tile's (t, h, w)
     const int32_t lw = l % p.tile_w, lh = (l / p.tile_w) % p.tile_h, lt = l / (p.tile_w * p.tile_h);
-    const int64_t token = (int64_t(it * p.tile_t + lt) * p.lat_h + ih * p.tile_h + lh) * p.lat_w + iw * p.tile_w + lw;
-    return int64_t(bh) * p.tokens + token;
+    const int32_t t = it * p.tile_t + lt, h = ih * p.tile_h + lh, w = iw * p.tile_w + lw;
+    if (kPadded && (t >= p.lat_t || h >= p.lat_h || w >= p.lat_w)) return -1;
+    const int64_t token = (int64_t(t) * p.lat_h + h) * p.lat_w + w;
+    return int64_t(bh) * p.tokens_raster + token;
 }
 
 // Bounded wait with this launch's status word and time limit.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          const FwdParams& p) {
     return wait_bar_limited(bar, parity, abort_flag, p.status, p.timeout_ns);
+}
+
+// Padded latents: scores of the chunk's padding keys become -inf, so they take
+// no softmax weight.  `m` holds the chunk's real-key bits.
+__device__ __forceinline__ void mask_scores(uint32_t (&sr)[128], const uint4 m) {
+    const uint32_t w[4] = {m.x, m.y, m.z, m.w};
+#pragma unroll
+    for (int j = 0; j < 128; ++j)
+        if (!((w[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0xff800000u;
 }
 
 // P = exp2(S * c - m * c) for one 128-score row, packed to bf16 pairs; returns
@@ -201,7 +218,9 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[128]) {
     return ptx::max3(a0, a1, fmaxf(a2, a3));
 }
 
-template <int D, bool kRaster>
+// kPadded: the latent has padding tokens (an axis that is not a multiple of
+// the tile): padding keys are masked and raster padding rows are not stored.
+template <int D, bool kRaster, bool kPadded>
 __global__ void __launch_bounds__(kThreads, 1)
 sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -458,6 +477,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
             const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
             const int32_t q_blk = slot == 0 ? w.qa : w.qb;
+            const int32_t kbeg = kPadded ? off[q_blk / SPT] : 0;  // this slot's key tiles
             float m_used = 0.0f, l = 0.0f;
             for (int32_t i = 0; i < n_chunks; ++i) {
                 if (!__all_sync(0xffffffffu, wait_bar(bar_s_full(slot), scnt & 1u, abort_flag, p))) {
@@ -471,9 +491,18 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float alpha = 1.0f;
                 float mx;
                 uint32_t sr[128];
+                const uint4* kmask =
+                    kPadded ? p.key_mask + int64_t(__ldg(p.ids + kbeg + i / SPT)) * SPT + i % SPT : nullptr;
                 ptx::tmem_ld128(tS, sr);
+                bool masked = false;  // warp-uniform: the chunk is one of an edge tile
+                if (kPadded) {
+                    const uint4 m = __ldg(kmask);
+                    masked = (m.x & m.y & m.z & m.w) != ~0u;
+                    if (masked) mask_scores(sr, m);
+                }
                 uint32_t pk[64];
                 if (i == 0) {
+                    // a tile's first chunk holds its first token, a real key: the max is finite
                     m_used = row_max(sr);
                     rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
                 } else {
@@ -490,6 +519,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         }
                         // S is still in TMEM (P has not been written over it yet)
                         ptx::tmem_ld128(tS, sr);
+                        if (kPadded && masked) mask_scores(sr, __ldg(kmask));
                         rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
                     }
                 }
@@ -531,26 +561,28 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             ++ocnt;
             ptx::tc_fence_after();
             const float inv_l = 1.0f / l;
-            const int64_t grow = out_row<kRaster>(p, w.bh, q_blk, row);
-            uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D);
+            const int64_t grow = out_row<kRaster, kPadded>(p, w.bh, q_blk, row);
+            uint4* dst = reinterpret_cast<uint4*>(p.o + (grow < 0 ? 0 : grow) * D);
 #pragma unroll 1
             for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t orr[32];
-                ptx::tmem_ld32(tO + cb * 32, orr);
+                ptx::tmem_ld32(tO + cb * 32, orr);  // every lane loads: the access is warp-wide
+                if (grow >= 0) {                   // a padding row of a raster output stores nothing
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    uint4 v;
-                    v.x = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 0]) * inv_l, __uint_as_float(orr[8 * j + 1]) * inv_l);
-                    v.y = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv_l, __uint_as_float(orr[8 * j + 3]) * inv_l);
-                    v.z = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv_l, __uint_as_float(orr[8 * j + 5]) * inv_l);
-                    v.w = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv_l, __uint_as_float(orr[8 * j + 7]) * inv_l);
-                    dst[cb * 4 + j] = v;
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 v;
+                        v.x = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 0]) * inv_l, __uint_as_float(orr[8 * j + 1]) * inv_l);
+                        v.y = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv_l, __uint_as_float(orr[8 * j + 3]) * inv_l);
+                        v.z = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv_l, __uint_as_float(orr[8 * j + 5]) * inv_l);
+                        v.w = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv_l, __uint_as_float(orr[8 * j + 7]) * inv_l);
+                        dst[cb * 4 + j] = v;
+                    }
                 }
             }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(bar_o_empty(slot));
-            p.lse[grow] = m_used * p.scale + logf(l);
+            if (grow >= 0) p.lse[grow] = m_used * p.scale + logf(l);
         }
     }
 
@@ -615,6 +647,16 @@ cudaError_t make_map_raster(CUtensorMap* m, const void* ptr, const sta_geom& g, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+template <int D, bool kRaster, bool kPadded>
+cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
+                          const CUtensorMap& mv, const FwdParams& fp) {
+    cudaError_t e = cudaFuncSetAttribute(sta_fwd_kernel<D, kRaster, kPadded>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    sta_fwd_kernel<D, kRaster, kPadded><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
+    return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const void* v, void* o,
                      float* lse, float scale, cudaStream_t stream, int inject, uint64_t timeout_ns,
@@ -645,6 +687,7 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.sub_per_tile = P.sub_per_tile;
     fp.tile_tokens = P.tile_tokens;
     fp.tokens = P.tiles_per_head * P.tile_tokens;
+    fp.tokens_raster = P.g.lat_t * P.g.lat_h * P.g.lat_w;
     fp.o = static_cast<__nv_bfloat16*>(o);
     fp.lse = lse;
     fp.scale = scale;
@@ -663,24 +706,19 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.box_h = rb.box_h;
     fp.blocks_per_slice = rb.blocks_per_slice;
     fp.tile_origin = reinterpret_cast<const int4*>(pl->d_origin);
+    fp.key_mask = reinterpret_cast<const uint4*>(pl->d_kmask);
+    fp.lat_t = P.g.lat_t;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
-    if (raster) {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<D>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        sta_fwd_kernel<D, true><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
-    } else {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<D>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        sta_fwd_kernel<D, false><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
-    }
-    return cudaGetLastError();
+    if (raster)
+        return P.padded ? launch_kernel<D, true, true>(grid, stream, mq, mk, mv, fp)
+                        : launch_kernel<D, true, false>(grid, stream, mq, mk, mv, fp);
+    return P.padded ? launch_kernel<D, false, true>(grid, stream, mq, mk, mv, fp)
+                    : launch_kernel<D, false, false>(grid, stream, mq, mk, mv, fp);
 }
 
 }  // namespace
@@ -688,17 +726,17 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
 RasterBox raster_box(const sta_geom& g) {
     RasterBox rb{0, 0, 0, false};
     const int32_t hw = g.tile_h * g.tile_w;
-    if (hw <= 0 || g.tile_w > 256) return rb;
+    if (hw <= 0 || g.tile_w > 256 || g.tile_w > g.lat_w) return rb;
     if (kSubRows % hw == 0) {  // a block is whole (h, w) slices: box_t of them
         rb.box_t = kSubRows / hw;
         rb.box_h = g.tile_h;
         rb.blocks_per_slice = 1;
-        rb.ok = g.tile_h <= 256 && g.tile_t % rb.box_t == 0;
+        rb.ok = g.tile_h <= 256 && g.tile_t % rb.box_t == 0 && rb.box_t <= g.lat_t && rb.box_h <= g.lat_h;
     } else if (hw % kSubRows == 0 && kSubRows % g.tile_w == 0) {  // a block is part of one slice
         rb.box_t = 1;
         rb.box_h = kSubRows / g.tile_w;
         rb.blocks_per_slice = hw / kSubRows;
-        rb.ok = true;
+        rb.ok = rb.box_h <= g.lat_h;  // boxes never wider than the latent (edge boxes read past it: zero fill)
     }
     return rb;
 }
@@ -742,18 +780,8 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     if (e != cudaSuccess) return e;
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
-    if (head_dim == 128) {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<128>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        sta_fwd_kernel<128, false><<<grid, kThreads, Cfg<128>::kSmemBytes, stream>>>(mq, mk, mv, fp);
-    } else {
-        e = cudaFuncSetAttribute(sta_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Cfg<64>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        sta_fwd_kernel<64, false><<<grid, kThreads, Cfg<64>::kSmemBytes, stream>>>(mq, mk, mv, fp);
-    }
-    return cudaGetLastError();
+    if (head_dim == 128) return launch_kernel<128, false, false>(grid, stream, mq, mk, mv, fp);
+    return launch_kernel<64, false, false>(grid, stream, mq, mk, mv, fp);
 }
 
 }  // namespace sta

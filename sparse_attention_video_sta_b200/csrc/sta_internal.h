@@ -48,6 +48,8 @@ struct PlanHost {
     std::vector<WorkItem> bq_items;
     std::vector<WorkItem> bkv_items;
     std::vector<int32_t> tile_origin;        // [tiles_per_head][4]: raster (w, h, t) origin of each tile, 0
+    bool padded = false;                     // some axis is not a multiple of the tile
+    std::vector<uint32_t> key_mask;          // padded only: [tiles][sub_per_tile][4] real-key bits per chunk
     int64_t computed_pairs = 0;              // B * sum_h sum_q |list|
 };
 
@@ -62,6 +64,7 @@ struct sta_plan_s {
     sta::WorkItem* d_items = nullptr;
     uint32_t* d_status = nullptr;
     int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
+    uint32_t* d_kmask = nullptr;  // device copy of key_mask (padded latents only)
     int32_t* d_toff = nullptr;
     int32_t* d_tids = nullptr;
     sta::WorkItem* d_bq_items = nullptr;

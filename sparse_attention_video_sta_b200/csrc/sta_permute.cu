@@ -10,6 +10,11 @@
 // so consecutive threads read and write consecutive addresses on both sides.
 // The per-tile map from local token index to raster offset is built once per
 // CTA in shared memory.  HBM-bound: 2 x tensor bytes per pass.
+//
+// A latent axis that is not a multiple of the tile is padded at its high end
+// to whole tiles: the tile-major layout holds every tile whole, and its
+// padding rows (tokens past the latent) are written as zeros by the reorder
+// and skipped by the inverse.  Only tiles at the padded edge test rows.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -22,12 +27,13 @@ constexpr int kPermThreads = 256;
 constexpr int kMaxTableTokens = 12288;  // 48 KB of int32 in shared memory
 
 struct PermGeom {
-    int32_t lat_h, lat_w;
+    int32_t lat_t, lat_h, lat_w;
     int32_t tile_t, tile_h, tile_w;
     int32_t n_h, n_w;       // tiles along h and w
     int32_t tiles;          // tiles per head
     int32_t tile_tokens;
-    int64_t tokens;         // tokens per head
+    int64_t tokens;         // raster tokens per head
+    int64_t tm_tokens;      // tile-major rows per head (tiles * tile_tokens)
 };
 
 __device__ __forceinline__ int64_t local_to_raster(const PermGeom& g, int32_t l) {
@@ -58,8 +64,13 @@ permute_kernel(const V* __restrict__ src, V* __restrict__ dst, PermGeom g, int32
         const int32_t iw = tile % g.n_w;
         const int64_t origin = (int64_t(it) * g.tile_t * g.lat_h + int64_t(ih) * g.tile_h) * g.lat_w +
                                int64_t(iw) * g.tile_w;
-        const int64_t slice = outer * g.tokens;
+        const int64_t r_slice = outer * g.tokens, t_slice = outer * g.tm_tokens;
         const int64_t tm_base = int64_t(tile) * g.tile_tokens;
+        // valid extents of this tile (smaller than the tile only at a padded edge)
+        const int32_t vt = min(g.tile_t, g.lat_t - it * g.tile_t);
+        const int32_t vh = min(g.tile_h, g.lat_h - ih * g.tile_h);
+        const int32_t vw = min(g.tile_w, g.lat_w - iw * g.tile_w);
+        const bool edge = vt < g.tile_t || vh < g.tile_h || vw < g.tile_w;
 #pragma unroll 4
         for (int64_t e = threadIdx.x; e < per_tile; e += blockDim.x) {
             int32_t l, c;
@@ -70,11 +81,19 @@ permute_kernel(const V* __restrict__ src, V* __restrict__ dst, PermGeom g, int32
                 l = int32_t(e / vpr);
                 c = int32_t(e - int64_t(l) * vpr);
             }
-            const int64_t raster = origin + (kTable ? int64_t(table[l]) : local_to_raster(g, l));
-            const int64_t tmaj = tm_base + l;
-            const int64_t s_row = slice + (inverse ? tmaj : raster);
-            const int64_t d_row = slice + (inverse ? raster : tmaj);
-            dst[d_row * vpr + c] = src[s_row * vpr + c];
+            const int64_t tmaj = t_slice + tm_base + l;
+            if (edge) {
+                const int32_t x = l % g.tile_w, y = (l / g.tile_w) % g.tile_h, t = l / (g.tile_w * g.tile_h);
+                if (t >= vt || y >= vh || x >= vw) {  // padding row
+                    if (!inverse) dst[tmaj * vpr + c] = V{};
+                    continue;
+                }
+            }
+            const int64_t raster = r_slice + origin + (kTable ? int64_t(table[l]) : local_to_raster(g, l));
+            if (inverse)
+                dst[raster * vpr + c] = src[tmaj * vpr + c];
+            else
+                dst[tmaj * vpr + c] = src[raster * vpr + c];
         }
     }
 }
@@ -116,16 +135,18 @@ cudaError_t launch_typed(const void* src, void* dst, int64_t outer, int32_t row_
 cudaError_t launch_permute(const void* src, void* dst, int64_t outer, int32_t row_bytes,
                            const sta_geom& sg, bool inverse, cudaStream_t stream) {
     PermGeom g;
+    g.lat_t = sg.lat_t;
     g.lat_h = sg.lat_h;
     g.lat_w = sg.lat_w;
     g.tile_t = sg.tile_t;
     g.tile_h = sg.tile_h;
     g.tile_w = sg.tile_w;
-    g.n_h = sg.lat_h / sg.tile_h;
-    g.n_w = sg.lat_w / sg.tile_w;
-    g.tiles = (sg.lat_t / sg.tile_t) * g.n_h * g.n_w;
+    g.n_h = (sg.lat_h + sg.tile_h - 1) / sg.tile_h;
+    g.n_w = (sg.lat_w + sg.tile_w - 1) / sg.tile_w;
+    g.tiles = ((sg.lat_t + sg.tile_t - 1) / sg.tile_t) * g.n_h * g.n_w;
     g.tile_tokens = sg.tile_t * sg.tile_h * sg.tile_w;
     g.tokens = int64_t(sg.lat_t) * sg.lat_h * sg.lat_w;
+    g.tm_tokens = int64_t(g.tiles) * g.tile_tokens;
     const uintptr_t align = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
                             uintptr_t(row_bytes);
     if (align % 16 == 0) return launch_typed<uint4>(src, dst, outer, row_bytes, g, inverse, stream);

@@ -95,14 +95,49 @@ def oracle_rows(q, k, v, latent, tile, windows, scale, bhs, tokens):
 # gradients are rounded to bf16 (up to 2^-9 |ref|).  A CPU emulation of that
 # arithmetic against the fp64 oracle on the tiny workload gives max
 # (|delta| - 2^-8 |ref|) / rms = 1.6e-2 and mean |delta| / rms = 1.8e-3.
+#
+# One more term matters for dQ when a row attends very few keys (possible on a
+# padded latent: a one-tile window on a mostly padded edge tile): D_i is
+# dO_i . O_i with the forward's bf16 O, so |delta D_i| <= 2^-9 sum_c |dO_ic O_ic|,
+# which shifts dQ_i by -scale delta D_i (P K)_i.  dS sums to zero over a row,
+# so with few keys dQ_i is small while (P K)_i is not, and this term
+# dominates.  `dq_d_term` gives the allowance 2^-8 scale sum_c |dO_ic O_ic|
+# |(P K)_ic| (twice the bound), from the oracle's O and P K; `dk_d_term` the
+# same error's effect on dK (a key seen by few queries).  A CPU emulation of
+# the kernels' arithmetic on a one-tile window over mostly padded tiles fails
+# without these terms (4.8e-2 rms on dK) and passes with them.
 GRAD_RMS_TOL = 3e-2
 GRAD_REL = 2.0 ** -8
 GRAD_MEAN_TOL = 3e-3
 
 
-def compare_grad(got, ref: np.ndarray, bh: np.ndarray, what: str = ""):
-    """got, ref: [R, d] rows; bh: [R] slice id of each row.  Asserts the
-    gradient tolerances per slice; returns the worst (max/rms, mean/rms)."""
+def dq_d_term(o_ref: np.ndarray, pk_ref: np.ndarray, dout, scale: float) -> np.ndarray:
+    """Per-element allowance for the bf16-O error in D (rows [R, d])."""
+    g = dout.detach().cpu().to(torch.float64).numpy() if hasattr(dout, "detach") else np.asarray(dout)
+    s1 = np.sum(np.abs(g * o_ref), axis=-1, keepdims=True)
+    return 2.0 ** -8 * scale * s1 * np.abs(pk_ref)
+
+
+def dk_d_term(q, k, v, o_ref: np.ndarray, dout, latent, tile, windows, scale: float) -> np.ndarray:
+    """Per-element allowance for the same bf16-O error in D on dK: delta D_i
+    shifts dK_j by -scale sum_i P_ij delta D_i q_i, bounded by
+    2^-8 scale (P^T W)_j with W_i = sum_c |dO_ic O_ic| |q_i|; P^T W is the
+    oracle's dV for upstream gradient W.  Shape [B, H, N, d]."""
+    g = dout.detach().cpu().to(torch.float64).numpy() if hasattr(dout, "detach") else np.asarray(dout)
+    qa = q.detach().cpu().to(torch.float64).numpy() if hasattr(q, "detach") else np.asarray(q)
+    w = np.sum(np.abs(g * o_ref), axis=-1, keepdims=True) * np.abs(qa)
+    # W rounded up to the next bf16 value keeps the allowance an upper bound
+    wt = torch.from_numpy(w.astype(np.float32)).to(torch.bfloat16)
+    wt = torch.where(wt.float() < torch.from_numpy(w.astype(np.float32)),
+                     torch.nextafter(wt, torch.tensor(float("inf"), dtype=torch.bfloat16)), wt)
+    _, ptw = oracle.sta_backward_dkdv(q, k, v, wt, latent, tile, windows, scale)
+    return 2.0 ** -8 * scale * np.abs(ptw)
+
+
+def compare_grad(got, ref: np.ndarray, bh: np.ndarray, what: str = "", extra: np.ndarray | None = None):
+    """got, ref: [R, d] rows; bh: [R] slice id of each row; `extra`: optional
+    per-element allowance added to the bound.  Asserts the gradient
+    tolerances per slice; returns the worst (max/rms, mean/rms)."""
     g = got.detach().cpu().to(torch.float64).numpy() if hasattr(got, "detach") else np.asarray(got)
     assert np.all(np.isfinite(g)), what
     worst = (0.0, 0.0)
@@ -112,7 +147,8 @@ def compare_grad(got, ref: np.ndarray, bh: np.ndarray, what: str = ""):
         rms = float(np.sqrt(np.mean(r * r)))
         e = np.abs(a - r)
         assert rms > 0, (what, int(s))
-        excess = float(np.max(e - GRAD_REL * np.abs(r))) / rms
+        allow = GRAD_REL * np.abs(r) + (extra[sel] if extra is not None else 0.0)
+        excess = float(np.max(e - allow)) / rms
         mean = float(np.mean(e)) / rms
         assert excess <= GRAD_RMS_TOL, (what, int(s), "max excess / rms", excess)
         assert mean <= GRAD_MEAN_TOL, (what, int(s), "mean / rms", mean)

@@ -52,7 +52,11 @@ def _raw_plan_host(latent, tile, batch, heads, windows):
 def test_plan_argument_validation():
     INV, UNS = sta.STA_ERR_INVALID_ARG, sta.STA_ERR_UNSUPPORTED
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == 0
-    assert _raw_plan_host((30, 48, 81), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == INV  # latent % tile
+    # a latent axis that is not a multiple of the tile is padded to whole tiles
+    assert _raw_plan_host((30, 48, 81), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == 0
+    assert _raw_plan_host((33, 45, 80), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == 0
+    assert _raw_plan_host((30, 48, 0), (6, 8, 8), 1, 1, [(18, 24, 24)])[0] == INV
+    assert _raw_plan_host((30, 48, 80), (6, 0, 8), 1, 1, [(18, 24, 24)])[0] == INV
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(18, 24, 20)])[0] == INV  # window % tile
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(0, 24, 24)])[0] == INV
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 0, 1, [(18, 24, 24)])[0] == INV
@@ -69,7 +73,7 @@ def test_calls_rejected_before_launch():
     INV = sta.STA_ERR_INVALID_ARG
     lib = sta._lib
     g = sta._geom((18, 24, 24), (6, 8, 8))
-    bad = sta._geom((18, 24, 25), (6, 8, 8))
+    bad = sta._geom((18, 24, 0), (6, 8, 8))
     p = ctypes.c_void_p(1 << 20)
     assert lib.sta_tile_reorder(None, p, 1, 128, ctypes.byref(g), None) == INV
     assert lib.sta_tile_reorder(p, None, 1, 128, ctypes.byref(g), None) == INV
@@ -204,3 +208,32 @@ def test_window_stats_rejected_before_launch():
     assert lib.sta_window_stats(a, a, a, a, 0, 128, 64, a, a, None) == INV     # no slices
     assert lib.sta_window_stats(a, a, a, a, 1, 0, 64, a, a, None) == INV       # no tokens
     assert lib.sta_window_stats(a, a, a, a, 1, 128, 12, a, a, None) == INV     # head_dim not a multiple of 8
+
+
+@pytest.mark.parametrize("latent,tile,windows", [
+    ((13, 21, 18), (6, 8, 8), [(6, 8, 8), (12, 16, 16), (18, 24, 24)]),
+    ((9, 8, 20), (4, 8, 8), [(8, 8, 16), (4, 8, 24)]),
+])
+def test_padded_plan_lists_match_oracle_mask(latent, tile, windows):
+    """Latents that are not a multiple of the tile: the plan's lists (and the
+    transposed lists) equal the tile sets read off the oracle's token mask."""
+    p = sta.sta_plan_host(latent, tile, 1, len(windows), windows)
+    n = [-(-latent[i] // tile[i]) for i in range(3)]
+    n_tiles = n[0] * n[1] * n[2]
+    assert p.tiles_per_head == n_tiles
+    assert p.padded_tokens == n_tiles * tile[0] * tile[1] * tile[2]
+    for h, win in enumerate(windows):
+        attends = []
+        for q in range(n_tiles):
+            toks = oracle.tile_tokens(latent, tile, q)
+            row = oracle.mask_row(latent, tile, win, int(toks[0]))
+            got = []
+            for t in range(n_tiles):
+                blk = row[oracle.tile_tokens(latent, tile, t)]
+                assert blk.all() or not blk.any()
+                if blk.all():
+                    got.append(t)
+            assert p.query(h, q) == got, (latent, win, q)
+            attends.append(set(got))
+        for kt in range(n_tiles):
+            assert p.key_query(h, kt) == [q for q in range(n_tiles) if kt in attends[q]]

@@ -1,0 +1,112 @@
+"""GPU parity on latents that are not a multiple of the tile (padded at the
+high end of each axis to whole tiles; padding tokens are neither keys nor
+queries), against the fp64 oracle.  Includes HunyuanVideo's own 720p latent
+33 x 45 x 80 (the 5 s clip before any cropping), which no 6 x 8 x 8 tile
+divides."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity_util import compare, compare_grad, dk_d_term, dq_d_term
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sta():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    import sparse_attention_video_sta_b200 as s
+    return s
+
+
+def padded(latent, tile):
+    return int(np.prod([-(-latent[i] // tile[i]) * tile[i] for i in range(3)]))
+
+
+@pytest.mark.parametrize("latent,tile,row_shape,dtype", [
+    ((13, 21, 18), (6, 8, 8), (128,), torch.bfloat16),
+    ((33, 45, 80), (6, 8, 8), (64,), torch.bfloat16),
+    ((13, 21, 18), (6, 8, 8), (), torch.float32),
+    ((5, 7, 9), (2, 4, 4), (3,), torch.int16),
+])
+def test_padded_permutation(sta, latent, tile, row_shape, dtype):
+    N = latent[0] * latent[1] * latent[2]
+    Np = padded(latent, tile)
+    g = torch.Generator().manual_seed(N)
+    if dtype.is_floating_point:
+        x = torch.randn((2, N) + row_shape, generator=g).to(dtype)
+    else:
+        x = torch.randint(-100, 100, (2, N) + row_shape, generator=g).to(dtype)
+    xd = x.cuda()
+    y = torch.full((2, Np) + row_shape, 7, dtype=dtype, device="cuda")
+    sta.sta_tile_reorder(xd, y, latent, tile, token_dim=1)
+    idx = torch.from_numpy(oracle.tile_major_index(latent, tile, np.arange(N)))
+    expect = torch.zeros((2, Np) + row_shape, dtype=dtype)
+    expect[:, idx] = x
+    assert torch.equal(y.cpu(), expect)  # padding rows are zero
+    z = torch.empty_like(xd)
+    sta.sta_tile_unreorder(y, z, latent, tile, token_dim=1)
+    assert torch.equal(z, xd)
+
+
+def inputs(latent, B, H, d, seed):
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(4)]
+
+
+@pytest.mark.parametrize("latent,tile,B,H,d,windows", [
+    ((13, 21, 18), (6, 8, 8), 1, 3, 128, [[6, 8, 8], [12, 16, 16], [18, 24, 24]]),
+    ((9, 8, 20), (4, 8, 8), 2, 2, 64, [[8, 8, 16], [4, 8, 24]]),
+    ((7, 9, 9), (2, 8, 8), 1, 2, 128, [[2, 8, 8], [8, 16, 16]]),
+])
+def test_padded_forward_and_backward_all_rows(sta, latent, tile, B, H, d, windows):
+    q, k, v, do = inputs(latent, B, H, d, seed=sum(latent) * 7 + d)
+    scale = 1.0 / np.sqrt(d)
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = sta.sta_attention(qd, kd, vd, plan, scale)
+    o2, lse2 = sta.sta_attention(qd, kd, vd, plan, scale, fused=False)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)  # fused raster path == reorder chain
+    assert sta.sta_last_device_status(plan) == 0
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, scale)
+    compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
+            what=f"padded {latent}")
+    dq, dk, dv = sta.sta_attention_backward(qd, kd, vd, o, lse, dod, plan, scale)
+    assert sta.sta_last_device_status(plan) == 0
+    rq, rk, rv = oracle.sta_backward(q, k, v, do, latent, tile, windows, scale)
+    N = q.shape[2]
+    bh = np.repeat(np.arange(B * H), N)
+    pk_ref, _ = oracle.sta_attention(q, k, k, latent, tile, windows, scale)  # (P K) rows
+    extra = {"dq": dq_d_term(o_ref.reshape(-1, d), pk_ref.reshape(-1, d), do.reshape(-1, d), scale),
+             "dk": dk_d_term(q, k, v, o_ref, do, latent, tile, windows, scale).reshape(-1, d), "dv": None}
+    for name, a, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        compare_grad(a.cpu().reshape(-1, d), r.reshape(-1, d), bh, what=f"{name} padded {latent}",
+                     extra=extra[name])
+
+
+def test_hunyuan_720p_latent_sampled(sta):
+    """33 x 45 x 80 latent, tile 6 x 8 x 8 (padded to 36 x 48 x 80), window
+    18 x 24 x 24, d = 128: sampled rows of corner and padded-edge tiles."""
+    latent, tile, B, H, d = (33, 45, 80), (6, 8, 8), 1, 2, 128
+    windows = [[18, 24, 24], [30, 40, 40]]
+    q, k, v, _ = inputs(latent, B, H, d, seed=3345)
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    o, lse = sta.sta_attention(q.cuda(), k.cuda(), v.cuda(), plan, 1.0 / np.sqrt(d))
+    assert sta.sta_last_device_status(plan) == 0
+    n = [-(-latent[i] // tile[i]) for i in range(3)]
+    tiles = [0, n[1] * n[2] - 1, (n[0] - 1) * n[1] * n[2], n[0] * n[1] * n[2] - 1,
+             ((n[0] - 1) * n[1] + n[1] - 1) * n[2] + 4, (2 * n[1] + n[1] - 1) * n[2] + 3]
+    rng = np.random.default_rng(5)
+    toks = []
+    for t in tiles:
+        tt = oracle.tile_tokens(latent, tile, t)
+        toks.extend(rng.choice(tt, min(24, len(tt)), replace=False).tolist() + [int(tt[0]), int(tt[-1])])
+    toks = sorted(set(toks))
+    rows = np.array([(h, t) for h in range(H) for t in toks], dtype=np.int64)
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, windows, 1.0 / np.sqrt(d), rows=rows)
+    og = o.reshape(-1, o.shape[2], d)[rows[:, 0], rows[:, 1]].cpu()
+    lg = lse.reshape(-1, lse.shape[2])[rows[:, 0], rows[:, 1]].cpu()
+    compare(og, lg, o_ref, lse_ref, what="33x45x80")
