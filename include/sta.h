@@ -214,6 +214,35 @@ STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, c
                                     const void* o_full, int64_t slices, int64_t tokens, int32_t head_dim,
                                     double* recall, double* mse, void* stream);
 
+/* Forward pipeline from host memory (no counterpart on the pages: a runtime
+ * piece for callers whose Q, K, V live in host memory).  At the pages' 720p
+ * size the PCIe copies of one call take longer than its attention, so the
+ * pipeline overlaps them across calls: a ring of `depth` device buffer sets
+ * and three streams, the copy-in of call i+1, the forward (sta_forward_raster)
+ * of call i and the copy-out of call i-1 running at once.
+ *
+ * sta_pipe_create: plan from sta_plan on the current device (its tile shape
+ *   must suit sta_forward_raster, else UNSUPPORTED); head_dim 64 or 128;
+ *   softmax_scale finite and > 0; 1 <= depth <= 8.  Allocates depth x (four
+ *   [B, heads, N, d] bf16 tensors + one fp32 LSE) of device memory and three
+ *   streams; OOM / CUDA on failure.  The plan must outlive the pipeline.
+ * sta_pipe_submit: enqueue one call on raster-order host tensors: q, k, v
+ *   read and o, lse written, shapes as sta_forward_raster.  Returns at once.
+ *   The host buffers should be pinned (cudaHostAlloc, or pin_memory in
+ *   PyTorch) or the copies do not overlap; q, k, v must stay unchanged and
+ *   o, lse unread until sta_pipe_wait.  INVALID_ARG on null pointers or a
+ *   different current device.
+ * sta_pipe_wait: block until all submitted calls are done; returns the first
+ *   CUDA error or the plan's device status (as sta_last_device_status).
+ * sta_pipe_destroy: wait, then free everything (NULL accepted). */
+typedef struct sta_pipe_s* sta_pipe_t;
+STA_API sta_status sta_pipe_create(sta_plan_t p, int32_t head_dim, float softmax_scale, int32_t depth,
+                                   sta_pipe_t* out);
+STA_API sta_status sta_pipe_submit(sta_pipe_t pipe, const void* q_host, const void* k_host,
+                                   const void* v_host, void* o_host, float* lse_host);
+STA_API sta_status sta_pipe_wait(sta_pipe_t pipe);
+STA_API sta_status sta_pipe_destroy(sta_pipe_t pipe);
+
 /* STA forward that allocates nothing (this call has no counterpart in the
  * paper; it exists for deployment).
  *

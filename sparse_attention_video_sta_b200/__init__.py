@@ -33,6 +33,7 @@ __all__ = [
     "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
     "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
     "sta_backward", "sta_attention_backward", "StaAttention", "sta_window_stats", "sta_window_search",
+    "Pipe", "sta_pipe_create",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +51,7 @@ EXPORTED_SYMBOLS = (
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
+    "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy",
 )
 
 
@@ -82,6 +84,10 @@ def _load() -> ctypes.CDLL:
         "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_backward": [vp] * 11 + [i32, ctypes.c_float, vp],
         "sta_window_stats": [vp, vp, vp, vp, i64, i64, i32, vp, vp, vp],
+        "sta_pipe_create": [vp, i32, ctypes.c_float, i32, ctypes.POINTER(vp)],
+        "sta_pipe_submit": [vp, vp, vp, vp, vp, vp],
+        "sta_pipe_wait": [vp],
+        "sta_pipe_destroy": [vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
     }
@@ -567,3 +573,55 @@ def sta_window_search(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, latent,
         chosen.append(list(pick))
     return {"windows": chosen, "recall": recall, "mse": mse, "candidates": [list(c) for c in cands],
             "tiles": tiles}
+
+
+class Pipe:
+    """STA forward from host memory with copy-in, forward and copy-out of
+    consecutive calls overlapped (``sta_pipe_*`` in ``include/sta.h``)."""
+
+    def __init__(self, handle: int, plan: Plan, head_dim: int):
+        self._h = ctypes.c_void_p(handle)
+        self.plan = plan  # kept alive: the pipeline uses it
+        self.head_dim = int(head_dim)
+
+    def submit(self, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+               lse: torch.Tensor) -> None:
+        """Enqueue one call on pinned host tensors (raster order): reads q, k, v,
+        writes o and lse once ``wait`` returns."""
+        B, H, N, d = self.plan.batch, self.plan.heads, self.plan.tokens, self.head_dim
+        for name, t, shape, dt in (("q", q, (B, H, N, d), torch.bfloat16), ("k", k, (B, H, N, d), torch.bfloat16),
+                                   ("v", v, (B, H, N, d), torch.bfloat16), ("o", o, (B, H, N, d), torch.bfloat16),
+                                   ("lse", lse, (B, H, N), torch.float32)):
+            if t.is_cuda or t.dtype != dt or not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be a contiguous host {dt} tensor of shape {shape}")
+            if not t.is_pinned():
+                raise ValueError(f"{name} must be in pinned host memory (tensor.pin_memory())")
+        _check(_lib.sta_pipe_submit(self._h, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                    ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                    ctypes.c_void_p(lse.data_ptr())), "sta_pipe_submit")
+
+    def wait(self) -> None:
+        _check(_lib.sta_pipe_wait(self._h), "sta_pipe_wait")
+
+    def destroy(self) -> None:
+        if self._h:
+            _check(_lib.sta_pipe_destroy(self._h), "sta_pipe_destroy")
+            self._h = ctypes.c_void_p(0)
+
+    def __del__(self):
+        try:
+            if self._h:
+                _lib.sta_pipe_destroy(self._h)
+                self._h = ctypes.c_void_p(0)
+        except Exception:
+            pass
+
+
+def sta_pipe_create(plan: Plan, head_dim: int, softmax_scale: float | None = None, depth: int = 2) -> Pipe:
+    """Pipeline of ``depth`` device buffer sets for ``plan`` on the current device."""
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(head_dim)
+    h = ctypes.c_void_p(0)
+    _check(_lib.sta_pipe_create(plan.handle, int(head_dim), float(softmax_scale), int(depth), ctypes.byref(h)),
+           "sta_pipe_create")
+    return Pipe(h.value, plan, head_dim)

@@ -11,7 +11,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libsta.so")
 
-SOURCES = ["sta_api.cu", "sta_permute.cu", "sta_forward.cu", "sta_backward.cu", "sta_search.cu", "sta_noalloc.cu"]
+SOURCES = ["sta_api.cu", "sta_permute.cu", "sta_forward.cu", "sta_backward.cu", "sta_search.cu", "sta_pipe.cu", "sta_noalloc.cu"]
 HEADERS = ["sta_internal.h", "sta_ptx.cuh", "sta_wait.cuh"]
 
 NVCC_FLAGS = [

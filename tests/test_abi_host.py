@@ -237,3 +237,17 @@ def test_padded_plan_lists_match_oracle_mask(latent, tile, windows):
             attends.append(set(got))
         for kt in range(n_tiles):
             assert p.key_query(h, kt) == [q for q in range(n_tiles) if kt in attends[q]]
+
+
+def test_pipe_rejected_before_allocation():
+    INV = sta.STA_ERR_INVALID_ARG
+    lib = sta._lib
+    hp = sta.sta_plan_host((18, 24, 24), (6, 8, 8), 1, 2, [(12, 16, 16)] * 2)
+    out = ctypes.c_void_p(0)
+    assert lib.sta_pipe_create(hp.handle, 64, 0.125, 2, ctypes.byref(out)) == INV  # host-only plan
+    assert lib.sta_pipe_create(None, 64, 0.125, 2, ctypes.byref(out)) == INV
+    assert lib.sta_pipe_create(hp.handle, 64, 0.125, 2, None) == INV
+    assert lib.sta_pipe_submit(None, None, None, None, None, None) == INV
+    assert lib.sta_pipe_wait(None) == INV
+    assert lib.sta_pipe_destroy(None) == 0
+    hp.destroy()
