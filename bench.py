@@ -241,21 +241,22 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def time_backward(sta, plan, forward, qt, kt, vt, ot, lset, scale, gen, flops, warmup, reps, reduce_max):
-    """Time sta_backward on the tile-major tensors after one forward; returns
-    its figures.  Algorithmic work: five tile-pair products (S, dP, dV, dK, dQ)
+def time_backward(sta, plan, q, k, v, o, lse, scale, gen, flops, warmup, reps, reduce_max):
+    """Time the backward on the raster tensors (``sta_backward_raster``, the
+    permutation fused; ``o``, ``lse`` from the fused forward); returns its
+    figures.  Algorithmic work: five tile-pair products (S, dP, dV, dK, dQ)
     against the forward's two."""
-    forward()
-    dout = torch.empty_like(qt)
-    B, H, N, d = qt.shape
+    sta.sta_forward_raster(plan, q, k, v, o, lse, scale)
+    dout = torch.empty_like(q)
+    B, H, N, d = q.shape
     for b in range(B):
         for h in range(H):
-            dout[b, h].copy_(torch.randn((N, d), generator=gen, device=qt.device, dtype=torch.float32))
-    dq, dk, dv = (torch.empty_like(qt) for _ in range(3))
-    ws = torch.empty(2 * B * H * N, dtype=torch.float32, device=qt.device)
+            dout[b, h].copy_(torch.randn((N, d), generator=gen, device=q.device, dtype=torch.float32))
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    ws = torch.empty(2 * B * H * plan.padded_tokens, dtype=torch.float32, device=q.device)
 
     def bwd_step():
-        sta.sta_backward(plan, qt, kt, vt, ot, lset, dout, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+        sta.sta_backward_raster(plan, q, k, v, o, lse, dout, scale, dq=dq, dk=dk, dv=dv, workspace=ws)
 
     for _ in range(warmup):
         bwd_step()
@@ -271,7 +272,7 @@ def time_backward(sta, plan, forward, qt, kt, vt, ot, lset, scale, gen, flops, w
         raise RuntimeError("device status error in the backward run")
     bwd_flops = 2.5 * flops
     return {"ms": bwd_ms, "tflops": bwd_flops / (bwd_ms * 1e-3) / 1e12, "flops": bwd_flops,
-            "launches": 3, "layout": "tile-major"}
+            "launches": 3, "layout": "raster (permutation fused)"}
 
 
 def main():
@@ -347,8 +348,8 @@ def main():
         sta.sta_tile_unreorder(lset, lse, L, T, token_dim=2)
 
     if args.backward_only:
-        res = time_backward(sta, plan, permuted_step, qt, kt, vt, ot, lset, scale, gen, flops,
-                            max(3, args.warmup), args.steps, reduce_max)
+        res = time_backward(sta, plan, q, k, v, o, lse, scale, gen, flops, max(3, args.warmup), args.steps,
+                            reduce_max)
         if rank == 0:
             print(json.dumps({"workload": w.name, "backward": res}), flush=True)
         return
@@ -454,8 +455,7 @@ def main():
                                  "bytes_per_launch": 2 * nbytes}
         extras["permutation"]["frac"] = extras["permutation"]["gbs"] / extras["permutation"]["peak_gbs"]
         # ------------------------------------------- backward (tile-major, 3 launches)
-        extras["backward"] = time_backward(sta, plan, permuted_step, qt, kt, vt, ot, lset, scale, gen,
-                                           flops, 2, 3, reduce_max)
+        extras["backward"] = time_backward(sta, plan, q, k, v, o, lse, scale, gen, flops, 2, 3, reduce_max)
         # ------------------------------------------- end to end from pinned host memory
         # Through the host-memory pipeline (sta_pipe_*): each step copies its
         # Q, K, V in from pinned host buffers and O, LSE back out; copy-in,

@@ -178,7 +178,8 @@ STA_API sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k
  *                from every input)
  *   workspace  : device fp32, 2 * B * heads * N floats, 16-byte aligned,
  *                caller-owned; on return plane 0 holds -D_i and plane 1
- *                -lse_i * log2(e) (row order of lse)
+ *                -lse_i * log2(e), tile-major (N = tiles x tile volume, the
+ *                tile-major row count)
  *   head_dim, softmax_scale: as sta_forward
  * P and dS enter the tensor-core products as bf16 with fp32 accumulation;
  * dq, dk, dv are rounded to bf16.  No atomics: results are deterministic.
@@ -189,6 +190,18 @@ STA_API sta_status sta_backward(sta_plan_t p, const void* q, const void* k, cons
                                 const void* o, const void* dout, const float* lse, void* dq,
                                 void* dk, void* dv, float* workspace, int32_t head_dim,
                                 float softmax_scale, void* stream);
+
+/* STA backward on raster-order tensors, the token permutation fused into the
+ * kernels' loads and stores: q, k, v, o, dout, dq, dk, dv are [B, heads, N, d]
+ * and lse [B, heads, N] in raster order (N = L_t * L_h * L_w), as written by
+ * sta_forward_raster; the workspace is as for sta_backward (tile-major, whole
+ * tiles: 2 * B * heads * tiles * tile volume floats).  Same arithmetic and
+ * results as permuting to tile-major, sta_backward, and permuting back, bit for
+ * bit.  Tile shapes as sta_forward_raster (else UNSUPPORTED). */
+STA_API sta_status sta_backward_raster(sta_plan_t p, const void* q, const void* k, const void* v,
+                                       const void* o, const void* dout, const float* lse, void* dq,
+                                       void* dk, void* dv, float* workspace, int32_t head_dim,
+                                       float softmax_scale, void* stream);
 
 /* Per-(b, h) statistics of a candidate window against the full window, for
  * choosing a window per head by profiling ("Fast Video Generation with Sliding

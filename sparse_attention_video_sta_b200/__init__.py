@@ -33,7 +33,7 @@ __all__ = [
     "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
     "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
     "sta_backward", "sta_attention_backward", "StaAttention", "sta_window_stats", "sta_window_search",
-    "Pipe", "sta_pipe_create",
+    "Pipe", "sta_pipe_create", "sta_backward_raster",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -51,7 +51,7 @@ EXPORTED_SYMBOLS = (
     "sta_plan_work_items", "sta_tile_reorder", "sta_tile_unreorder", "sta_forward",
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
-    "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy",
+    "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy", "sta_backward_raster",
 )
 
 
@@ -83,6 +83,7 @@ def _load() -> ctypes.CDLL:
         "sta_forward_raster": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_forward_noalloc": [G, i32, i32, i32p, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
         "sta_backward": [vp] * 11 + [i32, ctypes.c_float, vp],
+        "sta_backward_raster": [vp] * 11 + [i32, ctypes.c_float, vp],
         "sta_window_stats": [vp, vp, vp, vp, i64, i64, i32, vp, vp, vp],
         "sta_pipe_create": [vp, i32, ctypes.c_float, i32, ctypes.POINTER(vp)],
         "sta_pipe_submit": [vp, vp, vp, vp, vp, vp],
@@ -358,31 +359,46 @@ def sta_forward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Te
     return o, lse
 
 
-def sta_backward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
-                 lse: torch.Tensor, dout: torch.Tensor, softmax_scale: float, dq=None, dk=None, dv=None,
-                 workspace=None, stream=None):
-    """STA backward on tile-major ``[B, H, N, d]`` bf16 tensors (``o`` and ``lse``
-    from ``sta_forward``).  Returns ``(dq, dk, dv)``; outputs and the fp32
-    workspace (``2 * B * H * N`` floats) are allocated when not given."""
-    args = _forward_args(plan, q, k, v, o, lse)
-    B, H, N, d = q.shape
+def _backward_call(fn, what: str, plan: Plan, q, k, v, o, lse, dout, softmax_scale, dq, dk, dv, workspace,
+                   stream, raster: bool):
+    args = _forward_args(plan, q, k, v, o, lse, raster=raster)
+    B, H = plan.batch, plan.heads
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     for name, t in (("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
         if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
             raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(q.shape)}")
+    n_ws = 2 * B * H * plan.padded_tokens
     if workspace is None:
-        workspace = torch.empty(2 * B * H * N, dtype=torch.float32, device=q.device)
+        workspace = torch.empty(n_ws, dtype=torch.float32, device=q.device)
     if not workspace.is_cuda or workspace.dtype != torch.float32 or not workspace.is_contiguous() \
-            or workspace.numel() < 2 * B * H * N:
-        raise ValueError(f"workspace must be a contiguous CUDA fp32 tensor of {2 * B * H * N} floats")
+            or workspace.numel() < n_ws:
+        raise ValueError(f"workspace must be a contiguous CUDA fp32 tensor of {n_ws} floats")
     qp, kp, vp_, op, lp, hd = args
-    _check(_lib.sta_backward(plan.handle, qp, kp, vp_, op, ctypes.c_void_p(dout.data_ptr()), lp,
-                             ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
-                             ctypes.c_void_p(dv.data_ptr()), ctypes.c_void_p(workspace.data_ptr()), hd,
-                             float(softmax_scale), _stream(stream)), "sta_backward")
+    _check(fn(plan.handle, qp, kp, vp_, op, ctypes.c_void_p(dout.data_ptr()), lp,
+              ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()), ctypes.c_void_p(dv.data_ptr()),
+              ctypes.c_void_p(workspace.data_ptr()), hd, float(softmax_scale), _stream(stream)), what)
     return dq, dk, dv
+
+
+def sta_backward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                 lse: torch.Tensor, dout: torch.Tensor, softmax_scale: float, dq=None, dk=None, dv=None,
+                 workspace=None, stream=None):
+    """STA backward on tile-major ``[B, H, N_tiles, d]`` bf16 tensors (``o`` and
+    ``lse`` from ``sta_forward``).  Returns ``(dq, dk, dv)``; outputs and the fp32
+    workspace (``2 * B * H * N_tiles`` floats) are allocated when not given."""
+    return _backward_call(_lib.sta_backward, "sta_backward", plan, q, k, v, o, lse, dout, softmax_scale,
+                          dq, dk, dv, workspace, stream, raster=False)
+
+
+def sta_backward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                        lse: torch.Tensor, dout: torch.Tensor, softmax_scale: float, dq=None, dk=None, dv=None,
+                        workspace=None, stream=None):
+    """STA backward on raster-order ``[B, H, N, d]`` bf16 tensors (``o`` and
+    ``lse`` from ``sta_forward_raster``), the permutation fused into the kernels."""
+    return _backward_call(_lib.sta_backward_raster, "sta_backward_raster", plan, q, k, v, o, lse, dout,
+                          softmax_scale, dq, dk, dv, workspace, stream, raster=True)
 
 
 def raster_supported(tile, latent=None) -> bool:
@@ -465,13 +481,18 @@ def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,
 
 def sta_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                            lse: torch.Tensor, dout: torch.Tensor, plan: Plan,
-                           softmax_scale: float | None = None, stream=None):
-    """Gradients ``(dq, dk, dv)`` of ``sta_attention`` on raster-order tensors:
-    the inputs are permuted to tile-major order, ``sta_backward`` runs, and the
-    gradients are permuted back."""
+                           softmax_scale: float | None = None, stream=None, fused: bool = True):
+    """Gradients ``(dq, dk, dv)`` of ``sta_attention`` on raster-order tensors.
+
+    With ``fused`` (and a tile shape the fused kernels handle) the kernels read
+    and write raster order directly; otherwise the inputs are permuted to
+    tile-major order, ``sta_backward`` runs, and the gradients are permuted
+    back.  Both give the same bits."""
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(q.shape[-1])
     lat, tile = plan.latent, plan.tile
+    if fused and raster_supported(tile, lat):
+        return sta_backward_raster(plan, q, k, v, o, lse, dout, softmax_scale, stream=stream)
 
     def to_tiles(x):
         y = _tile_major_like(x, plan)

@@ -41,6 +41,20 @@ sta_status cuda_status(cudaError_t e) {
     return e == cudaErrorMemoryAllocation ? STA_ERR_OOM : STA_ERR_CUDA;
 }
 
+// Launches report their errors through cudaGetLastError, which also returns
+// an error left behind by any earlier runtime call of this thread (for
+// example one made by the framework on an autograd worker thread).  Entry
+// points clear that record before they launch, so a status describes only
+// this call.  Sticky errors (a lost context) are reported by the calls that
+// follow.
+void clear_stale_error() { (void)cudaGetLastError(); }
+
+// The kernels' tensor maps are encoded through the driver API, which needs
+// the device's context current in the calling thread; a thread whose first
+// CUDA call this is (an autograd worker thread, a thread pool) has none until
+// the runtime sets it up.  cudaSetDevice on the current device does.
+cudaError_t make_context_current(int dev) { return cudaSetDevice(dev); }
+
 bool geom_valid(const sta_geom* g) {
     if (g == nullptr) return false;
     const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
@@ -304,6 +318,7 @@ sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row
     const int64_t s_bytes = inverse ? t_bytes : r_bytes, d_bytes = inverse ? r_bytes : t_bytes;
     const uintptr_t s = reinterpret_cast<uintptr_t>(src), d = reinterpret_cast<uintptr_t>(dst);
     if (s < d + uint64_t(d_bytes) && d < s + uint64_t(s_bytes)) return STA_ERR_INVALID_ARG;  // overlap
+    clear_stale_error();
     return cuda_status(sta::launch_permute(src, dst, outer, row_bytes, *g, inverse,
                                            static_cast<cudaStream_t>(stream)));
 }
@@ -321,10 +336,12 @@ sta_status forward_common(sta_plan_t p, const void* q, const void* k, const void
     int dev = -1;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
     if (dev != p->device) return STA_ERR_INVALID_ARG;
+    if (cudaError_t e = make_context_current(dev); e != cudaSuccess) return cuda_status(e);
     const int inject = g_inject_timeout.load();
     const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
                                   : kDefaultTimeoutNs;
     if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
+    clear_stale_error();
     return cuda_status(sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
                                            static_cast<cudaStream_t>(stream), inject, limit, raster));
 }
@@ -349,6 +366,27 @@ sta_status plan_host_for(const sta_geom* g, int32_t batch, int32_t heads, const 
     }
     *out = p;
     return STA_OK;
+}
+
+sta_status backward_common(sta_plan_t p, const void* q, const void* k, const void* v, const void* o,
+                           const void* dout, const float* lse, void* dq, void* dk, void* dv, float* workspace,
+                           int32_t head_dim, float softmax_scale, void* stream, bool raster) {
+    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    const void* in16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
+    for (const void* x : in16)
+        if (x == nullptr || !aligned(x, 16)) return STA_ERR_INVALID_ARG;
+    if (lse == nullptr || !aligned(lse, 4)) return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
+    if (dev != p->device) return STA_ERR_INVALID_ARG;
+    if (cudaError_t e = make_context_current(dev); e != cudaSuccess) return cuda_status(e);
+    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
+    clear_stale_error();
+    return cuda_status(sta::launch_backward(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim,
+                                            softmax_scale, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs,
+                                            raster));
 }
 
 }  // namespace
@@ -492,19 +530,15 @@ sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k, const 
 sta_status sta_backward(sta_plan_t p, const void* q, const void* k, const void* v, const void* o,
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
                         float* workspace, int32_t head_dim, float softmax_scale, void* stream) {
-    if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
-    const void* in16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
-    for (const void* x : in16)
-        if (x == nullptr || !aligned(x, 16)) return STA_ERR_INVALID_ARG;
-    if (lse == nullptr || !aligned(lse, 4)) return STA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
-    int dev = -1;
-    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
-    if (dev != p->device) return STA_ERR_INVALID_ARG;
-    return cuda_status(sta::launch_backward(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim,
-                                            softmax_scale, static_cast<cudaStream_t>(stream),
-                                            kDefaultTimeoutNs));
+    return backward_common(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim, softmax_scale, stream,
+                           false);
+}
+
+sta_status sta_backward_raster(sta_plan_t p, const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               float* workspace, int32_t head_dim, float softmax_scale, void* stream) {
+    return backward_common(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim, softmax_scale, stream,
+                           true);
 }
 
 sta_status sta_window_stats(const float* lse_w, const float* lse_full, const void* o_w, const void* o_full,
@@ -519,6 +553,7 @@ sta_status sta_window_stats(const float* lse_w, const float* lse_full, const voi
     // 8 CTAs per slice in the launch grid
     if (slices < 1 || slices > (int64_t(1) << 28) || tokens < 1 || head_dim < 8 || head_dim % 8 != 0)
         return STA_ERR_INVALID_ARG;
+    clear_stale_error();
     return cuda_status(sta::launch_window_stats(lse_w, lse_full, o_w, o_full, slices, tokens, head_dim, recall,
                                                 mse, static_cast<cudaStream_t>(stream)));
 }

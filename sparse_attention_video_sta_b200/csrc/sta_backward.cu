@@ -45,6 +45,7 @@
 
 #include "sta_internal.h"
 #include "sta_ptx.cuh"
+#include "sta_raster.cuh"
 #include "sta_wait.cuh"
 
 namespace sta {
@@ -80,6 +81,7 @@ struct BwdParams {
     float scale;
     uint32_t* status;
     uint64_t timeout_ns;
+    RasterGeom rg;  // raster layout only
 };
 
 __device__ __forceinline__ bool wait_bw(uint32_t bar, uint32_t parity, volatile int* abort_flag, const BwdParams& p) {
@@ -93,6 +95,25 @@ __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* m, ui
     for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * kBoxBytes, m, bar, cb * 64, row);
 }
 
+// 128-row block `sub` of tile `tile` of head bh: tile-major rows (2D map) or
+// a raster box (5D map).
+template <int D, bool kRaster>
+__device__ __forceinline__ void load_blk(uint32_t dst, const CUtensorMap* m, uint32_t bar, const BwdParams& p,
+                                         int32_t bh, int32_t tile, int32_t sub) {
+    if (!kRaster)
+        load_rows<D>(dst, m, bar, bh * p.tokens + tile * p.tile_tokens + sub * 128);
+    else
+        raster_load(dst, m, bar, p.rg, bh, tile, sub, D / 64, kBoxBytes);
+}
+
+// Output row of row `r` of block `blk` of head bh; -1 for a padding row of a
+// raster output.
+template <bool kRaster, bool kPadded>
+__device__ __forceinline__ int64_t bwd_out_row(const BwdParams& p, int32_t bh, int32_t blk, int32_t r) {
+    if (!kRaster) return int64_t(bh) * p.tokens + int64_t(blk) * 128 + r;
+    return raster_row<kPadded>(p.rg, bh, blk, r);
+}
+
 // 64 fp32 values -> 32 bf16 pairs.
 __device__ __forceinline__ void pack64(const float (&x)[64], uint32_t (&pk)[32]) {
 #pragma unroll
@@ -101,13 +122,15 @@ __device__ __forceinline__ void pack64(const float (&x)[64], uint32_t (&pk)[32])
 
 // Epilogue: `cols` fp32 TMEM columns of this thread's lane (starting at taddr),
 // times `mul`, as bf16 to dst (16-byte aligned, cols contiguous elements).
+// Every lane loads (the TMEM access is warp-wide); only lanes with `store` write.
 template <int kCols>
-__device__ __forceinline__ void store_cols(uint32_t taddr, float mul, __nv_bfloat16* dst) {
+__device__ __forceinline__ void store_cols(uint32_t taddr, float mul, __nv_bfloat16* dst, bool store) {
     uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll 1
     for (int cb = 0; cb < kCols / 32; ++cb) {
         uint32_t r[32];
         ptx::tmem_ld32(taddr + cb * 32, r);
+        if (!store) continue;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             uint4 v;
@@ -126,19 +149,29 @@ __device__ __forceinline__ void store_cols(uint32_t taddr, float mul, __nv_bfloa
 __device__ __forceinline__ uint32_t a_col(int kk) { return uint32_t((kk >> 2) * 64 + (kk & 3) * 8); }
 
 // ---------------------------------------------------------------- prep
-// neg_d[r] = -sum_c dO[r, c] O[r, c];  neg_l[r] = -lse[r] log2(e).
+// neg_d[r] = -sum_c dO[r, c] O[r, c];  neg_l[r] = -lse[r] log2(e), for every
+// tile-major row r (the planes are tile-major in both layouts, so a 128-row
+// block's values are one contiguous 512-byte copy).  kRaster: O, dO and LSE
+// are raster tensors, read at the row's raster token; a padding row gets 0
+// for both (its dO is 0, so it adds nothing to dK or dV).
 // D / 8 threads per row, 16 bytes of each tensor per thread.
-template <int D>
+template <int D, bool kRaster, bool kPadded>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__ o, const uint4* __restrict__ dout,
                                                        const float* __restrict__ lse, float* __restrict__ neg_d,
-                                                       float* __restrict__ neg_l, int64_t rows) {
+                                                       float* __restrict__ neg_l, int64_t rows, int32_t tokens,
+                                                       const RasterGeom rg) {
     constexpr int kTpr = D / 8;
     const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t row = t / kTpr;
     const int part = int(t % kTpr);
+    int64_t src = row;
+    if (kRaster && row < rows) {
+        const int32_t bh = int32_t(row / tokens), within = int32_t(row % tokens);
+        src = raster_row<kPadded>(rg, bh, within / 128, within % 128);
+    }
     float acc = 0.0f;
-    if (row < rows) {
-        const uint4 a = __ldg(o + row * kTpr + part), b = __ldg(dout + row * kTpr + part);
+    if (row < rows && src >= 0) {
+        const uint4 a = __ldg(o + src * kTpr + part), b = __ldg(dout + src * kTpr + part);
         const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -150,7 +183,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__
     for (int s = kTpr / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
     if (row < rows && part == 0) {
         neg_d[row] = -acc;
-        neg_l[row] = -lse[row] * kLog2e;
+        neg_l[row] = src >= 0 ? -lse[src] * kLog2e : 0.0f;
     }
 }
 
@@ -173,7 +206,7 @@ struct DqCfg {
     static_assert(kColDQ + D <= kBwTmemCols, "TMEM budget");
 };
 
-template <int D>
+template <int D, bool kRaster, bool kPadded>
 __global__ void __launch_bounds__(kBwThreads, 1)
 sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -247,22 +280,20 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int32_t* list = p.ids + off[tile];
                 const int32_t n_kt = off[tile + 1] - off[tile];
                 if (!wait_bw(q_empty, (qc & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                const int32_t qrow = w.bh * p.tokens + w.qa * 128;
                 ptx::mbar_arrive_expect_tx(q_full, 2 * C::kBlk);
-                load_rows<D>(base + C::kQOff, &tm_q, q_full, qrow);
-                load_rows<D>(base + C::kDOOff, &tm_do, q_full, qrow);
+                load_blk<D, kRaster>(base + C::kQOff, &tm_q, q_full, p, w.bh, tile, w.qa - tile * SPT);
+                load_blk<D, kRaster>(base + C::kDOOff, &tm_do, q_full, p, w.bh, tile, w.qa - tile * SPT);
                 ++qc;
                 for (int32_t kt = 0; ok && kt < n_kt; ++kt) {
                     const int32_t t = __ldg(list + kt);
                     for (int32_t kc = 0; ok && kc < SPT; ++kc) {
-                        const int32_t row = w.bh * p.tokens + t * p.tile_tokens + kc * 128;
                         const int rk = int(kit % KS);
                         if (kit >= uint32_t(KS) && !wait_bw(k_empty(rk), ((kit / KS) - 1) & 1u, abort_flag, p)) {
                             ok = false;
                             break;
                         }
                         ptx::mbar_arrive_expect_tx(k_full(rk), C::kBlk);
-                        load_rows<D>(base + C::kKOff + rk * C::kBlk, &tm_k, k_full(rk), row);
+                        load_blk<D, kRaster>(base + C::kKOff + rk * C::kBlk, &tm_k, k_full(rk), p, w.bh, t, kc);
                         ++kit;
                         const int rv = int(vit % VS);
                         if (vit >= uint32_t(VS) && !wait_bw(v_empty(rv), ((vit / VS) - 1) & 1u, abort_flag, p)) {
@@ -270,7 +301,7 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             break;
                         }
                         ptx::mbar_arrive_expect_tx(v_full(rv), C::kBlk);
-                        load_rows<D>(base + C::kVOff + rv * C::kBlk, &tm_v, v_full(rv), row);
+                        load_blk<D, kRaster>(base + C::kVOff + rv * C::kBlk, &tm_v, v_full(rv), p, w.bh, t, kc);
                         ++vit;
                     }
                 }
@@ -425,8 +456,9 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (!__all_sync(0xffffffffu, wait_bw(dq_full, dqc & 1u, abort_flag, p))) break;
             ++dqc;
             ptx::tc_fence_after();
+            const int64_t orow = bwd_out_row<kRaster, kPadded>(p, w.bh, w.qa, row);
             store_cols<D / 2>(tmem + lane_addr + C::kColDQ + uint32_t(D / 2) * h, p.scale,
-                              p.out_a + grow * D + (D / 2) * h);
+                              p.out_a + (orow < 0 ? 0 : orow) * D + (D / 2) * h, orow >= 0);
             ptx::tc_fence_before();
             gs += uint32_t(n);
         }
@@ -463,7 +495,7 @@ struct DkvCfg {
     static_assert(kColDK + D <= kBwTmemCols, "TMEM budget");
 };
 
-template <int D>
+template <int D, bool kRaster, bool kPadded>
 __global__ void __launch_bounds__(kBwThreads, 1)
 sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -531,10 +563,9 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int32_t* list = p.ids + off[ktile];
                 const int32_t n_qt = off[ktile + 1] - off[ktile];
                 if (!wait_bw(kv_empty, (kvc & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                const int32_t krow = w.bh * p.tokens + w.qa * 128;
                 ptx::mbar_arrive_expect_tx(kv_full, 2 * C::kBlk);
-                load_rows<D>(base + C::kKOff, &tm_k, kv_full, krow);
-                load_rows<D>(base + C::kVOff, &tm_v, kv_full, krow);
+                load_blk<D, kRaster>(base + C::kKOff, &tm_k, kv_full, p, w.bh, ktile, w.qa - ktile * SPT);
+                load_blk<D, kRaster>(base + C::kVOff, &tm_v, kv_full, p, w.bh, ktile, w.qa - ktile * SPT);
                 ++kvc;
                 for (int32_t qt = 0; ok && qt < n_qt; ++qt) {
                     const int32_t t = __ldg(list + qt);
@@ -546,8 +577,8 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
                         const int32_t row = w.bh * p.tokens + t * p.tile_tokens + sub * 128;
                         ptx::mbar_arrive_expect_tx(st_full(r), C::kStageBytes);
-                        load_rows<D>(stage(r) + C::kStQ, &tm_q, st_full(r), row);
-                        load_rows<D>(stage(r) + C::kStDO, &tm_do, st_full(r), row);
+                        load_blk<D, kRaster>(stage(r) + C::kStQ, &tm_q, st_full(r), p, w.bh, t, sub);
+                        load_blk<D, kRaster>(stage(r) + C::kStDO, &tm_do, st_full(r), p, w.bh, t, sub);
                         ptx::bulk_load(stage(r) + C::kStL, p.neg_l + row, 512, st_full(r));
                         ptx::bulk_load(stage(r) + C::kStD, p.neg_d + row, 512, st_full(r));
                         ++sit;
@@ -728,11 +759,12 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!__all_sync(0xffffffffu, wait_bw(dkv_full, kvc & 1u, abort_flag, p))) break;
             ++kvc;
             ptx::tc_fence_after();
-            const int64_t grow = int64_t(w.bh) * p.tokens + int64_t(w.qa) * 128 + row;
+            const int64_t orow = bwd_out_row<kRaster, kPadded>(p, w.bh, w.qa, row);
+            const int64_t safe = orow < 0 ? 0 : orow;
             store_cols<D / 2>(tmem + lane_addr + C::kColDV + uint32_t(D / 2) * h, 1.0f,
-                              p.out_b + grow * D + (D / 2) * h);
+                              p.out_b + safe * D + (D / 2) * h, orow >= 0);
             store_cols<D / 2>(tmem + lane_addr + C::kColDK + uint32_t(D / 2) * h, p.scale,
-                              p.out_a + grow * D + (D / 2) * h);
+                              p.out_a + safe * D + (D / 2) * h, orow >= 0);
             ptx::tc_fence_before();
             gs += uint32_t(n);
             sbase += uint32_t(n);
@@ -780,27 +812,78 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D>
-cudaError_t launch_bwd_d(const sta_plan_s* pl, const void* q, const void* k, const void* v, const void* o,
-                         const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
-                         float scale, cudaStream_t stream, uint64_t timeout_ns) {
+// The three launches of one (layout, padding) variant.
+template <int D, bool kRaster, bool kPadded>
+cudaError_t launch_bwd_variant(const sta_plan_s* pl, const CUtensorMap& mq, const CUtensorMap& mk,
+                               const CUtensorMap& mv, const CUtensorMap& mdo, BwdParams bp, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv, int64_t rows,
+                               int sms, cudaStream_t stream) {
     const PlanHost& P = pl->h;
-    const int64_t rows = int64_t(P.batch) * P.heads * P.tiles_per_head * P.tile_tokens;
-    if (rows == 0) return cudaSuccess;
-    float* neg_d = ws;
-    float* neg_l = ws + rows;
     {
         const int64_t threads = rows * (D / 8);
         const int64_t blocks = (threads + 255) / 256;
-        bwd_prep_kernel<D><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
-            static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, neg_d, neg_l, rows);
+        bwd_prep_kernel<D, kRaster, kPadded><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
+            static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, const_cast<float*>(bp.neg_d),
+            const_cast<float*>(bp.neg_l), rows, bp.tokens, bp.rg);
         if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
     }
+    // dQ
+    bp.items = pl->d_bq_items;
+    bp.n_items = int32_t(P.bq_items.size());
+    bp.off = pl->d_off;
+    bp.ids = pl->d_ids;
+    bp.out_a = static_cast<__nv_bfloat16*>(dq);
+    bp.out_b = nullptr;
+    int grid = bp.n_items < sms ? bp.n_items : sms;
+    if (grid <= 0) return cudaSuccess;
+    constexpr int kSmemDq = smem_launch(DqCfg<D>::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(sta_bwd_dq_kernel<D, kRaster, kPadded>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
+    if (e != cudaSuccess) return e;
+    sta_bwd_dq_kernel<D, kRaster, kPadded><<<grid, kBwThreads, kSmemDq, stream>>>(mq, mk, mv, mdo, bp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // dK, dV
+    bp.items = pl->d_bkv_items;
+    bp.n_items = int32_t(P.bkv_items.size());
+    bp.off = pl->d_toff;
+    bp.ids = pl->d_tids;
+    bp.out_a = static_cast<__nv_bfloat16*>(dk);
+    bp.out_b = static_cast<__nv_bfloat16*>(dv);
+    grid = bp.n_items < sms ? bp.n_items : sms;
+    constexpr int kSmemDkv = smem_launch(DkvCfg<D>::kSmemBytes);
+    e = cudaFuncSetAttribute(sta_bwd_dkdv_kernel<D, kRaster, kPadded>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemDkv);
+    if (e != cudaSuccess) return e;
+    sta_bwd_dkdv_kernel<D, kRaster, kPadded><<<grid, kBwThreads, kSmemDkv, stream>>>(mq, mk, mv, mdo, bp);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const sta_plan_s* pl, const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
+                         float scale, cudaStream_t stream, uint64_t timeout_ns, bool raster) {
+    const PlanHost& P = pl->h;
+    // tile-major rows (whole tiles): the workspace planes are tile-major in both layouts
+    const int64_t rows = int64_t(P.batch) * P.heads * P.tiles_per_head * P.tile_tokens;
+    if (rows == 0) return cudaSuccess;
     CUtensorMap mq, mk, mv, mdo;
-    cudaError_t e = make_rows_map(&mq, q, rows, D);
-    if (e == cudaSuccess) e = make_rows_map(&mk, k, rows, D);
-    if (e == cudaSuccess) e = make_rows_map(&mv, v, rows, D);
-    if (e == cudaSuccess) e = make_rows_map(&mdo, dout, rows, D);
+    cudaError_t e;
+    if (raster) {
+        const RasterBox rb = raster_box(P.g);
+        if (!rb.ok) return cudaErrorInvalidValue;
+        EncodeTiled fn;
+        if ((e = encode_fn(&fn)) != cudaSuccess) return e;
+        const int64_t bh = int64_t(P.batch) * P.heads;
+        e = make_raster_map(fn, &mq, q, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_raster_map(fn, &mk, k, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_raster_map(fn, &mv, v, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_raster_map(fn, &mdo, dout, P.g, bh, D, rb.box_t, rb.box_h);
+    } else {
+        e = make_rows_map(&mq, q, rows, D);
+        if (e == cudaSuccess) e = make_rows_map(&mk, k, rows, D);
+        if (e == cudaSuccess) e = make_rows_map(&mv, v, rows, D);
+        if (e == cudaSuccess) e = make_rows_map(&mdo, dout, rows, D);
+    }
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
@@ -812,50 +895,33 @@ cudaError_t launch_bwd_d(const sta_plan_s* pl, const void* q, const void* k, con
     bp.sub_per_tile = P.sub_per_tile;
     bp.tile_tokens = P.tile_tokens;
     bp.tokens = P.tiles_per_head * P.tile_tokens;
-    bp.neg_d = neg_d;
-    bp.neg_l = neg_l;
+    bp.neg_d = ws;
+    bp.neg_l = ws + rows;
     bp.scale = scale;
     bp.scale_log2 = scale * kLog2e;
     bp.status = pl->d_status;
     bp.timeout_ns = timeout_ns;
-
-    // dQ
-    bp.items = pl->d_bq_items;
-    bp.n_items = int32_t(P.bq_items.size());
-    bp.off = pl->d_off;
-    bp.ids = pl->d_ids;
-    bp.out_a = static_cast<__nv_bfloat16*>(dq);
-    bp.out_b = nullptr;
-    int grid = bp.n_items < sms ? bp.n_items : sms;
-    constexpr int kSmemDq = smem_launch(DqCfg<D>::kSmemBytes);
-    e = cudaFuncSetAttribute(sta_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
-    if (e != cudaSuccess) return e;
-    sta_bwd_dq_kernel<D><<<grid, kBwThreads, kSmemDq, stream>>>(mq, mk, mv, mdo, bp);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    // dK, dV
-    bp.items = pl->d_bkv_items;
-    bp.n_items = int32_t(P.bkv_items.size());
-    bp.off = pl->d_toff;
-    bp.ids = pl->d_tids;
-    bp.out_a = static_cast<__nv_bfloat16*>(dk);
-    bp.out_b = static_cast<__nv_bfloat16*>(dv);
-    grid = bp.n_items < sms ? bp.n_items : sms;
-    constexpr int kSmemDkv = smem_launch(DkvCfg<D>::kSmemBytes);
-    e = cudaFuncSetAttribute(sta_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDkv);
-    if (e != cudaSuccess) return e;
-    sta_bwd_dkdv_kernel<D><<<grid, kBwThreads, kSmemDkv, stream>>>(mq, mk, mv, mdo, bp);
-    return cudaGetLastError();
+    bp.rg = raster_geom(pl);
+    if (raster)
+        return P.padded ? launch_bwd_variant<D, true, true>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, rows,
+                                                            sms, stream)
+                        : launch_bwd_variant<D, true, false>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv,
+                                                             rows, sms, stream);
+    return launch_bwd_variant<D, false, false>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, rows, sms,
+                                               stream);
 }
 
 }  // namespace
 
 cudaError_t launch_backward(const sta_plan_s* p, const void* q, const void* k, const void* v, const void* o,
                             const void* dout, const float* lse, void* dq, void* dk, void* dv, float* workspace,
-                            int head_dim, float softmax_scale, cudaStream_t stream, uint64_t timeout_ns) {
+                            int head_dim, float softmax_scale, cudaStream_t stream, uint64_t timeout_ns,
+                            bool raster) {
     if (head_dim == 128)
-        return launch_bwd_d<128>(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, softmax_scale, stream, timeout_ns);
-    return launch_bwd_d<64>(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, softmax_scale, stream, timeout_ns);
+        return launch_bwd_d<128>(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, softmax_scale, stream, timeout_ns,
+                                 raster);
+    return launch_bwd_d<64>(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, softmax_scale, stream, timeout_ns,
+                            raster);
 }
 
 }  // namespace sta

@@ -40,6 +40,7 @@
 
 #include "sta_internal.h"
 #include "sta_ptx.cuh"
+#include "sta_raster.cuh"
 #include "sta_wait.cuh"
 
 namespace sta {
@@ -93,7 +94,6 @@ struct FwdParams {
     int32_t sub_per_tile;  // 128-row blocks (= 128-key chunks) per tile
     int32_t tile_tokens;
     int32_t tokens;  // tile-major rows per (b, h): whole tiles
-    int32_t tokens_raster;  // raster rows per (b, h): the latent's tokens
     __nv_bfloat16* o;
     float* lse;
     float scale_log2;  // softmax_scale * log2(e)
@@ -101,17 +101,10 @@ struct FwdParams {
     uint32_t* status;
     uint64_t timeout_ns;
     int32_t inject;
-    // Raster layout only: latent and tile extents, tiles along h and w, and the
-    // shape of one 128-row block as a box of whole (t, h) slices.
-    int32_t lat_h, lat_w;
-    int32_t tile_t, tile_h, tile_w;
-    int32_t n_h, n_w;
-    int32_t box_t, box_h, blocks_per_slice;
-    const int4* tile_origin;  // [tiles]: raster (w, h, t) origin of each tile
+    RasterGeom rg;  // raster layout only
     // Padded latents (an axis not a multiple of the tile): real-key bits of
     // every 128-key chunk, [tiles][sub_per_tile] x 4 words; null otherwise.
     const uint4* key_mask;
-    int32_t lat_t;
 };
 
 // Load 128-row block `sub` of tile `tile` of head bh.  Tile-major layout: one
@@ -125,16 +118,7 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* m, u
         const int32_t row = bh * p.tokens + tile * p.tile_tokens + sub * kSubRows;
         for (int cb = 0; cb < col_blocks; ++cb) ptx::tma_load_2d(dst + cb * box_bytes, m, bar, cb * 64, row);
     } else {
-        const int4 org = p.tile_origin[tile];
-        int32_t t0 = org.z, h0 = org.y;
-        if (p.blocks_per_slice == 1) {
-            t0 += sub * p.box_t;
-        } else {
-            t0 += sub / p.blocks_per_slice;
-            h0 += (sub % p.blocks_per_slice) * p.box_h;
-        }
-        for (int cb = 0; cb < col_blocks; ++cb)
-            ptx::tma_load_5d(dst + cb * box_bytes, m, bar, cb * 64, org.x, h0, t0, bh);
+        raster_load(dst, m, bar, p.rg, bh, tile, sub, col_blocks, box_bytes);
     }
 }
 
@@ -143,14 +127,7 @@ __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* m, u
 template <bool kRaster, bool kPadded>
 __device__ __forceinline__ int64_t out_row(const FwdParams& p, int32_t bh, int32_t blk, int32_t r) {
     if (!kRaster) return int64_t(bh) * p.tokens + int64_t(blk) * kSubRows + r;
-    const int32_t tile = blk / p.sub_per_tile, sub = blk - tile * p.sub_per_tile;
-    const int32_t it = tile / (p.n_h * p.n_w), ih = (tile / p.n_w) % p.n_h, iw = tile % p.n_w;
-    const int32_t l = sub * kSubRows + r;  // tile-local row, raster over the tile's (t, h, w)
-    const int32_t lw = l % p.tile_w, lh = (l / p.tile_w) % p.tile_h, lt = l / (p.tile_w * p.tile_h);
-    const int32_t t = it * p.tile_t + lt, h = ih * p.tile_h + lh, w = iw * p.tile_w + lw;
-    if (kPadded && (t >= p.lat_t || h >= p.lat_h || w >= p.lat_w)) return -1;
-    const int64_t token = (int64_t(t) * p.lat_h + h) * p.lat_w + w;
-    return int64_t(bh) * p.tokens_raster + token;
+    return raster_row<kPadded>(p.rg, bh, blk, r);
 }
 
 // Bounded wait with this launch's status word and time limit.
@@ -628,25 +605,6 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) {
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// 5D map over a raster [BH, L_t, L_h, L_w, d] bf16 tensor whose box is one
-// 128-row block of a tile: 64 elements x tile_w x box_h x box_t x 1, with the
-// same 128-byte swizzle; TMA writes the box's rows in tile-major order.
-cudaError_t make_map_raster(CUtensorMap* m, const void* ptr, const sta_geom& g, int64_t bh, int d,
-                            int box_t, int box_h) {
-    const EncodeFn& e = encode_fn();
-    if (e.err != cudaSuccess) return e.err;
-    const cuuint64_t row = cuuint64_t(d) * 2;
-    cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(g.lat_w), cuuint64_t(g.lat_h), cuuint64_t(g.lat_t),
-                          cuuint64_t(bh)};
-    cuuint64_t strides[4] = {row, row * g.lat_w, row * g.lat_w * g.lat_h, row * g.lat_w * g.lat_h * g.lat_t};
-    cuuint32_t box[5] = {64, cuuint32_t(g.tile_w), cuuint32_t(box_h), cuuint32_t(box_t), 1};
-    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = e.fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box,
-                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 template <int D, bool kRaster, bool kPadded>
 cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
                           const CUtensorMap& mv, const FwdParams& fp) {
@@ -669,9 +627,11 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     CUtensorMap mq, mk, mv;
     cudaError_t e;
     if (raster) {
-        e = make_map_raster(&mq, q, P.g, bh, D, rb.box_t, rb.box_h);
-        if (e == cudaSuccess) e = make_map_raster(&mk, k, P.g, bh, D, rb.box_t, rb.box_h);
-        if (e == cudaSuccess) e = make_map_raster(&mv, v, P.g, bh, D, rb.box_t, rb.box_h);
+        const EncodeFn& ef = encode_fn();
+        if (ef.err != cudaSuccess) return ef.err;
+        e = make_raster_map(ef.fn, &mq, q, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_raster_map(ef.fn, &mk, k, P.g, bh, D, rb.box_t, rb.box_h);
+        if (e == cudaSuccess) e = make_raster_map(ef.fn, &mv, v, P.g, bh, D, rb.box_t, rb.box_h);
     } else {
         e = make_map(&mq, q, rows, D);
         if (e == cudaSuccess) e = make_map(&mk, k, rows, D);
@@ -687,7 +647,6 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.sub_per_tile = P.sub_per_tile;
     fp.tile_tokens = P.tile_tokens;
     fp.tokens = P.tiles_per_head * P.tile_tokens;
-    fp.tokens_raster = P.g.lat_t * P.g.lat_h * P.g.lat_w;
     fp.o = static_cast<__nv_bfloat16*>(o);
     fp.lse = lse;
     fp.scale = scale;
@@ -695,19 +654,8 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.status = pl->d_status;
     fp.timeout_ns = timeout_ns;
     fp.inject = inject;
-    fp.lat_h = P.g.lat_h;
-    fp.lat_w = P.g.lat_w;
-    fp.tile_t = P.g.tile_t;
-    fp.tile_h = P.g.tile_h;
-    fp.tile_w = P.g.tile_w;
-    fp.n_h = P.n_tiles[1];
-    fp.n_w = P.n_tiles[2];
-    fp.box_t = rb.box_t;
-    fp.box_h = rb.box_h;
-    fp.blocks_per_slice = rb.blocks_per_slice;
-    fp.tile_origin = reinterpret_cast<const int4*>(pl->d_origin);
+    fp.rg = raster_geom(pl);
     fp.key_mask = reinterpret_cast<const uint4*>(pl->d_kmask);
-    fp.lat_t = P.g.lat_t;
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

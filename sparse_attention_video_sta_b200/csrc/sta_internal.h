@@ -108,11 +108,12 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
                                cudaStream_t stream);
 
 // Backward launches (sta_backward.cu): the D / log2-LSE pass, then the dQ and
-// dK / dV kernels, on tile-major tensors.  Returns a CUDA error code.
+// dK / dV kernels, on tile-major tensors or (`raster`) on raster tensors with
+// the permutation fused.  Returns a CUDA error code.
 cudaError_t launch_backward(const sta_plan_s* p, const void* q, const void* k, const void* v,
                             const void* o, const void* dout, const float* lse, void* dq, void* dk,
                             void* dv, float* workspace, int head_dim, float softmax_scale,
-                            cudaStream_t stream, uint64_t timeout_ns);
+                            cudaStream_t stream, uint64_t timeout_ns, bool raster);
 
 // Per-slice recall / loss reduction for the window search (sta_search.cu).
 cudaError_t launch_window_stats(const float* lse_w, const float* lse_full, const void* o_w, const void* o_full,

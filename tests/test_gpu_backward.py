@@ -179,6 +179,26 @@ def test_backward_deterministic_and_tile_major_entry(sta):
     assert sta.sta_last_device_status(plan) == 0
 
 
+@pytest.mark.parametrize("latent,tile,d", [((30, 48, 80), (6, 8, 8), 128), ((12, 16, 16), (4, 8, 8), 128),
+                                            ((18, 24, 24), (6, 8, 8), 64), ((8, 16, 16), (2, 8, 8), 128)])
+def test_fused_raster_backward_equals_chain(sta, latent, tile, d):
+    """sta_backward_raster gives the same bits as reorder -> sta_backward ->
+    unreorder, on the 720p workload shape (2 heads) and smaller geometries."""
+    B, H = 1, 2
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator(device="cuda").manual_seed(N + d)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(4))
+    windows = [[3 * t for t in tile], list(tile)]
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = sta.sta_attention(q, k, v, plan, scale)
+    fused = sta.sta_attention_backward(q, k, v, o, lse, do, plan, scale)
+    chain = sta.sta_attention_backward(q, k, v, o, lse, do, plan, scale, fused=False)
+    for a, b in zip(fused, chain):
+        assert torch.equal(a, b)
+    assert sta.sta_last_device_status(plan) == 0
+
+
 def test_autograd_function(sta):
     """StaAttention.apply inside autograd gives the same gradients as the
     explicit backward call."""
@@ -195,3 +215,35 @@ def test_autograd_function(sta):
     ref = sta.sta_attention_backward(q, k, v, o2, lse, do, plan, 0.125)
     for got, r in zip((qa.grad, ka.grad, va.grad), ref):
         assert torch.equal(got, r)
+
+
+def test_calls_from_a_fresh_thread(sta):
+    """Forward and backward from a thread that has made no CUDA call before
+    (as autograd's worker threads and thread pools are)."""
+    import threading
+    latent, tile, B, H, d = (12, 16, 16), (6, 8, 8), 1, 2, 64
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator().manual_seed(79)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(4))
+    plan = sta.sta_plan(latent, tile, B, H, [[6, 8, 8]] * H)
+    o_ref, l_ref = sta.sta_attention(q, k, v, plan, 0.125)
+    ref = sta.sta_attention_backward(q, k, v, o_ref, l_ref, do, plan, 0.125)
+    torch.cuda.synchronize()
+    box = {}
+
+    def work():
+        try:
+            o, l = sta.sta_attention(q, k, v, plan, 0.125)
+            box["fwd"] = (o, l)
+            box["bwd"] = sta.sta_attention_backward(q, k, v, o, l, do, plan, 0.125)
+            torch.cuda.synchronize()
+        except Exception as e:  # reported below
+            box["err"] = e
+
+    t = threading.Thread(target=work)
+    t.start()
+    t.join()
+    assert "err" not in box, box.get("err")
+    assert torch.equal(box["fwd"][0], o_ref) and torch.equal(box["fwd"][1], l_ref)
+    for a, b in zip(box["bwd"], ref):
+        assert torch.equal(a, b)

@@ -75,6 +75,9 @@ def test_padded_forward_and_backward_all_rows(sta, latent, tile, B, H, d, window
     compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
             what=f"padded {latent}")
     dq, dk, dv = sta.sta_attention_backward(qd, kd, vd, o, lse, dod, plan, scale)
+    chain = sta.sta_attention_backward(qd, kd, vd, o, lse, dod, plan, scale, fused=False)
+    for a, b in zip((dq, dk, dv), chain):
+        assert torch.equal(a, b)  # fused raster kernels == reorder, tile-major backward, unreorder
     assert sta.sta_last_device_status(plan) == 0
     rq, rk, rv = oracle.sta_backward(q, k, v, do, latent, tile, windows, scale)
     N = q.shape[2]
