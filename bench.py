@@ -42,7 +42,9 @@ UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FWD_SOURCES = ["sparse_attention_video_sta_b200/csrc/sta_forward.cu",
                "sparse_attention_video_sta_b200/csrc/sta_ptx.cuh",
-               "sparse_attention_video_sta_b200/csrc/sta_internal.h"]
+               "sparse_attention_video_sta_b200/csrc/sta_internal.h",
+               "sparse_attention_video_sta_b200/csrc/sta_raster.cuh",
+               "sparse_attention_video_sta_b200/csrc/sta_wait.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sta_fwd_720p_traffic.json")
 
 

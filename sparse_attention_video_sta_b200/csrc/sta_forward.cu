@@ -58,7 +58,10 @@ constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsProducer = 88;
 static_assert(128 * (2 * kRegsSoftmax + kRegsProducer) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+// Lazy rescale: a chunk is exponentiated against the running max; only a row
+// whose chunk sum exceeds this (its max grew by more than 2^8, or many scores
+// grew a little) is redone against its own max, with O and l rescaled.
+constexpr float kRescaleRowSum = 256.0f;
 
 constexpr int kStagesD128 = 5;  // K/V ring stages of 32 KB at d = 128 (8 of 16 KB at d = 64)
 
@@ -111,15 +114,23 @@ struct FwdParams {
 // 2D row coordinate.  Raster layout: the (w, h, t) origin of the block's box
 // inside the tile (tile origin from the plan's table), whose rows TMA lays out
 // in tile-major order.
+// `org`: the tile's raster origin (raster layout only; read ahead by the caller).
 template <bool kRaster>
 __device__ __forceinline__ void load_block(uint32_t dst, const CUtensorMap* m, uint32_t bar, const FwdParams& p,
-                                           int32_t bh, int32_t tile, int32_t sub, int col_blocks, int box_bytes) {
+                                           int32_t bh, int32_t tile, int4 org, int32_t sub, int col_blocks,
+                                           int box_bytes) {
     if (!kRaster) {
         const int32_t row = bh * p.tokens + tile * p.tile_tokens + sub * kSubRows;
         for (int cb = 0; cb < col_blocks; ++cb) ptx::tma_load_2d(dst + cb * box_bytes, m, bar, cb * 64, row);
     } else {
-        raster_load(dst, m, bar, p.rg, bh, tile, sub, col_blocks, box_bytes);
+        raster_load_at(dst, m, bar, p.rg, bh, org, sub, col_blocks, box_bytes);
     }
+}
+
+// Raster origin of a tile (zeros for the tile-major layout, which has none).
+template <bool kRaster>
+__device__ __forceinline__ int4 tile_org(const FwdParams& p, int32_t tile) {
+    return kRaster ? __ldg(p.rg.tile_origin + tile) : make_int4(0, 0, 0, 0);
 }
 
 // Row of the output tensors that holds row `r` of block `blk` of head bh; -1
@@ -146,23 +157,14 @@ __device__ __forceinline__ void mask_scores(uint32_t (&sr)[128], const uint4 m) 
 }
 
 // P = exp2(S * c - m * c) for one 128-score row, packed to bf16 pairs; returns
-// the fp32 row sum.  With kTrack it also returns the row max of S in `mx`.
-template <bool kTrack>
-__device__ __forceinline__ float softmax_exp(const uint32_t (&sr)[128], float c, float m,
-                                             uint32_t (&pk)[64], float& mx) {
+// the fp32 row sum.
+__device__ __forceinline__ float softmax_exp(const uint32_t (&sr)[128], float c, float m, uint32_t (&pk)[64]) {
     const uint64_t c2 = ptx::f2(c, c);
     const uint64_t nmc2 = ptx::f2(-m * c, -m * c);
     uint64_t acc0 = ptx::f2(0.0f, 0.0f), acc1 = acc0;
-    float a0 = __int_as_float(0xff800000), a1 = a0;
 #pragma unroll
     for (int j = 0; j < 64; ++j) {
         const float s0 = __uint_as_float(sr[2 * j]), s1 = __uint_as_float(sr[2 * j + 1]);
-        if (kTrack) {
-            if (j & 1)
-                a1 = ptx::max3(a1, s0, s1);
-            else
-                a0 = ptx::max3(a0, s0, s1);
-        }
         float x0, x1, p0, p1;
         ptx::f2_split(ptx::f2_fma(ptx::f2(s0, s1), c2, nmc2), x0, x1);
         p0 = ptx::ex2(x0);
@@ -173,7 +175,6 @@ __device__ __forceinline__ float softmax_exp(const uint32_t (&sr)[128], float c,
             acc0 = ptx::f2_add(acc0, ptx::f2(p0, p1));
         pk[j] = ptx::pack_bf16x2(p0, p1);
     }
-    if (kTrack) mx = fmaxf(a0, a1);
     float r0, r1, r2, r3;
     ptx::f2_split(acc0, r0, r1);
     ptx::f2_split(acc1, r2, r3);
@@ -279,7 +280,8 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // Debug: wait on a barrier nothing arrives at; the limit runs out.
                 ok = wait_bar(bar_dead, 0, abort_flag, p);
             }
-            auto issue = [&](const CUtensorMap* m, int32_t bh, int32_t tile, int32_t sub, uint32_t mask) -> bool {
+            auto issue = [&](const CUtensorMap* m, int32_t bh, int32_t tile, int4 org, int32_t sub,
+                             uint32_t mask) -> bool {
                 const int r = int(item % S);
                 const uint32_t prev = (users >> (2 * r)) & 3u;
 #pragma unroll
@@ -290,7 +292,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 users = (users & ~(3u << (2 * r))) | (mask << (2 * r));
                 upar ^= mask << (2 * r);
                 ptx::mbar_arrive_expect_tx(bar_full(r), C::kKVBytes);
-                load_block<kRaster>(base + C::kRingOff + r * C::kKVBytes, m, bar_full(r), p, bh, tile, sub,
+                load_block<kRaster>(base + C::kRingOff + r * C::kKVBytes, m, bar_full(r), p, bh, tile, org, sub,
                                     C::kColBlocks, C::kBoxBytes);
                 ++item;
                 return true;
@@ -307,35 +309,41 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 // query blocks, one buffer per slot
                 if (!wait_bar(bar_q_empty(0), (qc0 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
                 ptx::mbar_arrive_expect_tx(bar_q_full(0), C::kQBytes);
-                load_block<kRaster>(base + C::kQOff, &tm_q, bar_q_full(0), p, w.bh, tile_a, w.qa - tile_a * SPT,
-                                    C::kColBlocks, C::kBoxBytes);
+                load_block<kRaster>(base + C::kQOff, &tm_q, bar_q_full(0), p, w.bh, tile_a, tile_org<kRaster>(p, tile_a),
+                                    w.qa - tile_a * SPT, C::kColBlocks, C::kBoxBytes);
                 ++qc0;
                 if (has_b) {
                     if (!wait_bar(bar_q_empty(1), (qc1 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(bar_q_full(1), C::kQBytes);
                     load_block<kRaster>(base + C::kQOff + C::kQBytes, &tm_q, bar_q_full(1), p, w.bh, tile_b,
-                                        w.qb - tile_b * SPT, C::kColBlocks, C::kBoxBytes);
+                                        tile_org<kRaster>(p, tile_b), w.qb - tile_b * SPT, C::kColBlocks,
+                                        C::kBoxBytes);
                     ++qc1;
                 }
                 // K / V chunks in the order the issuers consume them: chunk kc of
                 // key tile kt is one 128-row block.  The key-tile ids of the next
-                // tile are read one tile ahead so no TMA issue waits on them.
+                // tile, and in raster layout their origins, are read one tile
+                // ahead so no TMA issue waits on a load.
                 const uint32_t both = has_b ? 3u : 1u;
                 const int32_t n_kt = n_chunks / SPT;
                 int32_t ta = __ldg(list_a), tb = __ldg(list_b);
+                int4 oa = tile_org<kRaster>(p, ta), ob = tile_org<kRaster>(p, tb);
                 for (int32_t kt = 0; ok && kt < n_kt; ++kt) {
-                    const int32_t nta = kt + 1 < n_kt ? __ldg(list_a + kt + 1) : 0;
-                    const int32_t ntb = kt + 1 < n_kt ? __ldg(list_b + kt + 1) : 0;
+                    const int32_t nta = kt + 1 < n_kt ? __ldg(list_a + kt + 1) : ta;
+                    const int32_t ntb = kt + 1 < n_kt ? __ldg(list_b + kt + 1) : tb;
+                    const int4 noa = tile_org<kRaster>(p, nta), nob = tile_org<kRaster>(p, ntb);
                     for (int32_t kc = 0; ok && kc < SPT; ++kc) {
                         if (split) {
-                            ok = issue(&tm_k, w.bh, ta, kc, 1u) && issue(&tm_k, w.bh, tb, kc, 2u) &&
-                                 issue(&tm_v, w.bh, ta, kc, 1u) && issue(&tm_v, w.bh, tb, kc, 2u);
+                            ok = issue(&tm_k, w.bh, ta, oa, kc, 1u) && issue(&tm_k, w.bh, tb, ob, kc, 2u) &&
+                                 issue(&tm_v, w.bh, ta, oa, kc, 1u) && issue(&tm_v, w.bh, tb, ob, kc, 2u);
                         } else {
-                            ok = issue(&tm_k, w.bh, ta, kc, both) && issue(&tm_v, w.bh, ta, kc, both);
+                            ok = issue(&tm_k, w.bh, ta, oa, kc, both) && issue(&tm_v, w.bh, ta, oa, kc, both);
                         }
                     }
                     ta = nta;
                     tb = ntb;
+                    oa = noa;
+                    ob = nob;
                 }
             }
             // Drain: the copies issued last into each stage, and the last query loads.
@@ -466,7 +474,6 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 float rowsum;
                 bool rescale = false;
                 float alpha = 1.0f;
-                float mx;
                 uint32_t sr[128];
                 const uint4* kmask =
                     kPadded ? p.key_mask + int64_t(__ldg(p.ids + kbeg + i / SPT)) * SPT + i % SPT : nullptr;
@@ -481,23 +488,27 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (i == 0) {
                     // a tile's first chunk holds its first token, a real key: the max is finite
                     m_used = row_max(sr);
-                    rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
+                    rowsum = softmax_exp(sr, c, m_used, pk);
                 } else {
-                    // Exponentiate against the running max while finding this
-                    // chunk's max; only a row whose max grew by more than 2^8 is
-                    // redone (rarely) against its new max (lazy rescale).
-                    rowsum = softmax_exp<true>(sr, c, m_used, pk, mx);
-                    const bool need = (mx - m_used) * c > kRescaleThreshold;
+                    // Exponentiate against the running max (no max pass: it
+                    // costs an instruction per score pair on the critical
+                    // path); a row whose chunk sum says the max grew is redone
+                    // (rarely) against the chunk's own max (lazy rescale).
+                    rowsum = softmax_exp(sr, c, m_used, pk);
+                    const bool need = !(rowsum <= kRescaleRowSum);  // also catches inf
                     rescale = __any_sync(0xffffffffu, need);
                     if (rescale) {
-                        if (need) {
-                            alpha = ptx::ex2((m_used - mx) * c);
-                            m_used = mx;
-                        }
                         // S is still in TMEM (P has not been written over it yet)
                         ptx::tmem_ld128(tS, sr);
                         if (kPadded && masked) mask_scores(sr, __ldg(kmask));
-                        rowsum = softmax_exp<false>(sr, c, m_used, pk, mx);
+                        if (need) {
+                            const float mx = row_max(sr);
+                            if ((mx - m_used) * c > 0.0f) {
+                                alpha = ptx::ex2((m_used - mx) * c);
+                                m_used = mx;
+                            }
+                        }
+                        rowsum = softmax_exp(sr, c, m_used, pk);
                     }
                 }
                 ptx::tmem_st64(tS, pk);

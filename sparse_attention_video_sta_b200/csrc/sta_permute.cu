@@ -45,10 +45,11 @@ __device__ __forceinline__ int64_t local_to_raster(const PermGeom& g, int32_t l)
 }
 
 // V = element type moved per thread; vpr = elements per token row.
-template <typename V, bool kTable>
+// kInverse = false: raster -> tile-major.
+template <typename V, bool kTable, bool kInverse>
 __global__ void __launch_bounds__(kPermThreads)
 permute_kernel(const V* __restrict__ src, V* __restrict__ dst, PermGeom g, int32_t vpr,
-               int32_t vpr_shift, int64_t blocks, bool inverse) {
+               int32_t vpr_shift, int64_t blocks) {
     extern __shared__ int32_t table[];
     if (kTable) {
         for (int32_t l = threadIdx.x; l < g.tile_tokens; l += blockDim.x)
@@ -71,9 +72,7 @@ permute_kernel(const V* __restrict__ src, V* __restrict__ dst, PermGeom g, int32
         const int32_t vh = min(g.tile_h, g.lat_h - ih * g.tile_h);
         const int32_t vw = min(g.tile_w, g.lat_w - iw * g.tile_w);
         const bool edge = vt < g.tile_t || vh < g.tile_h || vw < g.tile_w;
-#pragma unroll 4
-        for (int64_t e = threadIdx.x; e < per_tile; e += blockDim.x) {
-            int32_t l, c;
+        auto split = [&](int64_t e, int32_t& l, int32_t& c) {
             if (vpr_shift >= 0) {
                 l = int32_t(e >> vpr_shift);
                 c = int32_t(e & (vpr - 1));
@@ -81,19 +80,35 @@ permute_kernel(const V* __restrict__ src, V* __restrict__ dst, PermGeom g, int32
                 l = int32_t(e / vpr);
                 c = int32_t(e - int64_t(l) * vpr);
             }
-            const int64_t tmaj = t_slice + tm_base + l;
-            if (edge) {
+        };
+        if (!edge) {  // a whole tile: no per-row test
+#pragma unroll 4
+            for (int64_t e = threadIdx.x; e < per_tile; e += blockDim.x) {
+                int32_t l, c;
+                split(e, l, c);
+                const int64_t tmaj = t_slice + tm_base + l;
+                const int64_t raster = r_slice + origin + (kTable ? int64_t(table[l]) : local_to_raster(g, l));
+                if (kInverse)
+                    dst[raster * vpr + c] = src[tmaj * vpr + c];
+                else
+                    dst[tmaj * vpr + c] = src[raster * vpr + c];
+            }
+        } else {  // a tile at the padded edge
+            for (int64_t e = threadIdx.x; e < per_tile; e += blockDim.x) {
+                int32_t l, c;
+                split(e, l, c);
+                const int64_t tmaj = t_slice + tm_base + l;
                 const int32_t x = l % g.tile_w, y = (l / g.tile_w) % g.tile_h, t = l / (g.tile_w * g.tile_h);
-                if (t >= vt || y >= vh || x >= vw) {  // padding row
-                    if (!inverse) dst[tmaj * vpr + c] = V{};
+                if (t >= vt || y >= vh || x >= vw) {  // padding row: zero in tile-major, absent in raster
+                    if (!kInverse) dst[tmaj * vpr + c] = V{};
                     continue;
                 }
+                const int64_t raster = r_slice + origin + (kTable ? int64_t(table[l]) : local_to_raster(g, l));
+                if (kInverse)
+                    dst[raster * vpr + c] = src[tmaj * vpr + c];
+                else
+                    dst[tmaj * vpr + c] = src[raster * vpr + c];
             }
-            const int64_t raster = r_slice + origin + (kTable ? int64_t(table[l]) : local_to_raster(g, l));
-            if (inverse)
-                dst[raster * vpr + c] = src[tmaj * vpr + c];
-            else
-                dst[tmaj * vpr + c] = src[raster * vpr + c];
         }
     }
 }
@@ -115,17 +130,17 @@ cudaError_t launch_typed(const void* src, void* dst, int64_t outer, int32_t row_
     const unsigned grid = unsigned(blocks < cap ? blocks : cap);
     if (g.tile_tokens <= kMaxTableTokens) {
         const size_t smem = size_t(g.tile_tokens) * sizeof(int32_t);
+        auto kern = inverse ? permute_kernel<V, true, true> : permute_kernel<V, true, false>;
         if (smem > 48 * 1024) {
-            cudaError_t e = cudaFuncSetAttribute(permute_kernel<V, true>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(smem));
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
             if (e != cudaSuccess) return e;
         }
-        permute_kernel<V, true><<<grid, kPermThreads, smem, stream>>>(
-            static_cast<const V*>(src), static_cast<V*>(dst), g, vpr, shift, blocks, inverse);
+        kern<<<grid, kPermThreads, smem, stream>>>(static_cast<const V*>(src), static_cast<V*>(dst), g, vpr, shift,
+                                                   blocks);
     } else {
-        permute_kernel<V, false><<<grid, kPermThreads, 0, stream>>>(
-            static_cast<const V*>(src), static_cast<V*>(dst), g, vpr, shift, blocks, inverse);
+        auto kern = inverse ? permute_kernel<V, false, true> : permute_kernel<V, false, false>;
+        kern<<<grid, kPermThreads, 0, stream>>>(static_cast<const V*>(src), static_cast<V*>(dst), g, vpr, shift,
+                                                blocks);
     }
     return cudaGetLastError();
 }

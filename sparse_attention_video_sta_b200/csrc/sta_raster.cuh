@@ -69,12 +69,13 @@ inline cudaError_t make_raster_map(PFN_cuTensorMapEncodeTiled_v12000 fn, CUtenso
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Load 128-row block `sub` of tile `tile` of head bh from a raster tensor:
-// the (w, h, t) origin of the block's box inside the tile (tile origin from
-// the plan's table), `col_blocks` boxes of 64 columns, `box_bytes` apart.
-__device__ __forceinline__ void raster_load(uint32_t dst, const CUtensorMap* m, uint32_t bar, const RasterGeom& g,
-                                            int32_t bh, int32_t tile, int32_t sub, int col_blocks, int box_bytes) {
-    const int4 org = g.tile_origin[tile];
+// Load 128-row block `sub` of the tile whose raster (w, h, t) origin is `org`
+// (from the plan's table) of head bh from a raster tensor: the origin of the
+// block's box inside the tile, `col_blocks` boxes of 64 columns, `box_bytes`
+// apart.
+__device__ __forceinline__ void raster_load_at(uint32_t dst, const CUtensorMap* m, uint32_t bar,
+                                               const RasterGeom& g, int32_t bh, int4 org, int32_t sub,
+                                               int col_blocks, int box_bytes) {
     int32_t t0 = org.z, h0 = org.y;
     if (g.blocks_per_slice == 1) {
         t0 += sub * g.box_t;
@@ -83,6 +84,12 @@ __device__ __forceinline__ void raster_load(uint32_t dst, const CUtensorMap* m, 
         h0 += (sub % g.blocks_per_slice) * g.box_h;
     }
     for (int cb = 0; cb < col_blocks; ++cb) ptx::tma_load_5d(dst + cb * box_bytes, m, bar, cb * 64, org.x, h0, t0, bh);
+}
+
+// The same for block `sub` of tile `tile` (origin looked up here).
+__device__ __forceinline__ void raster_load(uint32_t dst, const CUtensorMap* m, uint32_t bar, const RasterGeom& g,
+                                            int32_t bh, int32_t tile, int32_t sub, int col_blocks, int box_bytes) {
+    raster_load_at(dst, m, bar, g, bh, __ldg(g.tile_origin + tile), sub, col_blocks, box_bytes);
 }
 
 // Raster row of row `r` of 128-row block `blk` of head bh; -1 for a padding
