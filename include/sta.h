@@ -14,7 +14,10 @@
  * chosen per head (transcript, segment on head specialisation).
  *
  * Readings fixed by this library where the pages are silent:
- *   - window extent in tiles e_d = min(W_d / T_d, n_d), n_d = L_d / T_d;
+ *   - window extent in tiles e_d = min(W_d / T_d, n_d), n_d = ceil(L_d / T_d);
+ *   - a latent axis that is not a multiple of the tile is padded at its high
+ *     end to whole tiles; padding tokens are neither keys nor queries (the
+ *     pages describe divisible latents only);
  *   - window start s_d = clamp(q_d - floor(e_d / 2), 0, n_d - e_d): the window
  *     is shifted to stay inside the volume (this is the reading that gives the
  *     91% sparsity the atlas.scime.ai summary reports for w = (18,24,24));
@@ -23,9 +26,12 @@
  *   - LSE = m + ln(sum exp(s - m)) in natural-log, scaled-score units.
  *
  * Conventions for every call:
- *   - All tensors are row-major [B, heads, N, d] with N = L_t * L_h * L_w,
- *     owned by the caller, device-resident, contiguous.  q/k/v/o must be
- *     16-byte aligned.
+ *   - All tensors are row-major [B, heads, N, d], owned by the caller,
+ *     device-resident, contiguous, 16-byte aligned (fp32 LSE rows: 4-byte).
+ *     Raster-order tensors hold the latent's N = L_t * L_h * L_w tokens;
+ *     tile-major tensors hold whole tiles, N_tiles = n_t n_h n_w * tile volume
+ *     rows (equal to N when every axis is a multiple of the tile), with zero
+ *     padding rows as sta_tile_reorder writes them.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device work
  *     is enqueued asynchronously on it; nothing here synchronises except
  *     sta_plan, sta_plan_destroy and sta_last_device_status.
@@ -68,7 +74,8 @@ typedef struct {
 typedef struct sta_plan_s* sta_plan_t;
 
 /* Build a plan and upload it to the current CUDA device.
- *   g          : geometry; every L_d must be a positive multiple of T_d.
+ *   g          : geometry; L_d >= 1 and T_d >= 1 (an axis that is not a
+ *                multiple of its tile is padded to whole tiles).
  *   batch      : B >= 1;  heads: H >= 1
  *   window_thw : host array [heads][3], window per head in tokens; every entry
  *                a positive multiple of the tile extent on its axis (windows
@@ -76,10 +83,13 @@ typedef struct sta_plan_s* sta_plan_t;
  *   stream     : stream for the upload (the call waits for it to finish)
  *   out        : receives the plan handle
  * The plan holds, per distinct window, the ascending list of key-tile ids of
- * every query tile (CSR), and a work list of (b, h, query row block) items in
- * descending order of list length.  Allocates device memory; free it with
+ * every query tile (CSR) and its transpose, the forward work list of
+ * (b, h, query row block) items in descending order of list length, the
+ * backward's one-block work lists (ordered for a persistent grid of one CTA
+ * per SM), the raster origin of every tile, and for padded latents the real-key
+ * mask of every 128-key chunk.  Allocates device memory; free it with
  * sta_plan_destroy.  Errors: INVALID_ARG, UNSUPPORTED (tile volume not a
- * multiple of 128 tokens), OOM, CUDA. */
+ * multiple of 128 tokens, or more than 2^31 - 1 tile-major rows), OOM, CUDA. */
 STA_API sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
                     const int32_t* window_thw, void* stream, sta_plan_t* out);
 
@@ -117,7 +127,9 @@ STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, in
 STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
 
 /* Raster -> tile-major token permutation.
- *   src, dst  : device, [outer, N, row_bytes] bytes, distinct buffers
+ *   src       : device, [outer, N, row_bytes] bytes (raster)
+ *   dst       : device, [outer, N_tiles, row_bytes] bytes (tile-major; padding
+ *               rows written as zeros), not overlapping src
  *   outer     : B * heads (any count >= 1)
  *   row_bytes : bytes of one token row (d * element size; 4 for a fp32 LSE
  *               row); rows move intact, bit-exact
@@ -125,14 +137,16 @@ STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t ca
 STA_API sta_status sta_tile_reorder(const void* src, void* dst, int64_t outer,
                             int32_t row_bytes, const sta_geom* g, void* stream);
 
-/* Inverse permutation: dst[o, i] = src[o, tile_major(i)]. */
+/* Inverse permutation: dst[o, i] = src[o, tile_major(i)]; src is tile-major
+ * [outer, N_tiles, row_bytes] (its padding rows are not read), dst raster
+ * [outer, N, row_bytes]. */
 STA_API sta_status sta_tile_unreorder(const void* src, void* dst, int64_t outer,
                               int32_t row_bytes, const sta_geom* g, void* stream);
 
 /* STA forward on tile-major tensors.
- *   q, k, v : device bf16 [B, heads, N, d], tile-major token order
- *   o       : device bf16 [B, heads, N, d], tile-major (written)
- *   lse     : device fp32 [B, heads, N], tile-major (written): natural-log
+ *   q, k, v : device bf16 [B, heads, N_tiles, d], tile-major token order
+ *   o       : device bf16 [B, heads, N_tiles, d], tile-major (written)
+ *   lse     : device fp32 [B, heads, N_tiles], tile-major (written): natural-log
  *             log-sum-exp of the scaled scores of each query row
  *   head_dim: d, 64 or 128 (else UNSUPPORTED)
  *   softmax_scale: multiplies q . k before the softmax (e.g. 1/sqrt(d));
@@ -170,11 +184,11 @@ STA_API sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k
  *   D_i = dout_i . o_i,  dS_ij = P_ij (dout_i . v_j - D_i),
  *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
  *   dv_j = sum_i P_ij dout_i.
- *   q, k, v, o : device bf16 [B, heads, N, d], tile-major; o and lse as
+ *   q, k, v, o : device bf16 [B, heads, N_tiles, d], tile-major; o and lse as
  *                written by sta_forward for the same q, k, v and plan
- *   dout       : device bf16 [B, heads, N, d], tile-major: gradient w.r.t. o
- *   lse        : device fp32 [B, heads, N], tile-major
- *   dq, dk, dv : device bf16 [B, heads, N, d], tile-major (written; distinct
+ *   dout       : device bf16 [B, heads, N_tiles, d], tile-major: gradient w.r.t. o
+ *   lse        : device fp32 [B, heads, N_tiles], tile-major
+ *   dq, dk, dv : device bf16 [B, heads, N_tiles, d], tile-major (written; distinct
  *                from every input)
  *   workspace  : device fp32, 2 * B * heads * N floats, 16-byte aligned,
  *                caller-owned; on return plane 0 holds -D_i and plane 1
