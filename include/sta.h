@@ -126,6 +126,14 @@ STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, in
  * min(count, cap) items and the full count to *count.  For tests/inspection. */
 STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
 
+/* Copy one of the backward's work lists to host memory, four int32 per item:
+ * (b * heads + h, 128-row block, -1, window id); which = 0: the dQ kernel's
+ * query blocks, 1: the dK / dV kernel's key blocks.  Each lists every block
+ * of every (b, h) once, ordered for a persistent grid of one CTA per SM.
+ * Writes min(count, cap) items and the full count.  For tests/inspection. */
+STA_API sta_status sta_plan_backward_items(sta_plan_t p, int32_t which, int32_t* items4, int64_t cap,
+                                           int64_t* count);
+
 /* Raster -> tile-major token permutation.
  *   src       : device, [outer, N, row_bytes] bytes (raster)
  *   dst       : device, [outer, N_tiles, row_bytes] bytes (tile-major; padding

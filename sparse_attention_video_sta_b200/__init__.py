@@ -52,6 +52,7 @@ EXPORTED_SYMBOLS = (
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
     "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy", "sta_backward_raster",
+    "sta_plan_backward_items",
 )
 
 
@@ -77,6 +78,7 @@ def _load() -> ctypes.CDLL:
         "sta_plan_key_query": [vp, i32, i32, i32p, i32, i32p],
         "sta_plan_stats": [vp, i64p, i64p],
         "sta_plan_work_items": [vp, i32p, i64, i64p],
+        "sta_plan_backward_items": [vp, i32, i32p, i64, i64p],
         "sta_tile_reorder": [vp, vp, i64, i32, G, vp],
         "sta_tile_unreorder": [vp, vp, i64, i32, G, vp],
         "sta_forward": [vp, vp, vp, vp, vp, vp, i32, ctypes.c_float, vp],
@@ -222,6 +224,18 @@ class Plan:
         buf = (ctypes.c_int32 * max(4 * count.value, 4))()
         _check(_lib.sta_plan_work_items(self.handle, buf, count.value, ctypes.byref(count)),
                "sta_plan_work_items")
+        flat = list(buf[:4 * count.value])
+        return [tuple(flat[4 * i:4 * i + 4]) for i in range(count.value)]
+
+    def backward_items(self, which: int):
+        """Backward work list (0: dQ query blocks, 1: dK / dV key blocks) as
+        (bh, block, -1, window id) tuples, in the order the CTAs take them."""
+        count = ctypes.c_int64(0)
+        _check(_lib.sta_plan_backward_items(self.handle, int(which), None, 0, ctypes.byref(count)),
+               "sta_plan_backward_items")
+        buf = (ctypes.c_int32 * max(4 * count.value, 4))()
+        _check(_lib.sta_plan_backward_items(self.handle, int(which), buf, count.value, ctypes.byref(count)),
+               "sta_plan_backward_items")
         flat = list(buf[:4 * count.value])
         return [tuple(flat[4 * i:4 * i + 4]) for i in range(count.value)]
 

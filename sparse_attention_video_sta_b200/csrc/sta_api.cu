@@ -507,6 +507,21 @@ sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64
     return STA_OK;
 }
 
+sta_status sta_plan_backward_items(sta_plan_t p, int32_t which, int32_t* items4, int64_t cap, int64_t* count) {
+    if (p == nullptr || count == nullptr || cap < 0 || (cap > 0 && items4 == nullptr) || which < 0 || which > 1)
+        return STA_ERR_INVALID_ARG;
+    const auto& it = which == 0 ? p->h.bq_items : p->h.bkv_items;
+    *count = int64_t(it.size());
+    const int64_t n = std::min<int64_t>(cap, int64_t(it.size()));
+    for (int64_t i = 0; i < n; ++i) {
+        items4[4 * i + 0] = it[i].bh;
+        items4[4 * i + 1] = it[i].qa;
+        items4[4 * i + 2] = it[i].qb;
+        items4[4 * i + 3] = it[i].win;
+    }
+    return STA_OK;
+}
+
 sta_status sta_tile_reorder(const void* src, void* dst, int64_t outer, int32_t row_bytes,
                             const sta_geom* g, void* stream) {
     return permute_common(src, dst, outer, row_bytes, g, stream, false);

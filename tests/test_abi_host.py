@@ -251,3 +251,40 @@ def test_pipe_rejected_before_allocation():
     assert lib.sta_pipe_wait(None) == INV
     assert lib.sta_pipe_destroy(None) == 0
     hp.destroy()
+
+
+@pytest.mark.parametrize("latent,tile,heads,batch,wins", [
+    ((30, 48, 80), (6, 8, 8), 24, 1, None),
+    ((18, 24, 24), (6, 8, 8), 3, 2, [(6, 8, 8), (12, 16, 16), (18, 24, 24)]),
+    ((13, 21, 18), (6, 8, 8), 2, 1, [(6, 8, 8), (18, 24, 24)]),
+])
+def test_backward_work_lists(latent, tile, heads, batch, wins):
+    """Each backward list holds every (b, h, block) once; rounds of 148 items
+    (one per CTA of the host plan's grid) keep natural (b, h, block) order
+    between rounds, and per-CTA totals of list lengths stay level."""
+    wins = wins or [(18, 24, 24)] * heads
+    p = sta.sta_plan_host(latent, tile, batch, heads, wins)
+    S = (tile[0] * tile[1] * tile[2]) // 128
+    n_blocks = p.tiles_per_head * S
+    for which in (0, 1):
+        items = p.backward_items(which)
+        assert all(qb == -1 for _, _, qb, _ in items)
+        keys = sorted((bh, blk) for bh, blk, _, _ in items)
+        assert keys == [(bh, blk) for bh in range(batch * heads) for blk in range(n_blocks)]
+        R = 148
+        natural = [(bh, blk) for bh in range(batch * heads) for blk in range(n_blocks)]
+        for r0 in range(0, len(items), R):
+            assert sorted((bh, blk) for bh, blk, _, _ in items[r0:r0 + R]) == natural[r0:r0 + R]
+        def length(it):
+            bh, blk, _, win = it
+            h = bh % heads
+            t = blk // S
+            return len(p.query(h, t)) if which == 0 else len(p.key_query(h, t))
+        # after every full round the CTAs' totals differ by at most one item
+        # (a final partial round can only go to the first CTAs of the grid)
+        loads = [0] * R
+        longest = max(length(it) for it in items)
+        for r0 in range(0, len(items) - R + 1, R):
+            for c, it in enumerate(items[r0:r0 + R]):
+                loads[c] += length(it)
+            assert max(loads) - min(loads) <= longest, (which, r0, max(loads), min(loads))
