@@ -278,6 +278,8 @@ void free_device(sta_plan_s* p) {
     if (p->d_origin) cudaFree(p->d_origin);
     if (p->d_kmask) cudaFree(p->d_kmask);
     p->d_kmask = nullptr;
+    if (p->d_counters) cudaFree(p->d_counters);
+    p->d_counters = nullptr;
     if (p->d_toff) cudaFree(p->d_toff);
     if (p->d_tids) cudaFree(p->d_tids);
     if (p->d_bq_items) cudaFree(p->d_bq_items);
@@ -426,6 +428,8 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
     if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
     if (e == cudaSuccess && p->h.padded) e = upload(&p->d_kmask, p->h.key_mask, s);
+    if (e == cudaSuccess)
+        e = cudaMalloc(reinterpret_cast<void**>(&p->d_counters), sta::kCounterPool * sizeof(int32_t));
     if (e == cudaSuccess) e = upload(&p->d_toff, p->h.tcsr_off, s);
     if (e == cudaSuccess) e = upload(&p->d_tids, p->h.tcsr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_bq_items, p->h.bq_items, s);
@@ -448,7 +452,8 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_kmask || p->d_toff ||
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_kmask ||
+        p->d_counters || p->d_toff ||
         p->d_tids || p->d_bq_items || p->d_bkv_items) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
         free_device(p);

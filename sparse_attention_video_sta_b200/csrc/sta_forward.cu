@@ -64,6 +64,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleRowSum = 256.0f;
 
 constexpr int kStagesD128 = 5;  // K/V ring stages of 32 KB at d = 128 (8 of 16 KB at d = 64)
+// Work items are handed out at run time: the load warp takes the next item
+// index from a global counter and passes it to the other roles through a
+// queue of this many entries in shared memory.  CTAs that run slower (their
+// SM's share of L2 and HBM, their items' tiles) then take fewer items.
+constexpr int kItemQ = 4;
+constexpr int kItemConsumers = 2 + 8;  // the two issuing threads and the eight softmax warps
 
 template <int D>
 struct Cfg {
@@ -76,10 +82,10 @@ struct Cfg {
     static constexpr int kRingOff = 2 * kQBytes;
     static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
     // barriers: full[S], empty[S][2], q_full[2], q_empty[2], s_full[2], p_full[2],
-    // o_full[2], o_empty[2], dead, drain[2], turn[2]
-    static constexpr int kNumBars = 3 * kStages + 17;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot + abort flag
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+    // o_full[2], o_empty[2], dead, drain[2], turn[2], item_full[Q], item_empty[Q]
+    static constexpr int kNumBars = 3 * kStages + 17 + 2 * kItemQ;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag, item queue
+    static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemQ + 1024;  // + alignment slack
     // TMEM columns: S0 | S1 | O0 | O1
     __host__ __device__ static constexpr uint32_t col_s(int slot) { return uint32_t(slot) * 128u; }
     __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256u + uint32_t(slot) * D; }
@@ -91,6 +97,7 @@ struct Cfg {
 struct FwdParams {
     const WorkItem* items;
     int32_t n_items;
+    int32_t* item_counter;  // next item to hand out (zeroed before the launch); null: static striding
     const int32_t* off;  // CSR offsets [n_win][tiles + 1]
     const int32_t* ids;  // CSR key-tile ids
     int32_t tiles_per_head;
@@ -224,8 +231,19 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t bar_dead = bar0 + 8u * (3 * S + 12);
     auto bar_drain = [&](int s) { return bar0 + 8u * (3 * S + 13 + s); };
     auto bar_turn = [&](int s) { return bar0 + 8u * (3 * S + 15 + s); };
+    auto bar_item_full = [&](int q) { return bar0 + 8u * (3 * S + 17 + q); };
+    auto bar_item_empty = [&](int q) { return bar0 + 8u * (3 * S + 17 + kItemQ + q); };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(smem + C::kMiscOff + 8);
+    // Consumer side of the item queue: entry k holds the k-th item of this CTA
+    // (-1: none left).  Returns false when the CTA is aborting.
+    auto take_item = [&](uint32_t k, int32_t& u) -> bool {
+        const int q = int(k % kItemQ);
+        if (!wait_bar(bar_item_full(q), (k / kItemQ) & 1u, abort_flag, p)) return false;
+        u = item_q[q];
+        return true;
+    };
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < S; ++r) {
@@ -245,6 +263,10 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ptx::mbar_init(bar_dead, 1);
         ptx::mbar_init(bar_turn(0), 1);
         ptx::mbar_init(bar_turn(1), 1);
+        for (int q = 0; q < kItemQ; ++q) {
+            ptx::mbar_init(bar_item_full(q), 1);
+            ptx::mbar_init(bar_item_empty(q), kItemConsumers);
+        }
         *abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
@@ -297,7 +319,20 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 ++item;
                 return true;
             };
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t k = 0; ok; ++k) {
+                // producer side of the item queue
+                int32_t u = p.item_counter != nullptr ? atomicAdd(p.item_counter, 1)
+                                                      : int32_t(blockIdx.x + k * gridDim.x);
+                if (u >= p.n_items) u = -1;
+                const int qe = int(k % kItemQ);
+                if (k >= uint32_t(kItemQ) &&
+                    !wait_bar(bar_item_empty(qe), ((k / kItemQ) - 1) & 1u, abort_flag, p)) {
+                    ok = false;
+                    break;
+                }
+                item_q[qe] = u;
+                ptx::mbar_arrive(bar_item_full(qe));
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const bool has_b = w.qb >= 0;
                 const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
@@ -367,7 +402,11 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t qaddr = base + C::kQOff + s * C::kQBytes;
             uint32_t item = 0, qc = 0, pc = 0, oc = 0, tc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t kq = 0; ok; ++kq) {
+                int32_t u;
+                if (!take_item(kq, u)) { ok = false; break; }
+                ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const bool has_b = w.qb >= 0;
                 const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
@@ -455,7 +494,15 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float c = p.scale_log2;
         uint32_t scnt = 0, ocnt = 0;
         bool ok = true;
-        for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+        for (uint32_t kq = 0; ok; ++kq) {
+            int32_t u = -1;
+            if (!__all_sync(0xffffffffu, take_item(kq, u))) {
+                ok = false;
+                break;
+            }
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
+            if (u < 0) break;
             const WorkItem w = p.items[u];
             if (slot == 1 && w.qb < 0) continue;
             const int32_t tile_a = w.qa / SPT;
@@ -673,6 +720,8 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     if (e != cudaSuccess) return e;
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
+    fp.item_counter = pl->d_counters + pl->launch_seq.fetch_add(1) % uint32_t(kCounterPool);
+    if ((e = cudaMemsetAsync(fp.item_counter, 0, sizeof(int32_t), stream)) != cudaSuccess) return e;
     if (raster)
         return P.padded ? launch_kernel<D, true, true>(grid, stream, mq, mk, mv, fp)
                         : launch_kernel<D, true, false>(grid, stream, mq, mk, mv, fp);

@@ -4,11 +4,15 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <vector>
 
 #include "sta.h"
 
 namespace sta {
+
+// Work counters per plan (see sta_plan_s::d_counters).
+constexpr int kCounterPool = 256;
 
 // Query rows per MMA slot (tcgen05 M for cta_group::1) and keys per K/V chunk.
 constexpr int kSubRows = 128;
@@ -65,6 +69,12 @@ struct sta_plan_s {
     uint32_t* d_status = nullptr;
     int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
     uint32_t* d_kmask = nullptr;  // device copy of key_mask (padded latents only)
+    // Work counters of the forward's run-time item hand-out: each launch takes
+    // the next of a pool (zeroed on its stream first), so calls that share the
+    // plan on different streams use different counters (up to the pool size
+    // in flight at once).
+    int32_t* d_counters = nullptr;
+    mutable std::atomic<uint32_t> launch_seq{0};
     int32_t* d_toff = nullptr;
     int32_t* d_tids = nullptr;
     sta::WorkItem* d_bq_items = nullptr;
