@@ -58,6 +58,11 @@ constexpr int kEwWarps = 8;
 constexpr uint32_t kBwTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kBoxBytes = 128 * 128;  // one TMA box: 128 rows x 128 bytes (64 bf16)
+// Work items are handed out at run time, as in the forward: the load warp
+// takes the next item from a per-launch global counter and passes it to the
+// MMA thread and the eight elementwise warps through a queue in shared memory.
+constexpr int kItemQ = 4;
+constexpr int kItemConsumers = 1 + kEwWarps;
 // Shared memory requested at launch is at least this, so one CTA holds an SM
 // alone: a second CTA on the SM would wait in tcgen05.alloc for the 512 TMEM
 // columns until the first one exits.
@@ -81,7 +86,8 @@ struct BwdParams {
     float scale;
     uint32_t* status;
     uint64_t timeout_ns;
-    RasterGeom rg;  // raster layout only
+    RasterGeom rg;          // raster layout only
+    int32_t* item_counter;  // next item to hand out (zeroed before the launch); null: fixed stride
 };
 
 __device__ __forceinline__ bool wait_bw(uint32_t bar, uint32_t parity, volatile int* abort_flag, const BwdParams& p) {
@@ -93,6 +99,28 @@ template <int D>
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* m, uint32_t bar, int32_t row) {
 #pragma unroll
     for (int cb = 0; cb < D / 64; ++cb) ptx::tma_load_2d(dst + cb * kBoxBytes, m, bar, cb * 64, row);
+}
+
+// Producer side of the item queue (one thread): publish this CTA's k-th item
+// (-1: none left) in entry k % kItemQ once that entry's previous item has been
+// taken by every consumer.  Returns the item, or -2 when the CTA is aborting.
+__device__ __forceinline__ int32_t put_item(uint32_t k, uint32_t full0, uint32_t empty0, volatile int32_t* q,
+                                            volatile int* abort_flag, const BwdParams& p) {
+    int32_t u = p.item_counter != nullptr ? atomicAdd(p.item_counter, 1) : int32_t(blockIdx.x + k * gridDim.x);
+    if (u >= p.n_items) u = -1;
+    const uint32_t e = k % kItemQ;
+    if (k >= uint32_t(kItemQ) && !wait_bw(empty0 + 8u * e, ((k / kItemQ) - 1) & 1u, abort_flag, p)) return -2;
+    q[e] = u;
+    ptx::mbar_arrive(full0 + 8u * e);
+    return u;
+}
+
+// Consumer side: wait for entry k and read it; false when the CTA is aborting.
+__device__ __forceinline__ bool get_item(uint32_t k, uint32_t full0, volatile int32_t* q, volatile int* abort_flag,
+                                        const BwdParams& p, int32_t& u) {
+    if (!wait_bw(full0 + 8u * (k % kItemQ), (k / kItemQ) & 1u, abort_flag, p)) return false;
+    u = q[k % kItemQ];
+    return true;
 }
 
 // 128-row block `sub` of tile `tile` of head bh: tile-major rows (2D map) or
@@ -197,10 +225,10 @@ struct DqCfg {
     static constexpr int kVOff = kKOff + kKStages * kBlk;
     static constexpr int kBarOff = kVOff + kVStages * kBlk;
     // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], q_full, q_empty,
-    // s_full[2], dp_full, ds_full, dq_full, drain
-    static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 9;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+    // s_full[2], dp_full, ds_full, dq_full, drain, item_full[Q], item_empty[Q]
+    static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 9 + 2 * kItemQ;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, item queue
+    static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemQ + 1024;
     static constexpr uint32_t kColS0 = 0, kColDP = 256, kColDQ = 384;
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
     static_assert(kColDQ + D <= kBwTmemCols, "TMEM budget");
@@ -228,8 +256,10 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t q_full = xb, q_empty = xb + 8;
     auto s_full = [&](int b) { return xb + 16 + 8u * b; };
     const uint32_t dp_full = xb + 32, ds_full = xb + 40, dq_full = xb + 48, drain = xb + 56;
+    const uint32_t item_full0 = xb + 64, item_empty0 = xb + 64 + 8 * kItemQ;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(smem + C::kMiscOff + 8);
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < KS; ++r) {
@@ -248,6 +278,10 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ptx::mbar_init(ds_full, kEwWarps);
         ptx::mbar_init(dq_full, 1);
         ptx::mbar_init(drain, 1);
+        for (int q = 0; q < kItemQ; ++q) {
+            ptx::mbar_init(item_full0 + 8u * q, 1);
+            ptx::mbar_init(item_empty0 + 8u * q, kItemConsumers);
+        }
         *abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
@@ -273,7 +307,10 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // ------------------------------------------------------------ load
             uint32_t kit = 0, vit = 0, qc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t kq = 0; ok; ++kq) {
+                const int32_t u = put_item(kq, item_full0, item_empty0, item_q, abort_flag, p);
+                if (u == -2) { ok = false; break; }
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const int32_t tile = w.qa / SPT;
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -321,7 +358,11 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const uint32_t qaddr = base + C::kQOff, doaddr = base + C::kDOOff;
             uint32_t kbase = 0, vbase = 0, gs = 0, qc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t kq = 0; ok; ++kq) {
+                int32_t u;
+                if (!get_item(kq, item_full0, item_q, abort_flag, p, u)) { ok = false; break; }
+                ptx::mbar_arrive(item_empty0 + 8u * (kq % kItemQ));
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const int32_t tile = w.qa / SPT;
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -396,7 +437,12 @@ sta_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint64_t c2 = ptx::f2(p.scale_log2, p.scale_log2);
         uint32_t gs = 0, dqc = 0;
         bool ok = true;
-        for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+        for (uint32_t kq = 0; ok; ++kq) {
+            int32_t u = -1;
+            if (!__all_sync(0xffffffffu, get_item(kq, item_full0, item_q, abort_flag, p, u))) break;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(item_empty0 + 8u * (kq % kItemQ));
+            if (u < 0) break;
             const WorkItem w = p.items[u];
             const int32_t tile = w.qa / SPT;
             const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -485,10 +531,10 @@ struct DkvCfg {
     static constexpr int kStageOff = 2 * kBlk;
     static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
     // st_full[2], st_empty[2], kv_full, kv_empty, s_full, dp_full, p_full,
-    // ds_full, dkv_full, drain
-    static constexpr int kNumBars = 2 * kStages + 8;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+    // ds_full, dkv_full, drain, item_full[Q], item_empty[Q]
+    static constexpr int kNumBars = 2 * kStages + 8 + 2 * kItemQ;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem slot, abort flag, item queue
+    static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemQ + 1024;
     static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
     static_assert(kStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -514,9 +560,11 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t xb = bar0 + 8u * (2 * NS);
     const uint32_t kv_full = xb, kv_empty = xb + 8, s_full = xb + 16, dp_full = xb + 24, p_full = xb + 32,
                    ds_full = xb + 40, dkv_full = xb + 48, drain = xb + 56;
+    const uint32_t item_full0 = xb + 64, item_empty0 = xb + 64 + 8 * kItemQ;
     auto stage = [&](int r) { return base + C::kStageOff + uint32_t(r) * C::kStageBytes; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(smem + C::kMiscOff + 8);
 
     if (threadIdx.x == 0) {
         for (int r = 0; r < NS; ++r) {
@@ -531,6 +579,10 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         ptx::mbar_init(ds_full, kEwWarps);
         ptx::mbar_init(dkv_full, 1);
         ptx::mbar_init(drain, 1);
+        for (int q = 0; q < kItemQ; ++q) {
+            ptx::mbar_init(item_full0 + 8u * q, 1);
+            ptx::mbar_init(item_empty0 + 8u * q, kItemConsumers);
+        }
         *abort_flag = 0;
         ptx::fence_barrier_init();
         ptx::fence_proxy_async_smem();
@@ -556,7 +608,10 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // ------------------------------------------------------------ load
             uint32_t sit = 0, kvc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t kq = 0; ok; ++kq) {
+                const int32_t u = put_item(kq, item_full0, item_empty0, item_q, abort_flag, p);
+                if (u == -2) { ok = false; break; }
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const int32_t ktile = w.qa / SPT;
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -597,7 +652,11 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const uint32_t kaddr = base + C::kKOff, vaddr = base + C::kVOff;
             uint32_t sbase = 0, gs = 0, kvc = 0;
             bool ok = true;
-            for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+            for (uint32_t kq = 0; ok; ++kq) {
+                int32_t u;
+                if (!get_item(kq, item_full0, item_q, abort_flag, p, u)) { ok = false; break; }
+                ptx::mbar_arrive(item_empty0 + 8u * (kq % kItemQ));
+                if (u < 0) break;
                 const WorkItem w = p.items[u];
                 const int32_t ktile = w.qa / SPT;
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -676,7 +735,12 @@ sta_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const uint64_t c2 = ptx::f2(p.scale_log2, p.scale_log2);
         uint32_t gs = 0, sbase = 0, kvc = 0;
         bool ok = true;
-        for (int32_t u = blockIdx.x; ok && u < p.n_items; u += gridDim.x) {
+        for (uint32_t kq = 0; ok; ++kq) {
+            int32_t u = -1;
+            if (!__all_sync(0xffffffffu, get_item(kq, item_full0, item_q, abort_flag, p, u))) break;
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(item_empty0 + 8u * (kq % kItemQ));
+            if (u < 0) break;
             const WorkItem w = p.items[u];
             const int32_t ktile = w.qa / SPT;
             const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
@@ -828,6 +892,8 @@ cudaError_t launch_bwd_variant(const sta_plan_s* pl, const CUtensorMap& mq, cons
         if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
     }
     // dQ
+    bp.item_counter = pl->d_counters + pl->launch_seq.fetch_add(1) % uint32_t(kCounterPool);
+    if (cudaError_t e = cudaMemsetAsync(bp.item_counter, 0, sizeof(int32_t), stream); e != cudaSuccess) return e;
     bp.items = pl->d_bq_items;
     bp.n_items = int32_t(P.bq_items.size());
     bp.off = pl->d_off;
@@ -843,6 +909,8 @@ cudaError_t launch_bwd_variant(const sta_plan_s* pl, const CUtensorMap& mq, cons
     sta_bwd_dq_kernel<D, kRaster, kPadded><<<grid, kBwThreads, kSmemDq, stream>>>(mq, mk, mv, mdo, bp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // dK, dV
+    bp.item_counter = pl->d_counters + pl->launch_seq.fetch_add(1) % uint32_t(kCounterPool);
+    if ((e = cudaMemsetAsync(bp.item_counter, 0, sizeof(int32_t), stream)) != cudaSuccess) return e;
     bp.items = pl->d_bkv_items;
     bp.n_items = int32_t(P.bkv_items.size());
     bp.off = pl->d_toff;
