@@ -880,15 +880,15 @@ cudaError_t make_rows_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) 
 template <int D, bool kRaster, bool kPadded>
 cudaError_t launch_bwd_variant(const sta_plan_s* pl, const CUtensorMap& mq, const CUtensorMap& mk,
                                const CUtensorMap& mv, const CUtensorMap& mdo, BwdParams bp, const void* o,
-                               const void* dout, const float* lse, void* dq, void* dk, void* dv, int64_t rows,
-                               int sms, cudaStream_t stream) {
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv, float* ws,
+                               int64_t rows, int sms, cudaStream_t stream) {
     const PlanHost& P = pl->h;
     {
         const int64_t threads = rows * (D / 8);
         const int64_t blocks = (threads + 255) / 256;
         bwd_prep_kernel<D, kRaster, kPadded><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
-            static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, const_cast<float*>(bp.neg_d),
-            const_cast<float*>(bp.neg_l), rows, bp.tokens, bp.rg);
+            static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, ws, ws + rows, rows, bp.tokens,
+            bp.rg);
         if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
     }
     // dQ
@@ -971,11 +971,11 @@ cudaError_t launch_bwd_d(const sta_plan_s* pl, const void* q, const void* k, con
     bp.timeout_ns = timeout_ns;
     bp.rg = raster_geom(pl);
     if (raster)
-        return P.padded ? launch_bwd_variant<D, true, true>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, rows,
+        return P.padded ? launch_bwd_variant<D, true, true>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, ws, rows,
                                                             sms, stream)
                         : launch_bwd_variant<D, true, false>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv,
-                                                             rows, sms, stream);
-    return launch_bwd_variant<D, false, false>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, rows, sms,
+                                                             ws, rows, sms, stream);
+    return launch_bwd_variant<D, false, false>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, ws, rows, sms,
                                                stream);
 }
 
