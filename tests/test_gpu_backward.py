@@ -247,3 +247,44 @@ def test_calls_from_a_fresh_thread(sta):
     assert torch.equal(box["fwd"][0], o_ref) and torch.equal(box["fwd"][1], l_ref)
     for a, b in zip(box["bwd"], ref):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("idx", [2, 4, 5])
+def test_backward_full_size_invariants(sta, idx):
+    """At every workload's full size: sum over keys of dV equals sum over
+    queries of dO (each row of P sums to 1), and sum over keys of dK is ~0
+    (each row of dS sums to 0).  Both hold at any size, so they cover dK and dV
+    where the oracle cannot go.  Tolerances: the sums run over N rows whose
+    terms carry bf16 rounding (relative 2^-9, random sign), so they are
+    bounded against sqrt(sum of squares) of the summed terms: 2e-2 of it for
+    dV, and for dK 2e-2 of sqrt(N) rms(dK).  For dK the rounding of dS to bf16
+    (the operand of the dS^T Q product) and of O (inside D) dominates: an
+    fp64 emulation of exactly those two roundings on N(0, 1) inputs, d = 128,
+    1536 keys per query, gives a ratio of 6.7e-3 median and 1.0e-2 at the
+    worst of 24 heads, so the bound leaves about 2x.  A missing or wrong D
+    term leaves each row of dS summing to D_i instead of 0: an O(1) ratio."""
+    w = sta_inputs.WORKLOADS[idx]
+    q, k, v = sta_inputs.make_qkv(w, device="cuda")
+    do = sta_inputs.make_dout(w, device="cuda")
+    wins = sta_inputs.windows(w).tolist()
+    plan, dq, dk, dv = gpu_grads(sta, q, k, v, do, w.latent, w.tile, wins, w.softmax_scale)
+    for t in (dq, dk, dv):
+        assert bool(torch.isfinite(t).all())
+    dv_sum = dv.double().sum(dim=2)
+    do_sum = do.double().sum(dim=2)
+    do_norm = do.double().pow(2).sum(dim=2).sqrt()
+    r_dv = float(((dv_sum - do_sum).abs() / do_norm).max())
+    assert r_dv <= 2e-2, ("sum dV - sum dO", r_dv)
+    dk_sum = dk.double().sum(dim=2)
+    n = dk.shape[2]
+    dk_scale = dk.double().pow(2).mean(dim=(2, 3)).sqrt().unsqueeze(-1) * n ** 0.5
+    r_dk = float((dk_sum.abs() / dk_scale).max())
+    assert r_dk <= 2e-2, ("sum dK", r_dk)
+    print(f"workload {idx}: sum dV vs dO {r_dv:.2e}, sum dK {r_dk:.2e}")
+    if idx == 4:
+        # the full-window workload: dQ on sampled rows against the oracle
+        toks = tile_rows(w.latent, w.tile, sample_tiles(w.latent, w.tile, 1, seed=14), 2, seed=15)
+        rows = np.array([(h, t) for h in (0, 11) for t in toks], dtype=np.int64)
+        ref = oracle.sta_backward_dq(q.cpu(), k.cpu(), v.cpu(), do.cpu(), w.latent, w.tile, wins,
+                                     w.softmax_scale, rows=rows)
+        compare_grad(rows_of(dq, rows), ref, rows[:, 0], what="dq full window")
