@@ -12,7 +12,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libsta.so")
 
 SOURCES = ["sta_api.cu", "sta_permute.cu", "sta_forward.cu", "sta_backward.cu", "sta_search.cu", "sta_pipe.cu", "sta_noalloc.cu"]
-HEADERS = ["sta_internal.h", "sta_ptx.cuh", "sta_wait.cuh"]
+HEADERS = ["sta_internal.h", "sta_ptx.cuh", "sta_raster.cuh", "sta_wait.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
