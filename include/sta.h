@@ -38,6 +38,11 @@
  *   - Calls return a status and never throw, abort or print.  Argument errors
  *     are detected before any launch.  Faults and device-side timeouts of
  *     launched work are reported by sta_last_device_status.
+ *   - Empty problems: a plan may have batch 0, and the permutations take
+ *     outer 0 and sta_window_stats slices 0.  Such calls check their other
+ *     arguments, launch nothing and return STA_OK; their tensor pointers are
+ *     not read and may be NULL (an empty PyTorch tensor has a null data
+ *     pointer).
  */
 #ifndef STA_H_
 #define STA_H_
@@ -76,7 +81,7 @@ typedef struct sta_plan_s* sta_plan_t;
 /* Build a plan and upload it to the current CUDA device.
  *   g          : geometry; L_d >= 1 and T_d >= 1 (an axis that is not a
  *                multiple of its tile is padded to whole tiles).
- *   batch      : B >= 1;  heads: H >= 1
+ *   batch      : B >= 0 (0: an empty plan, see the conventions);  heads: H >= 1
  *   window_thw : host array [heads][3], window per head in tokens; every entry
  *                a positive multiple of the tile extent on its axis (windows
  *                wider than the volume are clamped to it)
@@ -138,7 +143,7 @@ STA_API sta_status sta_plan_backward_items(sta_plan_t p, int32_t which, int32_t*
  *   src       : device, [outer, N, row_bytes] bytes (raster)
  *   dst       : device, [outer, N_tiles, row_bytes] bytes (tile-major; padding
  *               rows written as zeros), not overlapping src
- *   outer     : B * heads (any count >= 1)
+ *   outer     : B * heads (any count >= 0)
  *   row_bytes : bytes of one token row (d * element size; 4 for a fp32 LSE
  *               row); rows move intact, bit-exact
  * dst[o, tile_major(i)] = src[o, i] for every raster token i. */
@@ -242,7 +247,7 @@ STA_API sta_status sta_backward_raster(sta_plan_t p, const void* q, const void* 
  *   mse             : device fp64 [slices] (written): mean of (o_w - o_full)^2
  *                     over rows and channels (the mask-search loss, read here
  *                     as the output's mean squared error against full attention)
- * 1 <= slices (B * heads) <= 2^28, tokens >= 1, head_dim a positive multiple
+ * 0 <= slices (B * heads) <= 2^28, tokens >= 1, head_dim a positive multiple
  * of 8, else INVALID_ARG.  One kernel (a cluster of 8 CTAs per slice),
  * deterministic; allocates nothing. */
 STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, const void* o_w,
@@ -257,7 +262,8 @@ STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, c
  * of call i and the copy-out of call i-1 running at once.
  *
  * sta_pipe_create: plan from sta_plan on the current device (its tile shape
- *   must suit sta_forward_raster, else UNSUPPORTED); head_dim 64 or 128;
+ *   must suit sta_forward_raster, else UNSUPPORTED; batch 0 is INVALID_ARG:
+ *   nothing to pipeline); head_dim 64 or 128;
  *   softmax_scale finite and > 0; 1 <= depth <= 8.  Allocates depth x (four
  *   [B, heads, N, d] bf16 tensors + one fp32 LSE) of device memory and three
  *   streams; OOM / CUDA on failure.  The plan must outlive the pipeline.
@@ -293,11 +299,13 @@ STA_API sta_status sta_pipe_destroy(sta_pipe_t pipe);
  * library: 4 MiB of device memory on every GPU that loads the library, held
  * until the process exits.
  *
- * Limits: heads <= 1024, and the plan must fit the scratch:
+ * Limits: every latent axis a multiple of its tile (padded latents need
+ * sta_plan + sta_forward), heads <= 1024, and the plan must fit the scratch:
  *   256 + 16 * work_items + 4 * (n_windows * (tiles + 1) + sum over distinct
  *   windows of tiles * window_tiles) <= 4 MiB
  * (the 720p and 42x64x112 workloads of this library use 0.7 and 1.3 MiB).
- * Larger problems, or heads > 1024, return STA_ERR_UNSUPPORTED before any work.
+ * Larger problems, heads > 1024 or a padded latent return STA_ERR_UNSUPPORTED
+ * before any work.  batch 0 returns STA_OK at once (pointers unread).
  *
  * Behaviour: the first call on a device looks up the scratch's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any stream

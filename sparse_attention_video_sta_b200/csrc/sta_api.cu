@@ -101,7 +101,7 @@ void order_rounds(std::vector<WorkItem>& items, const Len& len, int32_t ctas) {
 // device's SM count; 148 for host-only plans).
 sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
                            const int32_t* window_thw, int32_t ctas, PlanHost& P) {
-    if (!geom_valid(g) || batch < 1 || heads < 1 || window_thw == nullptr)
+    if (!geom_valid(g) || batch < 0 || heads < 1 || window_thw == nullptr)
         return STA_ERR_INVALID_ARG;
     const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
     const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
@@ -310,8 +310,9 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row_bytes,
                           const sta_geom* g, void* stream, bool inverse) {
-    if (src == nullptr || dst == nullptr || !geom_valid(g) || outer < 1 || row_bytes <= 0)
-        return STA_ERR_INVALID_ARG;
+    if (!geom_valid(g) || outer < 0 || row_bytes <= 0) return STA_ERR_INVALID_ARG;
+    if (outer == 0) return STA_OK;  // no rows: nothing to move
+    if (src == nullptr || dst == nullptr) return STA_ERR_INVALID_ARG;
     const int64_t n_tok = int64_t(g->lat_t) * g->lat_h * g->lat_w;
     int64_t n_pad = 1;  // tile-major rows per slice: whole tiles
     const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w}, T[3] = {g->tile_t, g->tile_h, g->tile_w};
@@ -328,13 +329,15 @@ sta_status permute_common(const void* src, void* dst, int64_t outer, int32_t row
 sta_status forward_common(sta_plan_t p, const void* q, const void* k, const void* v, void* o, float* lse,
                           int32_t head_dim, float softmax_scale, void* stream, bool raster) {
     if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
+    if (p->h.batch == 0) return STA_OK;  // no rows: nothing to compute
     if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
         return STA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
         return STA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
     int dev = -1;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
     if (dev != p->device) return STA_ERR_INVALID_ARG;
@@ -342,7 +345,6 @@ sta_status forward_common(sta_plan_t p, const void* q, const void* k, const void
     const int inject = g_inject_timeout.load();
     const uint64_t limit = inject ? uint64_t(g_inject_limit_ms.load()) * 1000000ull
                                   : kDefaultTimeoutNs;
-    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
     clear_stale_error();
     return cuda_status(sta::launch_forward(p, q, k, v, o, lse, head_dim, softmax_scale,
                                            static_cast<cudaStream_t>(stream), inject, limit, raster));
@@ -374,17 +376,18 @@ sta_status backward_common(sta_plan_t p, const void* q, const void* k, const voi
                            const void* dout, const float* lse, void* dq, void* dk, void* dv, float* workspace,
                            int32_t head_dim, float softmax_scale, void* stream, bool raster) {
     if (p == nullptr || !p->on_device) return STA_ERR_INVALID_ARG;
+    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
+    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
+    if (p->h.batch == 0) return STA_OK;  // no rows: nothing to compute
     const void* in16[] = {q, k, v, o, dout, dq, dk, dv, workspace};
     for (const void* x : in16)
         if (x == nullptr || !aligned(x, 16)) return STA_ERR_INVALID_ARG;
     if (lse == nullptr || !aligned(lse, 4)) return STA_ERR_INVALID_ARG;
-    if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
-    if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
     int dev = -1;
     if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return cuda_status(e);
     if (dev != p->device) return STA_ERR_INVALID_ARG;
     if (cudaError_t e = make_context_current(dev); e != cudaSuccess) return cuda_status(e);
-    if (raster && !sta::raster_box(p->h.g).ok) return STA_ERR_UNSUPPORTED;
     clear_stale_error();
     return cuda_status(sta::launch_backward(p, q, k, v, o, dout, lse, dq, dk, dv, workspace, head_dim,
                                             softmax_scale, static_cast<cudaStream_t>(stream), kDefaultTimeoutNs,
@@ -564,14 +567,15 @@ sta_status sta_backward_raster(sta_plan_t p, const void* q, const void* k, const
 sta_status sta_window_stats(const float* lse_w, const float* lse_full, const void* o_w, const void* o_full,
                             int64_t slices, int64_t tokens, int32_t head_dim, double* recall, double* mse,
                             void* stream) {
+    // 8 CTAs per slice in the launch grid
+    if (slices < 0 || slices > (int64_t(1) << 28) || tokens < 1 || head_dim < 8 || head_dim % 8 != 0)
+        return STA_ERR_INVALID_ARG;
+    if (slices == 0) return STA_OK;  // no slices: nothing to reduce
     if (lse_w == nullptr || lse_full == nullptr || o_w == nullptr || o_full == nullptr || recall == nullptr ||
         mse == nullptr)
         return STA_ERR_INVALID_ARG;
     if (!aligned(lse_w, 4) || !aligned(lse_full, 4) || !aligned(o_w, 16) || !aligned(o_full, 16) ||
         !aligned(recall, 8) || !aligned(mse, 8))
-        return STA_ERR_INVALID_ARG;
-    // 8 CTAs per slice in the launch grid
-    if (slices < 1 || slices > (int64_t(1) << 28) || tokens < 1 || head_dim < 8 || head_dim % 8 != 0)
         return STA_ERR_INVALID_ARG;
     clear_stale_error();
     return cuda_status(sta::launch_window_stats(lse_w, lse_full, o_w, o_full, slices, tokens, head_dim, recall,

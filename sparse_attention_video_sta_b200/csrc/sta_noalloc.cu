@@ -76,18 +76,14 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
                                           const void* v, void* o, float* lse, int32_t head_dim,
                                           float softmax_scale, void* stream) {
     // ---- arguments (same rules as sta_plan + sta_forward)
-    if (g == nullptr || window_thw == nullptr || batch < 1 || heads < 1) return STA_ERR_INVALID_ARG;
-    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
-        return STA_ERR_INVALID_ARG;
-    auto aligned = [](const void* p, uintptr_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; };
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
-        return STA_ERR_INVALID_ARG;
+    if (g == nullptr || window_thw == nullptr || batch < 0 || heads < 1) return STA_ERR_INVALID_ARG;
     if (!std::isfinite(softmax_scale) || !(softmax_scale > 0.0f)) return STA_ERR_INVALID_ARG;
     const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w};
     const int32_t T[3] = {g->tile_t, g->tile_h, g->tile_w};
     int32_t n[3];
     for (int d = 0; d < 3; ++d) {
-        if (L[d] <= 0 || T[d] <= 0 || L[d] % T[d] != 0) return STA_ERR_INVALID_ARG;
+        if (L[d] <= 0 || T[d] <= 0) return STA_ERR_INVALID_ARG;
+        if (L[d] % T[d] != 0) return STA_ERR_UNSUPPORTED;  // padded latents: sta_plan + sta_forward
         n[d] = L[d] / T[d];
     }
     for (int32_t h = 0; h < heads; ++h)
@@ -101,6 +97,12 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
     const int32_t tile_tokens = T[0] * T[1] * T[2];
     if (tile_tokens % sta::kSubRows != 0) return STA_ERR_UNSUPPORTED;
     if (int64_t(batch) * heads * n_tok > INT32_MAX) return STA_ERR_UNSUPPORTED;
+    if (batch == 0) return STA_OK;  // no rows: nothing to compute
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr)
+        return STA_ERR_INVALID_ARG;
+    auto aligned = [](const void* p, uintptr_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; };
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return STA_ERR_INVALID_ARG;
     const int32_t tiles = n[0] * n[1] * n[2];
     const int32_t S = tile_tokens / sta::kSubRows;
 

@@ -87,6 +87,7 @@ sta_status sta_pipe_create(sta_plan_t plan, int32_t head_dim, float softmax_scal
     if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
     // The pipeline keeps raster tensors and runs the fused forward.
     if (!sta::raster_box(plan->h.g).ok) return STA_ERR_UNSUPPORTED;
+    if (plan->h.batch == 0) return STA_ERR_INVALID_ARG;  // no rows to pipeline
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return STA_ERR_CUDA;
     if (dev != plan->device) return STA_ERR_INVALID_ARG;

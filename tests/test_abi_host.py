@@ -59,7 +59,7 @@ def test_plan_argument_validation():
     assert _raw_plan_host((30, 48, 80), (6, 0, 8), 1, 1, [(18, 24, 24)])[0] == INV
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(18, 24, 20)])[0] == INV  # window % tile
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 1, [(0, 24, 24)])[0] == INV
-    assert _raw_plan_host((30, 48, 80), (6, 8, 8), 0, 1, [(18, 24, 24)])[0] == INV
+    assert _raw_plan_host((30, 48, 80), (6, 8, 8), -1, 1, [(18, 24, 24)])[0] == INV
     assert _raw_plan_host((30, 48, 80), (6, 8, 8), 1, 0, [])[0] == INV
     assert _raw_plan_host((30, 48, 80), (3, 8, 8), 1, 1, [(18, 24, 24)])[0] == UNS  # 192 tokens
     # int32 row-coordinate limit of the kernel's tensor maps
@@ -78,7 +78,7 @@ def test_calls_rejected_before_launch():
     assert lib.sta_tile_reorder(None, p, 1, 128, ctypes.byref(g), None) == INV
     assert lib.sta_tile_reorder(p, None, 1, 128, ctypes.byref(g), None) == INV
     assert lib.sta_tile_reorder(p, ctypes.c_void_p((1 << 20) + 64), 1, 128, ctypes.byref(g), None) == INV
-    assert lib.sta_tile_reorder(p, ctypes.c_void_p(1 << 34), 0, 128, ctypes.byref(g), None) == INV
+    assert lib.sta_tile_reorder(p, ctypes.c_void_p(1 << 34), -1, 128, ctypes.byref(g), None) == INV
     assert lib.sta_tile_reorder(p, ctypes.c_void_p(1 << 34), 1, 0, ctypes.byref(g), None) == INV
     assert lib.sta_tile_unreorder(p, ctypes.c_void_p(1 << 34), 1, 128, ctypes.byref(bad), None) == INV
     # forward: host-only plan, null / misaligned pointers, bad scale, bad head_dim
@@ -205,7 +205,8 @@ def test_window_stats_rejected_before_launch():
     odd = ctypes.c_void_p((1 << 30) + 8)
     assert lib.sta_window_stats(None, a, a, a, 1, 128, 64, a, a, None) == INV
     assert lib.sta_window_stats(a, a, odd, a, 1, 128, 64, a, a, None) == INV   # o not 16-byte aligned
-    assert lib.sta_window_stats(a, a, a, a, 0, 128, 64, a, a, None) == INV     # no slices
+    assert lib.sta_window_stats(a, a, a, a, -1, 128, 64, a, a, None) == INV    # negative slice count
+    assert lib.sta_window_stats(a, a, a, a, 0, 128, 64, a, a, None) == 0       # no slices: a no-op
     assert lib.sta_window_stats(a, a, a, a, 1, 0, 64, a, a, None) == INV       # no tokens
     assert lib.sta_window_stats(a, a, a, a, 1, 128, 12, a, a, None) == INV     # head_dim not a multiple of 8
 
@@ -288,3 +289,51 @@ def test_backward_work_lists(latent, tile, heads, batch, wins):
             for c, it in enumerate(items[r0:r0 + R]):
                 loads[c] += length(it)
             assert max(loads) - min(loads) <= longest, (which, r0, max(loads), min(loads))
+
+
+def test_empty_problems_are_no_ops():
+    """Batch 0 (and outer 0, slices 0): the other arguments are still checked,
+    nothing is launched, STA_OK is returned and the tensor pointers (null for
+    an empty PyTorch tensor) are not read."""
+    INV, UNS = sta.STA_ERR_INVALID_ARG, sta.STA_ERR_UNSUPPORTED
+    lib = sta._lib
+    st, h = _raw_plan_host((18, 24, 24), (6, 8, 8), 0, 2, [(12, 16, 16), (18, 24, 24)])
+    assert st == 0
+    pairs, items = ctypes.c_int64(-1), ctypes.c_int64(-1)
+    assert lib.sta_plan_stats(h, ctypes.byref(pairs), ctypes.byref(items)) == 0
+    assert pairs.value == 0 and items.value == 0
+    for which in (0, 1):
+        cnt = ctypes.c_int64(-1)
+        assert lib.sta_plan_backward_items(h, which, None, 0, ctypes.byref(cnt)) == 0
+        assert cnt.value == 0
+    # the key-tile lists still exist: they do not depend on the batch
+    ids = (ctypes.c_int32 * 27)()
+    cnt32 = ctypes.c_int32(-1)
+    assert lib.sta_plan_query(h, 1, 13, ids, 27, ctypes.byref(cnt32)) == 0 and cnt32.value == 27
+    assert lib.sta_plan_destroy(h) == 0
+    g = sta._geom((18, 24, 24), (6, 8, 8))
+    bad = sta._geom((18, 24, 0), (6, 8, 8))
+    assert lib.sta_tile_reorder(None, None, 0, 256, ctypes.byref(g), None) == 0
+    assert lib.sta_tile_unreorder(None, None, 0, 256, ctypes.byref(g), None) == 0
+    assert lib.sta_tile_reorder(None, None, 0, 256, ctypes.byref(bad), None) == INV
+    assert lib.sta_tile_reorder(None, None, 0, 0, ctypes.byref(g), None) == INV
+    f64 = ctypes.POINTER(ctypes.c_double)
+    assert lib.sta_window_stats(None, None, None, None, 0, 100, 128, None, None, None) == 0
+    assert lib.sta_window_stats(None, None, None, None, 0, 0, 128, None, None, None) == INV
+    assert lib.sta_window_stats(None, None, None, None, -1, 100, 128, None, None, None) == INV
+    assert lib.sta_window_stats(None, None, None, None, 1, 100, 128, None, None, None) == INV
+    # the no-allocation forward: batch 0 is a no-op; a padded latent is unsupported
+    w = (ctypes.c_int32 * 3)(12, 16, 16)
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 0, 1, w, None, None, None, None, None, 128,
+                                   ctypes.c_float(0.088), None) == 0
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 0, 1, w, None, None, None, None, None, 96,
+                                   ctypes.c_float(0.088), None) == UNS
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 0, 1, w, None, None, None, None, None, 128,
+                                   ctypes.c_float(0.0), None) == INV
+    pad = sta._geom((18, 24, 20), (6, 8, 8))
+    assert lib.sta_forward_noalloc(ctypes.byref(pad), 1, 1, w, None, None, None, None, None, 128,
+                                   ctypes.c_float(0.088), None) == UNS
+    assert lib.sta_forward_noalloc(ctypes.byref(g), -1, 1, w, None, None, None, None, None, 128,
+                                   ctypes.c_float(0.088), None) == INV
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 1, 1, w, None, None, None, None, None, 128,
+                                   ctypes.c_float(0.088), None) == INV

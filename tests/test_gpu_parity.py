@@ -292,3 +292,38 @@ def test_fused_raster_rejects_unsupported_tiles(sta):
     o, l = sta.sta_attention(x, x, x, plan, 0.125)   # runs the reorder / forward / unreorder kernels
     assert sta.sta_last_device_status(plan) == 0
     assert torch.count_nonzero(o).item() == 0
+
+
+@pytest.mark.parametrize("latent", [(18, 24, 24), (13, 21, 18)])
+def test_empty_batch_is_a_no_op(sta, latent):
+    """B = 0: every call returns empty results without launching, for
+    divisible and padded latents, through the plan, the fused and the permuted
+    paths, the backward, autograd, the window statistics and the
+    no-allocation forward; a later non-empty call on the device is unaffected."""
+    tile, H, d = (6, 8, 8), 2, 64
+    N = latent[0] * latent[1] * latent[2]
+    plan = sta.sta_plan(latent, tile, 0, H, [(12, 16, 16)] * H)
+    assert plan.flops(d) == 0
+    q = torch.empty(0, H, N, d, device="cuda", dtype=torch.bfloat16)
+    for fused in (True, False):
+        o, lse = sta.sta_attention(q, q, q, plan, fused=fused)
+        assert o.shape == q.shape and tuple(lse.shape) == (0, H, N)
+        dq, dk, dv = sta.sta_attention_backward(q, q, q, o, lse, q, plan, fused=fused)
+        assert dq.shape == dk.shape == dv.shape == q.shape
+    qq = q.clone().requires_grad_(True)
+    sta.StaAttention.apply(qq, qq, qq, plan).sum().backward()
+    assert qq.grad.shape == q.shape
+    r, m = sta.sta_window_stats(lse, lse, o, o)
+    assert tuple(r.shape) == (0, H) and tuple(m.shape) == (0, H)
+    if latent == (18, 24, 24):
+        lse0 = torch.empty(0, H, N, device="cuda", dtype=torch.float32)
+        sta.sta_forward_noalloc(latent, tile, 0, H, [(12, 16, 16)] * H, q, q, q, q.clone(), lse0, 0.125)
+    assert sta.sta_last_device_status(plan) == 0
+    plan.destroy()
+    # the next real call runs normally
+    w = sta_inputs.WORKLOADS[1]
+    qa, ka, va = (x.cuda() for x in sta_inputs.make_qkv(w))
+    p1 = sta.sta_plan(w.latent, w.tile, w.batch, w.heads, sta_inputs.windows(w).tolist())
+    o1, l1 = sta.sta_attention(qa, ka, va, p1, w.softmax_scale)
+    assert sta.sta_last_device_status(p1) == 0
+    assert bool(torch.isfinite(o1.float()).all()) and bool(torch.isfinite(l1).all())
