@@ -94,7 +94,16 @@ typedef struct sta_plan_s* sta_plan_t;
  * per SM), the raster origin of every tile, and for padded latents the real-key
  * mask of every 128-key chunk.  Allocates device memory; free it with
  * sta_plan_destroy.  Errors: INVALID_ARG, UNSUPPORTED (tile volume not a
- * multiple of 128 tokens, or more than 2^31 - 1 tile-major rows), OOM, CUDA. */
+ * multiple of 128 tokens, or more than 2^31 - 1 tile-major rows), OOM, CUDA.
+ *
+ * Sharing a plan: the forward and backward kernels hand out work items at run
+ * time through a counter, which each launch takes from a pool of 256 in the
+ * plan (in turn) and zeroes on its own stream first.  Calls on one stream may
+ * share a plan without limit; calls running at the same time on different
+ * streams may share it while at most 256 of them are in flight at once.  A
+ * CUDA graph records the counter it was captured with: one captured graph
+ * must not be replayed on two streams at the same time (capture it once per
+ * stream, or use one plan per stream). */
 STA_API sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
                     const int32_t* window_thw, void* stream, sta_plan_t* out);
 
@@ -166,8 +175,9 @@ STA_API sta_status sta_tile_unreorder(const void* src, void* dst, int64_t outer,
  *             finite and > 0, else INVALID_ARG
  * For every (b, h) and query tile q, over the key tiles of the plan's list:
  * S = scale * Q_q K^T, exact online softmax with running max and sum in fp32,
- * O = softmax(S) V rounded to bf16.  Allocates nothing; enqueues one kernel on
- * `stream`.  The plan must come from sta_plan on the current device. */
+ * O = softmax(S) V rounded to bf16.  Allocates nothing; enqueues a 4-byte
+ * memset (the plan's work counter, see sta_plan) and one kernel on `stream`.
+ * The plan must come from sta_plan on the current device. */
 STA_API sta_status sta_forward(sta_plan_t p, const void* q, const void* k, const void* v,
                        void* o, float* lse, int32_t head_dim, float softmax_scale,
                        void* stream);
@@ -210,7 +220,8 @@ STA_API sta_status sta_forward_raster(sta_plan_t p, const void* q, const void* k
  *   head_dim, softmax_scale: as sta_forward
  * P and dS enter the tensor-core products as bf16 with fp32 accumulation;
  * dq, dk, dv are rounded to bf16.  No atomics: results are deterministic.
- * Allocates nothing; enqueues three kernels on `stream`.  Errors: INVALID_ARG
+ * Allocates nothing; enqueues three kernels (and two 4-byte memsets of work
+ * counters) on `stream`.  Errors: INVALID_ARG
  * (null or misaligned pointer, bad scale, plan not on the current device),
  * UNSUPPORTED (head_dim), CUDA. */
 STA_API sta_status sta_backward(sta_plan_t p, const void* q, const void* k, const void* v,
@@ -275,7 +286,9 @@ STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, c
  *   different current device.
  * sta_pipe_wait: block until all submitted calls are done; returns the first
  *   CUDA error or the plan's device status (as sta_last_device_status).
- * sta_pipe_destroy: wait, then free everything (NULL accepted). */
+ * sta_pipe_destroy: wait, then free everything (NULL accepted).
+ * A pipeline holds no lock: calls on one pipeline must come from one host
+ * thread at a time (separate pipelines may be driven from separate threads). */
 typedef struct sta_pipe_s* sta_pipe_t;
 STA_API sta_status sta_pipe_create(sta_plan_t p, int32_t head_dim, float softmax_scale, int32_t depth,
                                    sta_pipe_t* out);
