@@ -54,7 +54,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="sta", choices=["sta", "reference"])
-    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--workload", type=int, default=2, choices=[1, 2, 3, 4, 5],
+                    help="1 tiny, 2 720p (the default and the headline line), 3 mixed per-head windows, "
+                         "4 full window, 5 large with scaled heads")
     ap.add_argument("--heads", type=int, default=0,
                     help="override the head count (small cases for profiling only)")
     ap.add_argument("--no-extras", action="store_true",
