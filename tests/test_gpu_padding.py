@@ -63,6 +63,12 @@ def inputs(latent, B, H, d, seed):
     ((7, 9, 9), (2, 8, 8), 1, 2, 128, [[2, 8, 8], [8, 16, 16]]),
 ])
 def test_padded_forward_and_backward_all_rows(sta, latent, tile, B, H, d, windows):
+    check_all_rows(sta, latent, tile, B, H, d, windows)
+
+
+def check_all_rows(sta, latent, tile, B, H, d, windows):
+    """Forward and backward on every row against the oracle; the fused raster
+    kernels (where the tile shape and latent allow them) equal the reorder chain."""
     q, k, v, do = inputs(latent, B, H, d, seed=sum(latent) * 7 + d)
     scale = 1.0 / np.sqrt(d)
     plan = sta.sta_plan(latent, tile, B, H, windows)
@@ -88,6 +94,42 @@ def test_padded_forward_and_backward_all_rows(sta, latent, tile, B, H, d, window
     for name, a, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
         compare_grad(a.cpu().reshape(-1, d), r.reshape(-1, d), bh, what=f"{name} padded {latent}",
                      extra=extra[name])
+
+
+@pytest.mark.parametrize("latent,tile,d", [
+    ((6, 8, 8), (6, 8, 8), 128),    # the latent is exactly one tile
+    ((5, 7, 8), (6, 8, 8), 64),     # smaller than one tile: a single padded tile
+    ((1, 16, 16), (2, 8, 8), 128),  # the t axis is shorter than the tile
+    ((3, 3, 40), (6, 8, 8), 128),   # one row of tiles along w, padded in t and h
+])
+def test_degenerate_latents_all_rows(sta, latent, tile, d):
+    """Grids of one tile or one row of tiles, latents smaller than the tile:
+    a one-tile window and a window three tiles wide on every axis (clamped to
+    the volume)."""
+    check_all_rows(sta, latent, tile, 1, 2, d, [list(tile), [3 * x for x in tile]])
+
+
+def test_single_token_latent(sta):
+    """A 1 x 1 x 1 latent: each row's softmax has one key, so O = V and
+    dV = dO exactly (the weight is 1 and rounds to 1 in bf16), LSE is the one
+    scaled score, and dQ, dK vanish up to fp32 rounding: dS = P (dO.v - dO.o)
+    with o = v, the two dot products summed in different orders, at most
+    d 2^-24 sum |dO_c v_c| (~6e-4 for these N(0, 1) rows) times scale |k| <= 0.5."""
+    latent, tile, B, H, d = (1, 1, 1), (6, 8, 8), 2, 3, 128
+    q, k, v, do = inputs(latent, B, H, d, seed=11)
+    scale = 1.0 / np.sqrt(d)
+    plan = sta.sta_plan(latent, tile, B, H, [list(tile)] * H)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = sta.sta_attention(qd, kd, vd, plan, scale)
+    assert sta.sta_last_device_status(plan) == 0
+    assert torch.equal(o.cpu(), v)
+    o_ref, lse_ref = oracle.sta_attention(q, k, v, latent, tile, [list(tile)] * H, scale)
+    compare(o.cpu().reshape(-1, d), lse.cpu().reshape(-1), o_ref.reshape(-1, d), lse_ref.reshape(-1),
+            what="single token")
+    dq, dk, dv = sta.sta_attention_backward(qd, kd, vd, o, lse, dod, plan, scale)
+    assert sta.sta_last_device_status(plan) == 0
+    assert torch.equal(dv.cpu(), do)
+    assert float(dq.abs().max()) <= 2.0 ** -10 and float(dk.abs().max()) <= 2.0 ** -10
 
 
 def test_hunyuan_720p_latent_sampled(sta):
