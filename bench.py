@@ -84,13 +84,14 @@ def sources_hash():
     return h.hexdigest()[:16]
 
 
-def measured_traffic():
+def measured_traffic(workload_name: str):
     """DRAM bytes per forward launch from the committed ncu summary, or None
-    when the kernel sources changed since the counters were taken."""
+    when it covers another workload or the kernel sources changed since the
+    counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
-        if t.get("sources_hash") == sources_hash():
+        if t.get("sources_hash") == sources_hash() and t.get("workload") == workload_name:
             return float(t["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -498,8 +499,8 @@ def main():
             "config": workload_config(w, wins, world),
             "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": fwd_tflops / peak, "traffic": measured_traffic(),
-                         "kernel": "sta_fwd_kernel<128, raster>",
+                         "frac": fwd_tflops / peak, "traffic": measured_traffic(w.name),
+                         "kernel": f"sta_fwd_kernel<{d}, raster>",
                          "peak_source": f"bf16_tflops_sustained ({peak_kind})",
                          "frac_of_burst": fwd_tflops / float(peaks.get("bf16_tflops", 1590.0))},
             "gpu_launches": launches_per_step * args.steps,
