@@ -180,6 +180,23 @@ def weak_scaling_tflops(world: int, flops_per_rank: float, ms: float) -> float:
     return world * flops_per_rank / (ms * 1e-3) / 1e12
 
 
+def useful_flops(latent, tile, window, batch: int, heads: int, d: int) -> float:
+    """FLOPs of attention over real tokens only (4 d per attended real (query,
+    key) pair) on a padded tile grid; per axis, the real queries of each tile
+    times the real keys of its window's tiles, multiplied over the axes."""
+    total = 1.0
+    for L, T, W in zip(latent, tile, window):
+        n = -(-L // T)
+        e = min(W // T, n)
+        real = [min(T, L - i * T) for i in range(n)]
+        acc = 0
+        for q in range(n):
+            s0 = min(max(q - e // 2, 0), n - e)
+            acc += real[q] * sum(real[s0:s0 + e])
+        total *= acc
+    return 4.0 * d * total * batch * heads
+
+
 def cpu_baseline(w, n_tiles: int, heads):
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
     import oracle
@@ -433,6 +450,34 @@ def main():
                                   "recall_min_head": float(recall.mean(dim=0).min()),
                                   "mse_mean": float(err.mean())}
         del o_win, lse_win
+        # ------------------------------------------- padded latent (not a tile multiple)
+        # HunyuanVideo's own 5 s 720p latent, 33 x 45 x 80, padded to 36 x 48 x 80
+        # on the 6 x 8 x 8 tile grid; same heads, head dimension and window.
+        if tuple(w.latent) == (30, 48, 80):
+            pl = (33, 45, 80)
+            pn = pl[0] * pl[1] * pl[2]
+            pq, pk_, pv = (torch.randn((B, H, pn, d), generator=gen, device=dev).to(torch.bfloat16) for _ in range(3))
+            po, plse = torch.empty_like(pq), torch.empty((B, H, pn), dtype=torch.float32, device=dev)
+            pplan = sta.sta_plan(pl, T, B, H, wins)
+            for _ in range(2):
+                sta.sta_forward_raster(pplan, pq, pk_, pv, po, plse, scale)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(5):
+                sta.sta_forward_raster(pplan, pq, pk_, pv, po, plse, scale)
+            e1.record()
+            torch.cuda.synchronize()
+            if sta.sta_last_device_status(pplan) != 0:
+                raise RuntimeError("device status error in the padded-latent run")
+            p_ms = reduce_max(e0.elapsed_time(e1) / 5)
+            p_useful = useful_flops(pl, T, wins[0], B, H, d) if w.window is not None else None
+            extras["padded_latent"] = {"latent": list(pl), "padded_to": [-(-pl[i] // T[i]) * T[i] for i in range(3)],
+                                       "ms": p_ms, "tflops_executed": pplan.flops(d) / (p_ms * 1e-3) / 1e12,
+                                       "tflops_useful": (p_useful / (p_ms * 1e-3) / 1e12) if p_useful else None,
+                                       "kernel": f"sta_fwd_kernel<{d}, raster, padded>"}
+            pplan.destroy()
+            del pq, pk_, pv, po, plse
         # ------------------------------------------- unfused pipeline
         for _ in range(2):
             permuted_step()
