@@ -473,7 +473,7 @@ def main():
             p_ms = reduce_max(e0.elapsed_time(e1) / 5)
             p_useful = useful_flops(pl, T, wins[0], B, H, d) if w.window is not None else None
             extras["padded_latent"] = {"latent": list(pl), "padded_to": [-(-pl[i] // T[i]) * T[i] for i in range(3)],
-                                       "ms": p_ms, "tflops_executed": pplan.flops(d) / (p_ms * 1e-3) / 1e12,
+                                       "ms": p_ms, "tflops_tile_pairs": pplan.flops(d) / (p_ms * 1e-3) / 1e12,
                                        "tflops_useful": (p_useful / (p_ms * 1e-3) / 1e12) if p_useful else None,
                                        "kernel": f"sta_fwd_kernel<{d}, raster, padded>"}
             pplan.destroy()

@@ -30,8 +30,10 @@
  *     device-resident, contiguous, 16-byte aligned (fp32 LSE rows: 4-byte).
  *     Raster-order tensors hold the latent's N = L_t * L_h * L_w tokens;
  *     tile-major tensors hold whole tiles, N_tiles = n_t n_h n_w * tile volume
- *     rows (equal to N when every axis is a multiple of the tile), with zero
- *     padding rows as sta_tile_reorder writes them.
+ *     rows (equal to N when every axis is a multiple of the tile).  Tile-major
+ *     inputs have zero padding rows, as sta_tile_reorder writes them; in
+ *     tile-major outputs (o, lse, dq, dk, dv) the padding rows are unspecified:
+ *     a 128-row block of padding rows only is not computed at all.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Device work
  *     is enqueued asynchronously on it; nothing here synchronises except
  *     sta_plan, sta_plan_destroy and sta_last_device_status.
@@ -92,7 +94,8 @@ typedef struct sta_plan_s* sta_plan_t;
  * (b, h, query row block) items in descending order of list length, the
  * backward's one-block work lists (ordered for a persistent grid of one CTA
  * per SM), the raster origin of every tile, and for padded latents the real-key
- * mask of every 128-key chunk.  Allocates device memory; free it with
+ * mask of every 128-key chunk.  The work lists hold only row blocks with at
+ * least one real token.  Allocates device memory; free it with
  * sta_plan_destroy.  Errors: INVALID_ARG, UNSUPPORTED (tile volume not a
  * multiple of 128 tokens, or more than 2^31 - 1 tile-major rows), OOM, CUDA.
  *
@@ -136,14 +139,16 @@ STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, in
 
 /* Copy the plan's work list to host memory, four int32 per item:
  * (b * heads + h, first 128-row query block, second block or -1, window id).
- * Row block r covers tile-major rows [128 r, 128 r + 128) of its head.  Writes
+ * Row block r covers tile-major rows [128 r, 128 r + 128) of its head; every
+ * block holding a real token appears once, blocks of padding rows only never.  Writes
  * min(count, cap) items and the full count to *count.  For tests/inspection. */
 STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
 
 /* Copy one of the backward's work lists to host memory, four int32 per item:
  * (b * heads + h, 128-row block, -1, window id); which = 0: the dQ kernel's
  * query blocks, 1: the dK / dV kernel's key blocks.  Each lists every block
- * of every (b, h) once, ordered for a persistent grid of one CTA per SM.
+ * of every (b, h) that holds a real token once, ordered for a persistent grid
+ * of one CTA per SM.
  * Writes min(count, cap) items and the full count.  For tests/inspection. */
 STA_API sta_status sta_plan_backward_items(sta_plan_t p, int32_t which, int32_t* items4, int64_t cap,
                                            int64_t* count);

@@ -201,22 +201,36 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
         }
     }
 
+    // Row blocks holding at least one real token (all of them unless the
+    // latent is padded: a block of padding rows only has no output and no
+    // keys, and is left out of every work list).
+    const int32_t S = P.sub_per_tile;
+    std::vector<uint8_t> real_block(size_t(P.tiles_per_head) * S, 1);
+    if (P.padded)
+        for (size_t blk = 0; blk < real_block.size(); ++blk) {
+            const uint32_t* m = &P.key_mask[blk * 4];
+            real_block[blk] = (m[0] | m[1] | m[2] | m[3]) != 0u;
+        }
+
     // Work items.  Row blocks of one tile are paired so the pair shares K/V
     // loads; with an odd count per tile, the last block of consecutive tiles
     // are paired instead (each with its own list, same length).
-    const int32_t S = P.sub_per_tile;
     P.items.clear();
     P.computed_pairs = 0;
+    std::vector<int32_t> real;
     for (int32_t b = 0; b < batch; ++b)
         for (int32_t h = 0; h < heads; ++h) {
             const int32_t bh = b * heads + h, win = P.head_win[h];
             P.computed_pairs += int64_t(P.tiles_per_head) * list_len[win];
             int32_t pending = -1;
             for (int32_t t = 0; t < P.tiles_per_head; ++t) {
-                for (int32_t s = 0; s + 1 < S; s += 2)
-                    P.items.push_back(WorkItem{bh, t * S + s, t * S + s + 1, win});
-                if (S % 2 == 1) {
-                    const int32_t blk = t * S + S - 1;
+                real.clear();
+                for (int32_t s = 0; s < S; ++s)
+                    if (real_block[size_t(t) * S + s]) real.push_back(t * S + s);
+                const size_t n_real = real.size();
+                for (size_t i = 0; i + 1 < n_real; i += 2) P.items.push_back(WorkItem{bh, real[i], real[i + 1], win});
+                if (n_real % 2 == 1) {
+                    const int32_t blk = real[n_real - 1];
                     if (pending < 0) {
                         pending = blk;
                     } else {
@@ -255,6 +269,7 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
         for (int32_t h = 0; h < heads; ++h) {
             const int32_t bh = b * heads + h, win = P.head_win[h];
             for (int32_t blk = 0; blk < tph * S; ++blk) {
+                if (!real_block[size_t(blk)]) continue;  // padding rows only: no dQ, dK, dV to write
                 P.bq_items.push_back(WorkItem{bh, blk, -1, win});
                 P.bkv_items.push_back(WorkItem{bh, blk, -1, win});
             }

@@ -193,9 +193,13 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const uint4* __restrict__
     const int64_t row = t / kTpr;
     const int part = int(t % kTpr);
     int64_t src = row;
-    if (kRaster && row < rows) {
+    if ((kRaster || kPadded) && row < rows) {
+        // raster layout: the row's raster position; padded latents: -1 for a
+        // padding row, whose O and LSE rows may be unwritten (the forward skips
+        // blocks of padding rows only) and which gets 0 in both planes
         const int32_t bh = int32_t(row / tokens), within = int32_t(row % tokens);
-        src = raster_row<kPadded>(rg, bh, within / 128, within % 128);
+        const int64_t r = raster_row<kPadded>(rg, bh, within / 128, within % 128);
+        src = kRaster ? r : (r < 0 ? -1 : row);
     }
     float acc = 0.0f;
     if (row < rows && src >= 0) {
@@ -886,9 +890,17 @@ cudaError_t launch_bwd_variant(const sta_plan_s* pl, const CUtensorMap& mq, cons
     {
         const int64_t threads = rows * (D / 8);
         const int64_t blocks = (threads + 255) / 256;
-        bwd_prep_kernel<D, kRaster, kPadded><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
-            static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, ws, ws + rows, rows, bp.tokens,
-            bp.rg);
+        // Tile-major tensors of a padded latent: the row pass writes 0 for
+        // padding rows instead of reading them (the main kernels need no mask:
+        // padding rows of K, V and dO are zero).
+        if (!kRaster && P.padded)
+            bwd_prep_kernel<D, false, true><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
+                static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, ws, ws + rows, rows, bp.tokens,
+                bp.rg);
+        else
+            bwd_prep_kernel<D, kRaster, kPadded><<<dim3(uint32_t(blocks)), 256, 0, stream>>>(
+                static_cast<const uint4*>(o), static_cast<const uint4*>(dout), lse, ws, ws + rows, rows, bp.tokens,
+                bp.rg);
         if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return e;
     }
     // dQ

@@ -4,7 +4,8 @@
 - argument validation happens before any launch;
 - the plan's key-tile lists equal the sets derived from the oracle's
   token-level mask (bit-exact), for every workload geometry and window;
-- the work list covers every (b, h, 128-row block) exactly once.
+- the work list covers every (b, h, 128-row block) holding a real token
+  exactly once (blocks of padding rows only are left out).
 """
 import ctypes
 import os
@@ -138,10 +139,18 @@ def test_plan_lists_match_oracle_mask(idx):
     assert items >= w.batch * w.heads * n_tiles * (vol // 128) // 2
 
 
+def real_blocks(latent, tile):
+    """Tile-major 128-row blocks holding at least one real token, read off the
+    oracle's tile-major positions of the latent's tokens."""
+    N = latent[0] * latent[1] * latent[2]
+    return sorted(set((oracle.tile_major_index(latent, tile, np.arange(N)) // 128).tolist()))
+
+
 def test_work_list_covers_every_row_block_once():
     for latent, tile, heads, batch in [((18, 24, 24), (6, 8, 8), 2, 1), ((12, 16, 16), (4, 8, 8), 3, 2),
                                        ((6, 16, 16), (2, 8, 8), 1, 1), ((30, 48, 80), (6, 8, 8), 24, 1),
-                                       ((18, 24, 16), (6, 8, 8), 2, 2)]:
+                                       ((18, 24, 16), (6, 8, 8), 2, 2), ((33, 45, 80), (6, 8, 8), 3, 1),
+                                       ((13, 21, 18), (6, 8, 8), 2, 2), ((1, 1, 1), (6, 8, 8), 1, 2)]:
         wins = [tuple(3 * t for t in tile)] * (heads - 1) + [tile]
         p = sta.sta_plan_host(latent, tile, batch, heads, wins)
         items = p.work_items()
@@ -160,7 +169,8 @@ def test_work_list_covers_every_row_block_once():
             lens.append(len(p.query(h, qa // S)))
             if qb >= 0:
                 assert len(p.query(h, qb // S)) == lens[-1]
-        assert len(seen) == batch * heads * n_tiles * S
+        real = real_blocks(latent, tile)
+        assert sorted(seen) == [(bh, r) for bh in range(batch * heads) for r in real]
         assert all(c == 1 for c in seen.values())
         assert lens == sorted(lens, reverse=True)  # longest lists first
         pairs, n_items = p.stats()
@@ -258,22 +268,24 @@ def test_pipe_rejected_before_allocation():
     ((30, 48, 80), (6, 8, 8), 24, 1, None),
     ((18, 24, 24), (6, 8, 8), 3, 2, [(6, 8, 8), (12, 16, 16), (18, 24, 24)]),
     ((13, 21, 18), (6, 8, 8), 2, 1, [(6, 8, 8), (18, 24, 24)]),
+    ((33, 45, 80), (6, 8, 8), 24, 1, None),
 ])
 def test_backward_work_lists(latent, tile, heads, batch, wins):
-    """Each backward list holds every (b, h, block) once; rounds of 148 items
+    """Each backward list holds every (b, h, block) with a real token once
+    (blocks of padding rows only are left out); rounds of 148 items
     (one per CTA of the host plan's grid) keep natural (b, h, block) order
     between rounds, and per-CTA totals of list lengths stay level."""
     wins = wins or [(18, 24, 24)] * heads
     p = sta.sta_plan_host(latent, tile, batch, heads, wins)
     S = (tile[0] * tile[1] * tile[2]) // 128
-    n_blocks = p.tiles_per_head * S
+    real = real_blocks(latent, tile)
     for which in (0, 1):
         items = p.backward_items(which)
         assert all(qb == -1 for _, _, qb, _ in items)
         keys = sorted((bh, blk) for bh, blk, _, _ in items)
-        assert keys == [(bh, blk) for bh in range(batch * heads) for blk in range(n_blocks)]
+        natural = [(bh, blk) for bh in range(batch * heads) for blk in real]
+        assert keys == natural
         R = 148
-        natural = [(bh, blk) for bh in range(batch * heads) for blk in range(n_blocks)]
         for r0 in range(0, len(items), R):
             assert sorted((bh, blk) for bh, blk, _, _ in items[r0:r0 + R]) == natural[r0:r0 + R]
         def length(it):

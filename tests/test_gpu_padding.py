@@ -155,3 +155,42 @@ def test_hunyuan_720p_latent_sampled(sta):
     og = o.reshape(-1, o.shape[2], d)[rows[:, 0], rows[:, 1]].cpu()
     lg = lse.reshape(-1, lse.shape[2])[rows[:, 0], rows[:, 1]].cpu()
     compare(og, lg, o_ref, lse_ref, what="33x45x80")
+
+
+def test_padding_blocks_skipped_and_backward_ignores_their_rows(sta):
+    """A block of padding rows only is not computed: tile-major O and LSE
+    prefilled with NaN keep NaN there, every real row equals the raster
+    forward, and the tile-major backward fed those very outputs (NaN rows
+    included) gives the raster backward's bits: its row pass writes 0 for
+    padding rows instead of reading them."""
+    latent, tile, B, H, d = (9, 16, 16), (6, 8, 8), 1, 2, 128  # t: 9 = 6 + 3, so t 10-11 is one padding block
+    windows = [[6, 8, 8], [12, 16, 16]]
+    q, k, v, do = (x.cuda() for x in inputs(latent, B, H, d, seed=916))
+    scale = 1.0 / np.sqrt(d)
+    plan = sta.sta_plan(latent, tile, B, H, windows)
+    Np = plan.padded_tokens
+    qt, kt, vt, dot = (torch.empty((B, H, Np, d), dtype=torch.bfloat16, device="cuda") for _ in range(4))
+    for x, y in ((q, qt), (k, kt), (v, vt), (do, dot)):
+        sta.sta_tile_reorder(x, y, latent, tile)
+    ot = torch.full((B, H, Np, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lt = torch.full((B, H, Np), float("nan"), dtype=torch.float32, device="cuda")
+    sta.sta_forward(plan, qt, kt, vt, ot, lt, scale)
+    o, lse = sta.sta_attention(q, k, v, plan, scale)
+    o_back, lse_back = torch.empty_like(o), torch.empty_like(lse)
+    sta.sta_tile_unreorder(ot, o_back, latent, tile)
+    sta.sta_tile_unreorder(lt, lse_back, latent, tile)
+    assert torch.equal(o_back, o) and torch.equal(lse_back, lse)
+    N = latent[0] * latent[1] * latent[2]
+    real = set((oracle.tile_major_index(latent, tile, np.arange(N)) // 128).tolist())
+    skipped = [b for b in range(Np // 128) if b not in real]
+    assert skipped, "the geometry must have a block of padding rows only"
+    for b in skipped:
+        assert bool(torch.isnan(ot[:, :, 128 * b:128 * (b + 1)].float()).all())
+        assert bool(torch.isnan(lt[:, :, 128 * b:128 * (b + 1)]).all())
+    dq, dk, dv = sta.sta_backward(plan, qt, kt, vt, ot, lt, dot, scale)
+    ref = sta.sta_attention_backward(q, k, v, o, lse, do, plan, scale)
+    for x, r in zip((dq, dk, dv), ref):
+        back = torch.empty_like(r)
+        sta.sta_tile_unreorder(x, back, latent, tile)
+        assert torch.equal(back, r)
+    assert sta.sta_last_device_status(plan) == 0
