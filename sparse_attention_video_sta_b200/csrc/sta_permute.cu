@@ -123,9 +123,9 @@ cudaError_t launch_typed(const void* src, void* dst, int64_t outer, int32_t row_
         while ((1 << shift) < vpr) ++shift;
     }
     const int64_t blocks = outer * g.tiles;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int dev = 0, sms = 0;
+    if (cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return e;
+    if (cudaError_t e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev); e != cudaSuccess) return e;
     const int64_t cap = int64_t(sms) * 16;
     const unsigned grid = unsigned(blocks < cap ? blocks : cap);
     if (g.tile_tokens <= kMaxTableTokens) {
