@@ -147,6 +147,18 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(int(stream))
 
 
+def _device(tensors, plan=None) -> torch.device:
+    """The one CUDA device of ``tensors`` (and of ``plan``, when it has one).
+    Calls into the library run with it current, so the library's device
+    checks and the default stream refer to the tensors' device."""
+    idx = {t.device.index for t in tensors if t is not None and t.is_cuda}
+    if plan is not None and plan.device is not None:
+        idx.add(plan.device)
+    if len(idx) != 1:
+        raise ValueError(f"tensors and plan must be on one CUDA device (got devices {sorted(idx)})")
+    return torch.device("cuda", idx.pop())
+
+
 def _windows(heads: int, windows) -> ctypes.Array:
     w = torch.as_tensor(windows, dtype=torch.int32).reshape(-1, 3)
     if w.shape[0] == 1 and heads > 1:
@@ -160,8 +172,9 @@ def _windows(heads: int, windows) -> ctypes.Array:
 class Plan:
     """Owner of a ``sta_plan_t`` handle (freed on ``destroy`` / garbage collection)."""
 
-    def __init__(self, handle: int, latent, tile, batch: int, heads: int, windows):
+    def __init__(self, handle: int, latent, tile, batch: int, heads: int, windows, device: int | None = None):
         self._h = ctypes.c_void_p(handle)
+        self.device = device  # CUDA device index of a device plan; None for a host-only plan
         self.latent = tuple(int(x) for x in latent)
         self.tile = tuple(int(x) for x in tile)
         self.batch = int(batch)
@@ -268,9 +281,10 @@ def sta_plan(latent, tile, batch: int, heads: int, windows, stream=None) -> Plan
     """Build a plan on the current CUDA device (windows: ``[heads, 3]`` tokens)."""
     h = ctypes.c_void_p(0)
     g = _geom(latent, tile)
+    dev = torch.cuda.current_device()
     _check(_lib.sta_plan(ctypes.byref(g), int(batch), int(heads), _windows(heads, windows),
                          _stream(stream), ctypes.byref(h)), "sta_plan")
-    return Plan(h.value, latent, tile, batch, heads, windows)
+    return Plan(h.value, latent, tile, batch, heads, windows, device=dev)
 
 
 def sta_plan_host(latent, tile, batch: int, heads: int, windows) -> Plan:
@@ -319,9 +333,10 @@ def sta_tile_reorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token_d
     N = latent[0] * latent[1] * latent[2]
     outer, row_bytes = _perm_args(src, dst, N, token_dim, N, _padded_tokens(latent, tile))
     g = _geom(latent, tile)
-    _check(_lib.sta_tile_reorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
-                                 outer, row_bytes, ctypes.byref(g), _stream(stream)),
-           "sta_tile_reorder")
+    with torch.cuda.device(_device((src, dst))):
+        _check(_lib.sta_tile_reorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
+                                     outer, row_bytes, ctypes.byref(g), _stream(stream)),
+               "sta_tile_reorder")
     return dst
 
 
@@ -332,9 +347,10 @@ def sta_tile_unreorder(src: torch.Tensor, dst: torch.Tensor, latent, tile, token
     N = latent[0] * latent[1] * latent[2]
     outer, row_bytes = _perm_args(src, dst, N, token_dim, _padded_tokens(latent, tile), N)
     g = _geom(latent, tile)
-    _check(_lib.sta_tile_unreorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
-                                   outer, row_bytes, ctypes.byref(g), _stream(stream)),
-           "sta_tile_unreorder")
+    with torch.cuda.device(_device((src, dst))):
+        _check(_lib.sta_tile_unreorder(ctypes.c_void_p(src.data_ptr()), ctypes.c_void_p(dst.data_ptr()),
+                                       outer, row_bytes, ctypes.byref(g), _stream(stream)),
+               "sta_tile_unreorder")
     return dst
 
 
@@ -360,7 +376,8 @@ def sta_forward(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                 o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
     """STA forward on tile-major ``[B, H, N, d]`` bf16 tensors; writes ``o`` and ``lse``."""
     args = _forward_args(plan, q, k, v, o, lse)
-    _check(_lib.sta_forward(plan.handle, *args, float(softmax_scale), _stream(stream)), "sta_forward")
+    with torch.cuda.device(_device((q, k, v, o, lse), plan)):
+        _check(_lib.sta_forward(plan.handle, *args, float(softmax_scale), _stream(stream)), "sta_forward")
     return o, lse
 
 
@@ -368,8 +385,9 @@ def sta_forward_raster(plan: Plan, q: torch.Tensor, k: torch.Tensor, v: torch.Te
                        o: torch.Tensor, lse: torch.Tensor, softmax_scale: float, stream=None):
     """STA forward on raster-order ``[B, H, N, d]`` bf16 tensors (permutation fused)."""
     args = _forward_args(plan, q, k, v, o, lse, raster=True)
-    _check(_lib.sta_forward_raster(plan.handle, *args, float(softmax_scale), _stream(stream)),
-           "sta_forward_raster")
+    with torch.cuda.device(_device((q, k, v, o, lse), plan)):
+        _check(_lib.sta_forward_raster(plan.handle, *args, float(softmax_scale), _stream(stream)),
+               "sta_forward_raster")
     return o, lse
 
 
@@ -390,9 +408,10 @@ def _backward_call(fn, what: str, plan: Plan, q, k, v, o, lse, dout, softmax_sca
             or workspace.numel() < n_ws:
         raise ValueError(f"workspace must be a contiguous CUDA fp32 tensor of {n_ws} floats")
     qp, kp, vp_, op, lp, hd = args
-    _check(fn(plan.handle, qp, kp, vp_, op, ctypes.c_void_p(dout.data_ptr()), lp,
-              ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()), ctypes.c_void_p(dv.data_ptr()),
-              ctypes.c_void_p(workspace.data_ptr()), hd, float(softmax_scale), _stream(stream)), what)
+    with torch.cuda.device(_device((q, k, v, o, lse, dout, dq, dk, dv, workspace), plan)):
+        _check(fn(plan.handle, qp, kp, vp_, op, ctypes.c_void_p(dout.data_ptr()), lp,
+                  ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()), ctypes.c_void_p(dv.data_ptr()),
+                  ctypes.c_void_p(workspace.data_ptr()), hd, float(softmax_scale), _stream(stream)), what)
     return dq, dk, dv
 
 
@@ -446,17 +465,21 @@ def sta_forward_noalloc(latent, tile, batch: int, heads: int, windows, q: torch.
             or tuple(lse.shape) != (B, H, N):
         raise ValueError(f"lse must be a contiguous CUDA fp32 tensor of shape [{B}, {H}, {N}]")
     g = _geom(latent, tile)
-    _check(_lib.sta_forward_noalloc(ctypes.byref(g), B, H, _windows(H, windows),
-                                    ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                    ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
-                                    ctypes.c_void_p(lse.data_ptr()), int(q.shape[3]),
-                                    float(softmax_scale), _stream(stream)), "sta_forward_noalloc")
+    with torch.cuda.device(_device((q, k, v, o, lse))):
+        _check(_lib.sta_forward_noalloc(ctypes.byref(g), B, H, _windows(H, windows),
+                                        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                        ctypes.c_void_p(lse.data_ptr()), int(q.shape[3]),
+                                        float(softmax_scale), _stream(stream)), "sta_forward_noalloc")
     return o, lse
 
 
 def sta_last_device_status(plan: Plan, stream=None) -> int:
     """Synchronise and return (clearing it) the plan's device status code."""
-    return int(_lib.sta_last_device_status(plan.handle, _stream(stream)))
+    if plan.device is None:
+        return int(_lib.sta_last_device_status(plan.handle, None))  # host-only plan: INVALID_ARG
+    with torch.cuda.device(plan.device):
+        return int(_lib.sta_last_device_status(plan.handle, _stream(stream)))
 
 
 def sta_debug_inject_timeout(enable: bool, limit_ms: int = 50) -> None:
@@ -555,12 +578,14 @@ def sta_window_stats(lse_w: torch.Tensor, lse_full: torch.Tensor, o_w: torch.Ten
         if not t.is_cuda or t.dtype != dt or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA {dt} tensor")
     B, H, N, d = o_w.shape
-    recall = torch.empty((B, H), dtype=torch.float64, device=o_w.device)
+    dev = _device((lse_w, lse_full, o_w, o_full))
+    recall = torch.empty((B, H), dtype=torch.float64, device=dev)
     mse = torch.empty_like(recall)
-    _check(_lib.sta_window_stats(ctypes.c_void_p(lse_w.data_ptr()), ctypes.c_void_p(lse_full.data_ptr()),
-                                 ctypes.c_void_p(o_w.data_ptr()), ctypes.c_void_p(o_full.data_ptr()),
-                                 B * H, N, d, ctypes.c_void_p(recall.data_ptr()),
-                                 ctypes.c_void_p(mse.data_ptr()), _stream(stream)), "sta_window_stats")
+    with torch.cuda.device(dev):
+        _check(_lib.sta_window_stats(ctypes.c_void_p(lse_w.data_ptr()), ctypes.c_void_p(lse_full.data_ptr()),
+                                     ctypes.c_void_p(o_w.data_ptr()), ctypes.c_void_p(o_full.data_ptr()),
+                                     B * H, N, d, ctypes.c_void_p(recall.data_ptr()),
+                                     ctypes.c_void_p(mse.data_ptr()), _stream(stream)), "sta_window_stats")
     return recall, mse
 
 
@@ -582,12 +607,15 @@ def sta_window_search(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, latent,
     B, H = int(q.shape[0]), int(q.shape[1])
     lat = tuple(int(x) for x in latent)
     cands = [tuple(int(x) for x in c) for c in candidates]
-    full = sta_plan(lat, tile, B, H, [lat] * H, stream=stream)
+    dev = _device((q, k, v))
+    with torch.cuda.device(dev):  # plans live on the inputs' device
+        full = sta_plan(lat, tile, B, H, [lat] * H, stream=stream)
     o_full, lse_full = sta_attention(q, k, v, full, softmax_scale, stream=stream)
-    n = [lat[i] // int(tile[i]) for i in range(3)]
+    n = [-(-lat[i] // int(tile[i])) for i in range(3)]  # tiles per axis (padded latents: whole tiles)
     tiles, rec, err = [], [], []
     for c in cands:
-        plan = sta_plan(lat, tile, B, H, [c] * H, stream=stream)
+        with torch.cuda.device(dev):
+            plan = sta_plan(lat, tile, B, H, [c] * H, stream=stream)
         o_c, lse_c = sta_attention(q, k, v, plan, softmax_scale, stream=stream)
         r, m = sta_window_stats(lse_c, lse_full, o_c, o_full, stream=stream)
         rec.append(r.mean(dim=0))
@@ -631,12 +659,14 @@ class Pipe:
                 raise ValueError(f"{name} must be a contiguous host {dt} tensor of shape {shape}")
             if not t.is_pinned():
                 raise ValueError(f"{name} must be in pinned host memory (tensor.pin_memory())")
-        _check(_lib.sta_pipe_submit(self._h, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
-                                    ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
-                                    ctypes.c_void_p(lse.data_ptr())), "sta_pipe_submit")
+        with torch.cuda.device(self.plan.device):
+            _check(_lib.sta_pipe_submit(self._h, ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                                        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(o.data_ptr()),
+                                        ctypes.c_void_p(lse.data_ptr())), "sta_pipe_submit")
 
     def wait(self) -> None:
-        _check(_lib.sta_pipe_wait(self._h), "sta_pipe_wait")
+        with torch.cuda.device(self.plan.device):
+            _check(_lib.sta_pipe_wait(self._h), "sta_pipe_wait")
 
     def destroy(self) -> None:
         if self._h:
@@ -653,10 +683,13 @@ class Pipe:
 
 
 def sta_pipe_create(plan: Plan, head_dim: int, softmax_scale: float | None = None, depth: int = 2) -> Pipe:
-    """Pipeline of ``depth`` device buffer sets for ``plan`` on the current device."""
+    """Pipeline of ``depth`` device buffer sets for ``plan``, on the plan's device."""
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(head_dim)
+    if plan.device is None:
+        raise ValueError("sta_pipe_create needs a device plan (sta_plan), not a host-only one")
     h = ctypes.c_void_p(0)
-    _check(_lib.sta_pipe_create(plan.handle, int(head_dim), float(softmax_scale), int(depth), ctypes.byref(h)),
-           "sta_pipe_create")
+    with torch.cuda.device(plan.device):
+        _check(_lib.sta_pipe_create(plan.handle, int(head_dim), float(softmax_scale), int(depth), ctypes.byref(h)),
+               "sta_pipe_create")
     return Pipe(h.value, plan, head_dim)

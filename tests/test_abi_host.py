@@ -349,3 +349,17 @@ def test_empty_problems_are_no_ops():
                                    ctypes.c_float(0.088), None) == INV
     assert lib.sta_forward_noalloc(ctypes.byref(g), 1, 1, w, None, None, None, None, None, 128,
                                    ctypes.c_float(0.088), None) == INV
+
+
+def test_device_helper_requires_one_cuda_device():
+    """The binding's device check (no GPU needed): host tensors alone name no
+    CUDA device; a plan's device is used when no tensor is given."""
+    import torch
+    with pytest.raises(ValueError, match="one CUDA device"):
+        sta._device((torch.zeros(1),))
+    p = sta.sta_plan_host((18, 24, 24), (6, 8, 8), 1, 1, [(12, 16, 16)])
+    assert p.device is None
+    p.device = 3
+    assert sta._device((), p) == torch.device("cuda", 3)
+    p.device = None
+    p.destroy()

@@ -86,3 +86,25 @@ def test_graph_capture_replays_forward_and_backward(sta):
         for a, b in ((o_g, o), (lse_g, lse), (dq_g, dq), (dk_g, dk), (dv_g, dv)):
             assert torch.equal(a, b), seed
     del graph
+
+
+def test_tensors_on_another_device_than_the_plan_are_rejected(sta):
+    """The binding runs every call on the device of its tensors and its plan,
+    and refuses a mismatch before any launch (checked here by marking the plan
+    as another device's: nothing reaches the library or that device)."""
+    w = sta_inputs.WORKLOADS[1]
+    plan = sta.sta_plan(w.latent, w.tile, w.batch, w.heads, sta_inputs.windows(w).tolist())
+    assert plan.device == torch.cuda.current_device()
+    q, k, v, do = _inputs(w, 3)
+    o, lse = sta.sta_attention(q, k, v, plan, w.softmax_scale)
+    real = plan.device
+    plan.device = real + 1
+    try:
+        for call in (lambda: sta.sta_attention(q, k, v, plan, w.softmax_scale),
+                     lambda: sta.sta_attention(q, k, v, plan, w.softmax_scale, fused=False),
+                     lambda: sta.sta_attention_backward(q, k, v, o, lse, do, plan, w.softmax_scale)):
+            with pytest.raises(ValueError, match="one CUDA device"):
+                call()
+    finally:
+        plan.device = real
+    assert sta.sta_last_device_status(plan) == 0
