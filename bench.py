@@ -546,7 +546,7 @@ def main():
             "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tflops / peak, "traffic": measured_traffic(w.name),
-                         "kernel": f"sta_fwd_kernel<{d}, raster>",
+                         "kernel": f"sta_fwd_split_kernel<{d}, raster>",
                          "peak_source": f"bf16_tflops_sustained ({peak_kind})",
                          "frac_of_burst": fwd_tflops / float(peaks.get("bf16_tflops", 1590.0))},
             "gpu_launches": launches_per_step * args.steps,

@@ -245,6 +245,16 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
     std::stable_sort(P.items.begin(), P.items.end(), [&](const WorkItem& a, const WorkItem& b) {
         return list_len[a.win] > list_len[b.win];
     });
+    // One-block items (the key-split forward kernel): every real row block,
+    // in (head, block) order, longest lists first.
+    P.f1_items.clear();
+    for (int32_t b = 0; b < batch; ++b)
+        for (int32_t h = 0; h < heads; ++h)
+            for (int32_t blk = 0; blk < P.tiles_per_head * S; ++blk)
+                if (real_block[size_t(blk)]) P.f1_items.push_back(WorkItem{b * heads + h, blk, -1, P.head_win[h]});
+    std::stable_sort(P.f1_items.begin(), P.f1_items.end(), [&](const WorkItem& a, const WorkItem& b) {
+        return list_len[a.win] > list_len[b.win];
+    });
 
     // Backward: transposed lists (query tiles ascending for each key tile).
     const int32_t tph = P.tiles_per_head;
@@ -289,6 +299,8 @@ void free_device(sta_plan_s* p) {
     if (p->d_off) cudaFree(p->d_off);
     if (p->d_ids) cudaFree(p->d_ids);
     if (p->d_items) cudaFree(p->d_items);
+    if (p->d_f1_items) cudaFree(p->d_f1_items);
+    p->d_f1_items = nullptr;
     if (p->d_status) cudaFree(p->d_status);
     if (p->d_origin) cudaFree(p->d_origin);
     if (p->d_kmask) cudaFree(p->d_kmask);
@@ -444,6 +456,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     if (e == cudaSuccess) e = upload(&p->d_off, p->h.csr_off, s);
     if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
     if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
+    if (e == cudaSuccess) e = upload(&p->d_f1_items, p->h.f1_items, s);
     if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
     if (e == cudaSuccess && p->h.padded) e = upload(&p->d_kmask, p->h.key_mask, s);
     if (e == cudaSuccess)
@@ -470,7 +483,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_status || p->d_origin || p->d_kmask ||
+    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_f1_items || p->d_status || p->d_origin || p->d_kmask ||
         p->d_counters || p->d_toff ||
         p->d_tids || p->d_bq_items || p->d_bkv_items) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;

@@ -43,7 +43,8 @@ struct PlanHost {
     std::vector<int32_t> win_ext;            // [n_win][3] clamped extents in tiles
     std::vector<int32_t> csr_off;            // [n_win][tiles_per_head + 1], global offsets
     std::vector<int32_t> csr_ids;            // key-tile ids, ascending per list
-    std::vector<WorkItem> items;             // forward work list
+    std::vector<WorkItem> items;             // forward work list (two-block items)
+    std::vector<WorkItem> f1_items;          // forward work list of one-block items, longest lists first
     // Backward: for each key tile the query tiles whose window holds it
     // (the forward lists transposed), and one-block work lists for the dQ
     // kernel (qa = query block) and the dK/dV kernel (qa = key block).
@@ -66,6 +67,7 @@ struct sta_plan_s {
     int32_t* d_off = nullptr;
     int32_t* d_ids = nullptr;
     sta::WorkItem* d_items = nullptr;
+    sta::WorkItem* d_f1_items = nullptr;
     uint32_t* d_status = nullptr;
     int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
     uint32_t* d_kmask = nullptr;  // device copy of key_mask (padded latents only)
