@@ -475,7 +475,7 @@ def main():
             extras["padded_latent"] = {"latent": list(pl), "padded_to": [-(-pl[i] // T[i]) * T[i] for i in range(3)],
                                        "ms": p_ms, "tflops_tile_pairs": pplan.flops(d) / (p_ms * 1e-3) / 1e12,
                                        "tflops_useful": (p_useful / (p_ms * 1e-3) / 1e12) if p_useful else None,
-                                       "kernel": f"sta_fwd_kernel<{d}, raster, padded>"}
+                                       "kernel": f"sta_fwd_split_kernel<{d}, raster, padded>"}
             pplan.destroy()
             del pq, pk_, pv, po, plse
         # ------------------------------------------- unfused pipeline

@@ -142,10 +142,10 @@ STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, in
  * Row block r covers tile-major rows [128 r, 128 r + 128) of its head; every
  * block holding a real token appears once, blocks of padding rows only never.  Writes
  * min(count, cap) items and the full count to *count.  For tests/inspection.
- * The forward runs this list on padded latents; on latents that are a
- * multiple of the tile it runs the same blocks one per item (longest key
- * lists first), each block's 128-key chunks split between two softmax
- * warpgroups. */
+ * sta_forward_noalloc runs two-block items like these (built in its own
+ * scratch); sta_forward and sta_forward_raster run the same blocks one per
+ * item (longest key lists first), each block's 128-key chunks split between
+ * two softmax warpgroups. */
 STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
 
 /* Copy one of the backward's work lists to host memory, four int32 per item:

@@ -11,12 +11,13 @@
 // split but are built for Blackwell.  Two kernels share the roles and the
 // helpers:
 //
-//   sta_fwd_split_kernel (latents that are a multiple of the tile): one
-//   128-row query block per work item, every 128-key chunk split between two
-//   softmax warpgroups, S double buffered in TMEM; see its own comment.
+//   sta_fwd_split_kernel (sta_forward, sta_forward_raster): one 128-row query
+//   block per work item, every 128-key chunk split between two softmax
+//   warpgroups, S double buffered in TMEM; see its own comment.
 //
-//   sta_fwd_kernel (padded latents, with per-chunk key masks; also the
-//   allocation-free entry point):
+//   sta_fwd_kernel (the allocation-free entry point, whose plan lives in a
+//   fixed scratch array; its padded-latent and raster branches are kept for
+//   comparison but not instantiated):
 //   warp 8 (load)      : TMA loads of the query blocks and of the 128-key K / V
 //                        chunks of the listed key tiles into a ring of stages
 //   warps 9, 10 (MMA)  : one thread each, for query slot 0 / 1, issues
@@ -210,6 +211,14 @@ __device__ __forceinline__ float row_max(const uint32_t (&sr)[128]) {
     a0 = ptx::max3(a0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
     a1 = ptx::max3(a1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
     return ptx::max3(a0, a1, fmaxf(a2, a3));
+}
+
+// The same for one 64-score half row (key-split kernel): `lo`, `hi` hold the
+// real-key bits of the half's 64 keys.
+__device__ __forceinline__ void mask_scores64(uint32_t (&sr)[64], uint32_t lo, uint32_t hi) {
+#pragma unroll
+    for (int j = 0; j < 64; ++j)
+        if (!(((j < 32 ? lo : hi) >> (j & 31)) & 1u)) sr[j] = 0xff800000u;
 }
 
 // The same for one 64-score half row (key-split kernel).
@@ -679,7 +688,7 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 }
 
 // ---------------------------------------------------------------------------
-// Key-split forward kernel (latents that are a multiple of the tile).
+// Key-split forward kernel.
 //
 // One work item is one 128-row query block.  Every 128-key chunk is split in
 // two halves of 64 keys: softmax warpgroup A (warps 0-3) owns keys 0-63 of each
@@ -704,7 +713,10 @@ sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // TMEM (512 columns): S0 | S1 | O_A | O_B (d = 128).  P_A (bf16) is written
 // over the first 32 columns of its half of S, P_B over the first 32 of its.
 // The epilogue exchanges the halves' running max and sum through the query
-// buffer of the finished block.  The two-slot kernel's ping-pong needed the
+// buffer of the finished block.  Padded latents (kPadded): each half masks
+// its padding keys from the chunk's real-key bits, and a half that meets no
+// real key in the whole block (a block whose key tiles are all edge tiles)
+// keeps l = 0 and drops out of the merge.  The two-slot kernel's ping-pong needed the
 // chain [PV, S] batch -> softmax -> P to fit in two batches; here the softmax
 // of chunk g + 1 only needs S(g + 1), issued a chunk earlier.
 namespace split {
@@ -732,7 +744,9 @@ struct Cfg {
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
-template <int D, bool kRaster>
+// kPadded: the latent has padding tokens; padding keys are masked per chunk
+// and raster padding rows are not stored.
+template <int D, bool kRaster, bool kPadded>
 __global__ void __launch_bounds__(kThreads, 1)
 sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -991,6 +1005,7 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int32_t tile_q = w.qa / SPT;
             const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
             const uint32_t n = uint32_t(off[tile_q + 1] - off[tile_q]) * uint32_t(SPT);
+            const int32_t kbeg = off[tile_q];  // this block's key tiles (padded latents: their masks)
             float m_used = 0.0f, l = 0.0f;
             for (uint32_t i = 0; i < n; ++i, ++g) {
                 const uint32_t b = g & 1u;
@@ -1001,12 +1016,24 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 ptx::tc_fence_after();
                 const uint32_t tS = tmem + lane_addr + C::col_s(int(b)) + uint32_t(half) * 64u;
                 uint32_t sr[64];
+                uint32_t mlo = ~0u, mhi = ~0u;  // real-key bits of this half's 64 keys
+                if (kPadded) {
+                    const uint4 m4 = __ldg(p.key_mask + int64_t(__ldg(p.ids + kbeg + int32_t(i) / SPT)) * SPT +
+                                           int32_t(i) % SPT);
+                    mlo = half == 0 ? m4.x : m4.z;
+                    mhi = half == 0 ? m4.y : m4.w;
+                }
                 ptx::tmem_ld64(tS, sr);
+                if (kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
                 uint32_t pk[32];
                 float rowsum, alpha = 1.0f;
                 bool rescale = false;
                 if (i == 0) {
                     m_used = row_max64(sr);
+                    // Padded latents: this half of the first chunk may hold no real
+                    // key; any finite reference works, the lazy rescale below
+                    // moves it once real keys arrive.
+                    if (kPadded && m_used == -INFINITY) m_used = 0.0f;
                     rowsum = softmax_exp64(sr, c, m_used, pk);
                 } else {
                     rowsum = softmax_exp64(sr, c, m_used, pk);
@@ -1078,14 +1105,17 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const float l_o = xch[((1 - half) * 128 + row) * 2 + 1];
             const float m_a = half == 0 ? m_used : m_o, l_a = half == 0 ? l : l_o;
             const float m_b = half == 0 ? m_o : m_used, l_b = half == 0 ? l_o : l;
-            const float m = fmaxf(m_a, m_b);
-            const float a_a = ptx::ex2((m_a - m) * c), a_b = ptx::ex2((m_b - m) * c);
+            // A half that met no real key (padded latents only) has l = 0 and
+            // O = 0 and takes no part in the merge.
+            const float m = l_a == 0.0f ? m_b : (l_b == 0.0f ? m_a : fmaxf(m_a, m_b));
+            const float a_a = l_a == 0.0f ? 0.0f : ptx::ex2((m_a - m) * c);
+            const float a_b = l_b == 0.0f ? 0.0f : ptx::ex2((m_b - m) * c);
             const float l_sum = a_a * l_a + a_b * l_b;
             const float inv_l = 1.0f / l_sum;
             const uint64_t f_a = ptx::f2(a_a * inv_l, a_a * inv_l), f_b = ptx::f2(a_b * inv_l, a_b * inv_l);
-            const int64_t grow = out_row<kRaster, false>(p, w.bh, w.qa, row);
+            const int64_t grow = out_row<kRaster, kPadded>(p, w.bh, w.qa, row);
             // this warp's half of the columns: [half * D / 2, half * D / 2 + D / 2)
-            uint4* dst = reinterpret_cast<uint4*>(p.o + grow * D + half * (D / 2));
+            uint4* dst = reinterpret_cast<uint4*>(p.o + (grow < 0 ? 0 : grow) * D + half * (D / 2));
             const uint32_t tOa = tmem + lane_addr + C::col_o(0) + uint32_t(half) * (D / 2);
             const uint32_t tOb = tmem + lane_addr + C::col_o(1) + uint32_t(half) * (D / 2);
 #pragma unroll 1
@@ -1102,10 +1132,13 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     ptx::f2_split(ptx::f2_fma(va, f_a, ptx::f2_mul(vb, f_b)), o0, o1);
                     pk[j] = ptx::pack_bf16x2(o0, o1);
                 }
+                if (grow >= 0) {  // a padding row of a raster output stores nothing
 #pragma unroll
-                for (int j = 0; j < 4; ++j) dst[cb * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    for (int j = 0; j < 4; ++j)
+                        dst[cb * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                }
             }
-            if (half == 0) p.lse[grow] = m * p.scale + logf(l_sum);
+            if (half == 0 && grow >= 0) p.lse[grow] = m * p.scale + logf(l_sum);
             ptx::tc_fence_before();
             ptx::fence_proxy_async_smem();  // the exchange writes precede the next query load into this buffer
             __syncwarp();
@@ -1170,14 +1203,14 @@ cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, 
     return cudaGetLastError();
 }
 
-template <int D, bool kRaster>
+template <int D, bool kRaster, bool kPadded>
 cudaError_t launch_split_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const FwdParams& fp) {
     constexpr int kSmem = split::Cfg<D>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(split::sta_fwd_split_kernel<D, kRaster>,
+    cudaError_t e = cudaFuncSetAttribute(split::sta_fwd_split_kernel<D, kRaster, kPadded>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
-    split::sta_fwd_split_kernel<D, kRaster><<<grid, kThreads, kSmem, stream>>>(mq, mk, mv, fp);
+    split::sta_fwd_split_kernel<D, kRaster, kPadded><<<grid, kThreads, kSmem, stream>>>(mq, mk, mv, fp);
     return cudaGetLastError();
 }
 
@@ -1226,25 +1259,19 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // Latents that are a multiple of the tile run the key-split kernel over
-    // one-block items; padded latents the two-slot kernel with key masks.
-    const bool key_split = !P.padded;
-    if (key_split) {
-        fp.items = pl->d_f1_items;
-        fp.n_items = int32_t(P.f1_items.size());
-    }
+    // The key-split kernel over one-block items (with per-chunk key masks on
+    // padded latents).
+    fp.items = pl->d_f1_items;
+    fp.n_items = int32_t(P.f1_items.size());
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
     fp.item_counter = pl->d_counters + pl->launch_seq.fetch_add(1) % uint32_t(kCounterPool);
     if ((e = cudaMemsetAsync(fp.item_counter, 0, sizeof(int32_t), stream)) != cudaSuccess) return e;
-    if (key_split)
-        return raster ? launch_split_kernel<D, true>(grid, stream, mq, mk, mv, fp)
-                      : launch_split_kernel<D, false>(grid, stream, mq, mk, mv, fp);
     if (raster)
-        return P.padded ? launch_kernel<D, true, true>(grid, stream, mq, mk, mv, fp)
-                        : launch_kernel<D, true, false>(grid, stream, mq, mk, mv, fp);
-    return P.padded ? launch_kernel<D, false, true>(grid, stream, mq, mk, mv, fp)
-                    : launch_kernel<D, false, false>(grid, stream, mq, mk, mv, fp);
+        return P.padded ? launch_split_kernel<D, true, true>(grid, stream, mq, mk, mv, fp)
+                        : launch_split_kernel<D, true, false>(grid, stream, mq, mk, mv, fp);
+    return P.padded ? launch_split_kernel<D, false, true>(grid, stream, mq, mk, mv, fp)
+                    : launch_split_kernel<D, false, false>(grid, stream, mq, mk, mv, fp);
 }
 
 }  // namespace
