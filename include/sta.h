@@ -137,15 +137,13 @@ STA_API sta_status sta_plan_key_query(sta_plan_t p, int32_t head, int32_t k_tile
  * heads, and number of work items.  Either pointer may be NULL. */
 STA_API sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, int64_t* work_items);
 
-/* Copy the plan's two-block work list to host memory, four int32 per item:
- * (b * heads + h, first 128-row query block, second block or -1, window id).
- * Row block r covers tile-major rows [128 r, 128 r + 128) of its head; every
- * block holding a real token appears once, blocks of padding rows only never.  Writes
- * min(count, cap) items and the full count to *count.  For tests/inspection.
- * sta_forward_noalloc runs two-block items like these (built in its own
- * scratch); sta_forward and sta_forward_raster run the same blocks one per
- * item (longest key lists first), each block's 128-key chunks split between
- * two softmax warpgroups. */
+/* Copy the forward's work list to host memory, four int32 per item:
+ * (b * heads + h, 128-row query block, -1, window id), in the order the
+ * kernel hands the items out (longest key lists first).  Row block r covers
+ * tile-major rows [128 r, 128 r + 128) of its head; every block holding a real
+ * token appears once, blocks of padding rows only never.  Writes min(count,
+ * cap) items and the full count to *count.  For tests/inspection.  Each
+ * block's 128-key chunks are split between two softmax warpgroups. */
 STA_API sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count);
 
 /* Copy one of the backward's work lists to host memory, four int32 per item:

@@ -212,41 +212,13 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
             real_block[blk] = (m[0] | m[1] | m[2] | m[3]) != 0u;
         }
 
-    // Work items.  Row blocks of one tile are paired so the pair shares K/V
-    // loads; with an odd count per tile, the last block of consecutive tiles
-    // are paired instead (each with its own list, same length).
-    P.items.clear();
+    P.items.clear();  // two-block items: no longer built (the forward runs one-block items)
     P.computed_pairs = 0;
-    std::vector<int32_t> real;
     for (int32_t b = 0; b < batch; ++b)
-        for (int32_t h = 0; h < heads; ++h) {
-            const int32_t bh = b * heads + h, win = P.head_win[h];
-            P.computed_pairs += int64_t(P.tiles_per_head) * list_len[win];
-            int32_t pending = -1;
-            for (int32_t t = 0; t < P.tiles_per_head; ++t) {
-                real.clear();
-                for (int32_t s = 0; s < S; ++s)
-                    if (real_block[size_t(t) * S + s]) real.push_back(t * S + s);
-                const size_t n_real = real.size();
-                for (size_t i = 0; i + 1 < n_real; i += 2) P.items.push_back(WorkItem{bh, real[i], real[i + 1], win});
-                if (n_real % 2 == 1) {
-                    const int32_t blk = real[n_real - 1];
-                    if (pending < 0) {
-                        pending = blk;
-                    } else {
-                        P.items.push_back(WorkItem{bh, pending, blk, win});
-                        pending = -1;
-                    }
-                }
-            }
-            if (pending >= 0) P.items.push_back(WorkItem{bh, pending, -1, win});
-        }
-    // Longest lists first (stable: neighbouring tiles stay together for L2 reuse).
-    std::stable_sort(P.items.begin(), P.items.end(), [&](const WorkItem& a, const WorkItem& b) {
-        return list_len[a.win] > list_len[b.win];
-    });
-    // One-block items (the key-split forward kernel): every real row block,
-    // in (head, block) order, longest lists first.
+        for (int32_t h = 0; h < heads; ++h) P.computed_pairs += int64_t(P.tiles_per_head) * list_len[P.head_win[h]];
+    // Forward work items (the key-split kernel): every real row block once,
+    // in (head, block) order, longest lists first (stable: neighbouring tiles
+    // stay together for L2 reuse).
     P.f1_items.clear();
     for (int32_t b = 0; b < batch; ++b)
         for (int32_t h = 0; h < heads; ++h)
@@ -455,7 +427,6 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
     cudaError_t e = cudaGetDevice(&p->device);
     if (e == cudaSuccess) e = upload(&p->d_off, p->h.csr_off, s);
     if (e == cudaSuccess) e = upload(&p->d_ids, p->h.csr_ids, s);
-    if (e == cudaSuccess) e = upload(&p->d_items, p->h.items, s);
     if (e == cudaSuccess) e = upload(&p->d_f1_items, p->h.f1_items, s);
     if (e == cudaSuccess) e = upload(&p->d_origin, p->h.tile_origin, s);
     if (e == cudaSuccess && p->h.padded) e = upload(&p->d_kmask, p->h.key_mask, s);
@@ -524,14 +495,14 @@ sta_status sta_plan_key_query(sta_plan_t p, int32_t head, int32_t k_tile, int32_
 sta_status sta_plan_stats(sta_plan_t p, int64_t* computed_tile_pairs, int64_t* work_items) {
     if (p == nullptr) return STA_ERR_INVALID_ARG;
     if (computed_tile_pairs) *computed_tile_pairs = p->h.computed_pairs;
-    if (work_items) *work_items = int64_t(p->h.items.size());
+    if (work_items) *work_items = int64_t(p->h.f1_items.size());
     return STA_OK;
 }
 
 sta_status sta_plan_work_items(sta_plan_t p, int32_t* items4, int64_t cap, int64_t* count) {
     if (p == nullptr || count == nullptr || cap < 0 || (cap > 0 && items4 == nullptr))
         return STA_ERR_INVALID_ARG;
-    const auto& it = p->h.items;
+    const auto& it = p->h.f1_items;
     *count = int64_t(it.size());
     const int64_t n = std::min<int64_t>(cap, int64_t(it.size()));
     for (int64_t i = 0; i < n; ++i) {

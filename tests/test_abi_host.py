@@ -160,15 +160,10 @@ def test_work_list_covers_every_row_block_once():
         lens = []
         for bh, qa, qb, win in items:
             h = bh % heads
-            blocks = [qa] + ([qb] if qb >= 0 else [])
-            for r in blocks:
-                assert 0 <= r < n_tiles * S
-                seen[(bh, r)] = seen.get((bh, r), 0) + 1
-            if qb >= 0 and S % 2 == 0:
-                assert qa // S == qb // S  # paired blocks of one tile share K/V
+            assert qb == -1  # one query block per item
+            assert 0 <= qa < n_tiles * S
+            seen[(bh, qa)] = seen.get((bh, qa), 0) + 1
             lens.append(len(p.query(h, qa // S)))
-            if qb >= 0:
-                assert len(p.query(h, qb // S)) == lens[-1]
         real = real_blocks(latent, tile)
         assert sorted(seen) == [(bh, r) for bh in range(batch * heads) for r in real]
         assert all(c == 1 for c in seen.values())
