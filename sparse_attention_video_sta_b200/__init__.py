@@ -231,7 +231,8 @@ class Plan:
         return pairs.value, items.value
 
     def work_items(self):
-        """Work list as a list of (bh, first row block, second row block or -1, window id)."""
+        """The forward's work list as (bh, query row block, -1, window id)
+        tuples, in the order the kernel hands them out."""
         count = ctypes.c_int64(0)
         _check(_lib.sta_plan_work_items(self.handle, None, 0, ctypes.byref(count)), "sta_plan_work_items")
         buf = (ctypes.c_int32 * max(4 * count.value, 4))()
