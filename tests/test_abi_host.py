@@ -346,6 +346,28 @@ def test_empty_problems_are_no_ops():
                                    ctypes.c_float(0.088), None) == INV
 
 
+def test_noalloc_limits_rejected_before_any_cuda_call():
+    """The allocation-free forward rejects problems beyond its fixed scratch
+    (more than 1024 heads, or a plan image above 4 MiB) with UNSUPPORTED
+    before it looks up the scratch or launches anything, so the placeholder
+    (never dereferenced) tensor addresses below are safe on any machine."""
+    lib = sta._lib
+    UNS = 2
+    g = sta._geom((30, 48, 80), (6, 8, 8))
+    fake = ctypes.c_void_p(1 << 20)
+    lse = ctypes.cast(fake, ctypes.POINTER(ctypes.c_float))
+    scale = ctypes.c_float(0.088)
+    heads = 1025
+    w = (ctypes.c_int32 * (3 * heads))(*([18, 24, 24] * heads))
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 1, heads, w, fake, fake, fake, fake, lse, 128,
+                                   scale, None) == UNS
+    # 1024 heads of the 720p latent: 460 800 two-block items, 7.4 MB of plan
+    heads = 1024
+    w = (ctypes.c_int32 * (3 * heads))(*([18, 24, 24] * heads))
+    assert lib.sta_forward_noalloc(ctypes.byref(g), 1, heads, w, fake, fake, fake, fake, lse, 128,
+                                   scale, None) == UNS
+
+
 def test_device_helper_requires_one_cuda_device():
     """The binding's device check (no GPU needed): host tensors alone name no
     CUDA device; a plan's device is used when no tensor is given."""
