@@ -155,6 +155,21 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+REJECTED_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+def clocks_rejected(clocks) -> bool:
+    """A timed region is measured again when its clock record shows a
+    hardware or thermal slowdown, or SM clocks far below their maximum with no
+    reason given (a clock lock left behind).  The power cap alone is normal
+    for a dense tensor-core kernel and is kept."""
+    if not clocks:
+        return False
+    if REJECTED_REASONS & set(clocks.get("reasons", [])):
+        return True
+    return not clocks.get("reasons") and clocks["sm_mhz"] < 0.75 * clocks["sm_max_mhz"]
+
+
 def workload_config(w, wins, world: int) -> dict:
     """The ``config`` object both arms print."""
     return {"workload": w.name, "batch": w.batch, "heads": w.heads, "head_dim": w.head_dim,
@@ -385,21 +400,32 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {sta.sta_status_string(status)} after warm-up")
 
-    sampler = ClockSampler(dev.index) if rank == 0 else None
-    if sampler:
-        sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    start.record()
-    for _ in range(args.steps):
-        step(record=True)
-    stop.record()
-    torch.cuda.synchronize()
-    barrier()
-    clocks = sampler.stop() if sampler else None
-    ms_local = start.elapsed_time(stop) / args.steps
-    fwd_ms_local = statistics.mean(a.elapsed_time(b) for a, b in ev_fwd)
+    def timed_region():
+        ev_fwd.clear()
+        sampler = ClockSampler(dev.index) if rank == 0 else None
+        if sampler:
+            sampler.start()
+        barrier()
+        torch.cuda.synchronize()
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(args.steps):
+            step(record=True)
+        stop.record()
+        torch.cuda.synchronize()
+        barrier()
+        clocks = sampler.stop() if sampler else None
+        return (start.elapsed_time(stop) / args.steps, statistics.mean(a.elapsed_time(b) for a, b in ev_fwd),
+                clocks)
+
+    ms_local, fwd_ms_local, clocks = timed_region()
+    # Rank 0 samples the clocks; every rank takes its decision, so all of them
+    # run the second timed region together.
+    if reduce_max(1.0 if clocks_rejected(clocks) else 0.0) > 0.5:
+        first = clocks
+        ms_local, fwd_ms_local, clocks = timed_region()
+        if clocks is not None:
+            clocks["remeasured_after"] = first
     ms = reduce_max(ms_local)
     fwd_ms = reduce_max(fwd_ms_local)
     status = sta.sta_last_device_status(plan)

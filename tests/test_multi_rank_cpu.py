@@ -63,3 +63,16 @@ def test_reference_arm_exits_quietly_on_other_ranks():
                        timeout=120)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def test_clock_records_that_are_measured_again():
+    import bench
+    cap = {"sm_mhz": 1400.0, "sm_max_mhz": 1965.0, "samples": 10, "reasons": ["sw_power_cap"]}
+    assert not bench.clocks_rejected(cap)  # the power cap alone is kept
+    assert not bench.clocks_rejected(None)
+    assert not bench.clocks_rejected({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "samples": 5, "reasons": []})
+    for bad in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"):
+        assert bench.clocks_rejected({"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "samples": 5,
+                                      "reasons": ["sw_power_cap", bad]})
+    # clocks far below their maximum with no reason: a clock lock left behind
+    assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "samples": 5, "reasons": []})
