@@ -1,15 +1,19 @@
 """Shared helpers of the GPU parity tests: sampling, oracle rows, tolerances.
 
 Tolerances (CUDA path vs the fp64 oracle on the same bf16 inputs):
-  O   : |delta| <= 2e-2 + 2^-9 |O_ref| element-wise, and mean |delta| <= 2e-3
+  O   : |delta| <= max(2e-2, 2^-9 |O_ref| (1 + 2^-8)) element-wise, and
+        mean |delta| <= 2e-3
   LSE : |delta| <= 1e-3 * max(|LSE_ref|, 1)
 Plan and permutation results are compared bit-exactly.
 
 The 2e-2 / 2e-3 budget is the stated one.  The outputs are bf16 by
 specification, and rounding an exact value to bf16 alone moves it by up to half
-an ulp, 2^-9 |O|: more than 2e-2 once |O| >= 8 (possible on the workload whose
-heads are scaled by up to 2).  That unavoidable rounding is allowed on top of
-the budget; for |O| < 1 the bound stays within 2.2e-2.
+an ulp, 2^-9 |O|: that reaches 2e-2 only once |O| >= 10.24, which the workload
+whose heads are scaled by up to 2 can approach.  There the bound becomes that
+half ulp (with a 2^-8 relative margin); below it, the stated 2e-2 holds as is.
+
+Every comparison is recorded in ``REPORT`` (case, max |dO|, mean |dO|, max
+relative dLSE), which ``conftest.py`` prints at the end of the run.
 """
 from __future__ import annotations
 
@@ -20,8 +24,26 @@ import oracle
 
 O_MAX_TOL = 2e-2
 BF16_HALF_ULP_REL = 2.0 ** -9
+BF16_ULP_MARGIN = 1.0 + 2.0 ** -8
 O_MEAN_TOL = 2e-3
 LSE_REL_TOL = 1e-3
+
+# (case, max |dO|, mean |dO|, max relative dLSE) of every forward comparison
+REPORT: list[tuple[str, float, float, float]] = []
+# (case, worst max excess / rms, worst mean / rms) of every gradient comparison
+GRAD_REPORT: list[tuple[str, float, float]] = []
+
+
+def o_bound(o_ref):
+    """Element-wise bound on |O_gpu - O_ref|: the stated 2e-2, or the bf16
+    half ulp of the reference value where that is larger (|O_ref| > 10.24)."""
+    if isinstance(o_ref, torch.Tensor):
+        return torch.clamp(BF16_HALF_ULP_REL * BF16_ULP_MARGIN * o_ref.abs(), min=O_MAX_TOL)
+    return np.maximum(O_MAX_TOL, BF16_HALF_ULP_REL * BF16_ULP_MARGIN * np.abs(o_ref))
+
+
+def record(what: str, stats) -> None:
+    REPORT.append((what or "(unnamed)", float(stats[0]), float(stats[1]), float(stats[2])))
 
 
 def grid(latent, tile):
@@ -69,9 +91,10 @@ def compare(o_gpu: torch.Tensor, lse_gpu: torch.Tensor, o_ref: np.ndarray, lse_r
     lse = lse_gpu.detach().cpu().to(torch.float64).numpy()
     assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), what
     do = np.abs(o - o_ref)
-    bound = O_MAX_TOL + BF16_HALF_ULP_REL * np.abs(o_ref)
+    bound = o_bound(o_ref)
     dl = np.abs(lse - lse_ref) / np.maximum(np.abs(lse_ref), 1.0)
     stats = (float(do.max()), float(do.mean()), float(dl.max()))
+    record(what, stats)
     worst = np.unravel_index(int(np.argmax(do - bound)), do.shape)
     assert np.all(do <= bound), (what, stats, "worst", worst, float(o_ref[worst]), float(o[worst]))
     assert stats[1] <= O_MEAN_TOL, (what, stats)
@@ -157,4 +180,5 @@ def compare_grad(got, ref: np.ndarray, bh: np.ndarray, what: str = "", extra: np
         assert excess <= GRAD_RMS_TOL, (what, int(s), "max excess / rms", excess)
         assert mean <= GRAD_MEAN_TOL, (what, int(s), "mean / rms", mean)
         worst = (max(worst[0], excess), max(worst[1], mean))
+    GRAD_REPORT.append((what or "(unnamed)", worst[0], worst[1]))
     return worst

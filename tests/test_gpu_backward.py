@@ -76,6 +76,26 @@ def test_backward_small_geometries_all_rows(sta, latent, tile, B, H, d, windows)
     check_all_rows(sta, latent, tile, B, H, d, windows, 1.0 / np.sqrt(d), seed=sum(latent) + H + d)
 
 
+def test_backward_long_transposed_lists_all_keys(sta):
+    """Full window over a 5 x 4 x 5 grid of 6 x 8 x 8 tiles (100 tiles, 38 400
+    tokens): every key block's transposed list holds all 100 query tiles, so
+    the dK / dV kernel accumulates over 300 query blocks per item, the longest
+    lists any element-wise check here reaches.  dK and dV at every key row,
+    against the oracle (about a minute of host work on 16 cores)."""
+    latent, tile, B, H, d = (30, 32, 40), (6, 8, 8), 1, 1, 128
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator().manual_seed(4242)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(4))
+    windows = [list(latent)]
+    scale = 1.0 / np.sqrt(d)
+    plan, dq, dk, dv = gpu_grads(sta, q, k, v, do, latent, tile, windows, scale)
+    assert len(plan.key_query(0, 0)) == 100 and len(plan.key_query(0, 57)) == 100
+    rk, rv = oracle.sta_backward_dkdv(q, k, v, do, latent, tile, windows, scale)
+    bh = np.repeat(np.arange(B * H), N)
+    compare_grad(dk.cpu().reshape(-1, d), rk.reshape(-1, d), bh, what="dk full window, 100-tile lists")
+    compare_grad(dv.cpu().reshape(-1, d), rv.reshape(-1, d), bh, what="dv full window, 100-tile lists")
+
+
 def test_backward_720p_sampled(sta):
     """The 720p workload with window (18,24,24): dQ on sampled query rows of
     every tile class, dK / dV on sampled keys of corner, edge and centre tiles."""

@@ -110,7 +110,7 @@ def sampled_parity(sta, idx, heads, n_random, rows_per_tile, fused=True):
     bhs = [b * w.heads + h for b in range(w.batch) for h in heads]
     rows, o_ref, lse_ref = oracle_rows(q, k, v, w.latent, w.tile, wins, w.softmax_scale, bhs, toks)
     og, lg = gather_rows(o, lse, rows, w.heads)
-    stats = compare(og, lg, o_ref, lse_ref, what=f"workload {idx}")
+    stats = compare(og, lg, o_ref, lse_ref, what=f"workload {idx}" + ("" if fused else " (permuted path)"))
     return w, plan, o, lse, stats
 
 

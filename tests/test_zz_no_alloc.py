@@ -15,7 +15,7 @@ import math
 import pytest
 import torch
 
-from parity_util import BF16_HALF_ULP_REL, LSE_REL_TOL, O_MAX_TOL, O_MEAN_TOL
+from parity_util import LSE_REL_TOL, O_MEAN_TOL, o_bound
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ CASES = [
 
 def check_close(o, lse, o_ref, lse_ref):
     do = (o.double() - o_ref.double()).abs()
-    bound = O_MAX_TOL + BF16_HALF_ULP_REL * o_ref.double().abs()
+    bound = o_bound(o_ref.double())
     assert bool((do <= bound).all()), float(do.max())
     assert float(do.mean()) <= O_MEAN_TOL
     dl = (lse.double() - lse_ref.double()).abs() / lse_ref.double().abs().clamp_min(1.0)
