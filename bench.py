@@ -45,7 +45,7 @@ FWD_SOURCES = ["sparse_attention_video_sta_b200/csrc/sta_forward.cu",
                "sparse_attention_video_sta_b200/csrc/sta_internal.h",
                "sparse_attention_video_sta_b200/csrc/sta_raster.cuh",
                "sparse_attention_video_sta_b200/csrc/sta_wait.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "sta_fwd_720p_traffic.json")
+COUNTERS_FILE = os.path.join(ROOT, "profiles", "sta_fwd_counters.json")
 
 
 def parse():
@@ -84,17 +84,20 @@ def sources_hash():
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload_name: str):
-    """DRAM bytes per forward launch from the committed ncu summary, or None
-    when it covers another workload or the kernel sources changed since the
-    counters were taken."""
+def measured_counters(workload_name: str):
+    """ncu counters of one forward launch of ``workload_name`` from the
+    committed capture (DRAM bytes per full launch, tensor-pipe and XU/ex2-pipe
+    activity), or None when the capture covers another workload or the kernel
+    sources changed since the counters were taken."""
     try:
-        with open(TRAFFIC_FILE) as f:
-            t = json.load(f)
-        if t.get("sources_hash") == sources_hash() and t.get("workload") == workload_name:
-            return float(t["dram_bytes_per_launch"])
+        with open(COUNTERS_FILE) as f:
+            entries = json.load(f)["captures"]
     except Exception:
-        pass
+        return None
+    h = sources_hash()
+    for t in entries:
+        if t.get("sources_hash") == h and t.get("workload") == workload_name:
+            return t
     return None
 
 
@@ -151,8 +154,10 @@ class ClockSampler:
         if not sm:
             return None
         busy = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        rec = {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "samples": len(sm),
+               "reasons": sorted(reasons)}
+        rec["rejected"] = clocks_rejected(rec)
+        return rec
 
 
 REJECTED_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
@@ -313,7 +318,115 @@ def time_backward(sta, plan, q, k, v, o, lse, scale, gen, flops, warmup, reps, r
             "launches": 3, "layout": "raster (permutation fused)"}
 
 
+def make_inputs(w, dev, rank: int):
+    """Q, K, V of workload ``w`` on the device: N(0, 1) bf16, times the
+    workload's per-head factor where it has one (seeded per rank)."""
+    B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
+    gen = torch.Generator(device=dev).manual_seed(w.seed * 1000 + rank)
+    out = [torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    f = sta_inputs.head_factors(w)
+    for t in out:
+        for b in range(B):
+            for h in range(H):
+                x = torch.randn((N, d), generator=gen, device=dev, dtype=torch.float32)
+                if f is not None:
+                    x.mul_(float(f[h]))
+                t[b, h].copy_(x)
+    return out, gen
+
+
+def time_calls(fn, reps: int, warmup: int, dev, sample_clocks: bool):
+    """Mean device time of ``fn`` over ``reps`` calls after ``warmup`` calls
+    (CUDA events on the current stream), with the clock record of the timed
+    region when ``sample_clocks``."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index) if sample_clocks else None
+    if sampler:
+        sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    return e0.elapsed_time(e1) / reps, clocks
+
+
+def roofline_peak(peaks, region_ms: float):
+    """Dense bf16 peak for a kernel timed over ``region_ms``: the burst figure
+    for a region under 4 s, the sustained (power-capped) one beyond."""
+    if region_ms < 4000.0:
+        return float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), "bf16_tflops (burst)"
+    return (float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])),
+            "bf16_tflops_sustained")
+
+
+def workload_leg(sta, idx: int, dev, rank: int, peaks, reduce_max, full_720p_ms=None):
+    """Time the fused forward on workload ``idx`` at full size, with its clock
+    record and, where a capture of the current kernel exists, its ncu pipe
+    counters.  The mixed-window workload gets its speedup over the
+    full-window run of the same latent (``full_720p_ms``) against the ideal
+    ratio of its drawn heads; the large workload its own full-window run."""
+    w = sta_inputs.WORKLOADS[idx]
+    (q, k, v), _ = make_inputs(w, dev, rank)
+    wins = sta_inputs.windows(w).tolist()
+    plan = sta.sta_plan(w.latent, w.tile, w.batch, w.heads, wins)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.batch, w.heads, w.tokens), dtype=torch.float32, device=dev)
+    scale = w.softmax_scale
+    flops = plan.flops(w.head_dim)
+    est_ms = max(flops / 1.0e15 * 1e3, 0.01)  # at ~1 PFLOP/s
+    reps = int(min(50, max(3, 1500.0 / est_ms)))
+    ms, clocks = time_calls(lambda: sta.sta_forward_raster(plan, q, k, v, o, lse, scale), reps, 3, dev,
+                            rank == 0)
+    ms = reduce_max(ms)
+    if sta.sta_last_device_status(plan) != 0:
+        raise RuntimeError(f"device status error in workload {idx}")
+    tflops = flops / (ms * 1e-3) / 1e12
+    peak, peak_name = roofline_peak(peaks, ms * reps)
+    in_bytes = 3 * q.numel() * q.element_size()
+    res = {"workload": w.name, "ms": ms, "reps": reps, "tflops": tflops, "flops": flops,
+           "frac": tflops / peak, "peak": peak, "peak_source": peak_name, "clocks": clocks,
+           "l2": ("inputs larger than L2, no flush" if in_bytes > 126e6
+                  else "inputs fit in L2 (%.1f MB): L2-resident timing" % (in_bytes / 1e6))}
+    cnt = measured_counters(w.name)
+    res["tensor_pipe_pct"] = cnt.get("tensor_pipe_pct") if cnt else None
+    res["xu_pipe_pct"] = cnt.get("xu_pipe_pct") if cnt else None
+    res["traffic"] = cnt.get("dram_bytes_per_launch") if cnt else None
+    pairs = plan.stats()[0]
+    if idx == 3 and full_720p_ms is not None:
+        tiles = 1
+        for i in range(3):
+            tiles *= w.latent[i] // w.tile[i]
+        ideal = (w.batch * w.heads * tiles * tiles) / pairs  # the full window: every tile attends every tile
+        res["speedup_vs_full"] = full_720p_ms / ms
+        res["ideal_speedup"] = ideal
+        res["frac_of_ideal"] = res["speedup_vs_full"] / ideal
+    if idx == 5:
+        full = sta.sta_plan(w.latent, w.tile, w.batch, w.heads, [tuple(w.latent)] * w.heads)
+        f_ms, f_clocks = time_calls(lambda: sta.sta_forward_raster(full, q, k, v, o, lse, scale), 2, 1, dev,
+                                    rank == 0)
+        f_ms = reduce_max(f_ms)
+        if sta.sta_last_device_status(full) != 0:
+            raise RuntimeError("device status error in the large workload's full-window run")
+        ideal = full.stats()[0] / pairs
+        res["full_window"] = {"ms": f_ms, "reps": 2, "tflops": full.flops(w.head_dim) / (f_ms * 1e-3) / 1e12,
+                              "clocks": f_clocks}
+        res["speedup_vs_full"] = f_ms / ms
+        res["ideal_speedup"] = ideal
+        res["frac_of_ideal"] = res["speedup_vs_full"] / ideal
+        full.destroy()
+    plan.destroy()
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
+
     args = parse()
     w = sta_inputs.WORKLOADS[args.workload]
     if args.heads > 0:
@@ -347,16 +460,7 @@ def main():
     # ---------------------------------------------------------------- inputs
     B, H, N, d = w.batch, w.heads, w.tokens, w.head_dim
     shape = (B, H, N, d)
-    gen = torch.Generator(device=dev).manual_seed(w.seed * 1000 + rank)
-    q, k, v = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
-    f = sta_inputs.head_factors(w)
-    for t in (q, k, v):
-        for b in range(B):
-            for h in range(H):
-                x = torch.randn((N, d), generator=gen, device=dev, dtype=torch.float32)
-                if f is not None:
-                    x.mul_(float(f[h]))
-                t[b, h].copy_(x)
+    (q, k, v), gen = make_inputs(w, dev, rank)
     wins = sta_inputs.windows(w).tolist()
     plan = sta.sta_plan(w.latent, w.tile, B, H, wins)
     flops = plan.flops(d)
@@ -435,7 +539,9 @@ def main():
     value = weak_scaling_tflops(world, flops, ms)
     fwd_tflops = flops / (fwd_ms * 1e-3) / 1e12
     peaks, peak_kind = load_peaks()
-    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak, peak_name = roofline_peak(peaks, ms * args.steps)
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    counters = measured_counters(w.name)
 
     extras = {}
     e2e = None
@@ -443,21 +549,17 @@ def main():
         # ------------------------------------------- full-window denominator
         o_win, lse_win = o.clone(), lse.clone()  # the timed step's output (the STA window)
         full = sta.sta_plan(L, T, B, H, [tuple(L)] * H)
-        for _ in range(2):
-            sta.sta_forward_raster(full, q, k, v, o, lse, scale)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 3
-        e0.record()
-        for _ in range(reps):
-            sta.sta_forward_raster(full, q, k, v, o, lse, scale)
-        e1.record()
-        torch.cuda.synchronize()
-        full_ms = reduce_max(e0.elapsed_time(e1) / reps)
+        full_ms, full_clocks = time_calls(lambda: sta.sta_forward_raster(full, q, k, v, o, lse, scale), 5, 2,
+                                          dev, rank == 0)
+        full_ms = reduce_max(full_ms)
         ideal = full.stats()[0] / plan.stats()[0]
         extras["full_window"] = {"ms": full_ms, "tflops": full.flops(d) / (full_ms * 1e-3) / 1e12,
                                  "speedup": full_ms / fwd_ms, "ideal_speedup": ideal,
-                                 "frac_of_ideal": (full_ms / fwd_ms) / ideal}
+                                 "frac_of_ideal": (full_ms / fwd_ms) / ideal, "reps": 5, "clocks": full_clocks}
+        fw_cnt = measured_counters(sta_inputs.WORKLOADS[4].name) if tuple(w.latent) == (30, 48, 80) else None
+        if fw_cnt:
+            extras["full_window"]["tensor_pipe_pct"] = fw_cnt.get("tensor_pipe_pct")
+            extras["full_window"]["traffic"] = fw_cnt.get("dram_bytes_per_launch")
         if sta.sta_last_device_status(full) != 0:
             raise RuntimeError("device status error in the full-window run")
         full.destroy()
@@ -559,6 +661,12 @@ def main():
                "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
                "api": "sta_pipe (copies overlapped across steps)", "steps": e2e_steps}
 
+    if not args.no_extras and args.workload == 2 and args.heads == 0:
+        # ------------------------------------------- the other workloads at full size
+        full_720p = extras.get("full_window", {}).get("ms")
+        extras["workloads"] = {str(i): workload_leg(sta, i, dev, rank, peaks, reduce_max, full_720p)
+                               for i in (1, 3, 5)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_extras:
         cpu = cpu_baseline(w, n_tiles=64, heads=[0, 1])  # ~13 s on 16 host cores
@@ -571,10 +679,16 @@ def main():
             "config": workload_config(w, wins, world),
             "fwd_ms": fwd_ms, "fwd_tflops": fwd_tflops, "flops_per_step": flops,
             "roofline": {"bound": "tensor", "achieved": fwd_tflops, "peak": peak, "unit": "TFLOP/s",
-                         "frac": fwd_tflops / peak, "traffic": measured_traffic(w.name),
+                         "frac": fwd_tflops / peak,
+                         "traffic": counters.get("dram_bytes_per_launch") if counters else None,
                          "kernel": f"sta_fwd_split_kernel<{d}, raster>",
-                         "peak_source": f"bf16_tflops_sustained ({peak_kind})",
-                         "frac_of_burst": fwd_tflops / float(peaks.get("bf16_tflops", 1590.0))},
+                         "peak_source": f"{peak_name} ({peak_kind}); timed region {ms * args.steps:.0f} ms",
+                         "frac_sustained": fwd_tflops / sustained,
+                         "tensor_pipe_pct": counters.get("tensor_pipe_pct") if counters else None,
+                         "xu_pipe_pct": counters.get("xu_pipe_pct") if counters else None,
+                         "counters_from": counters.get("captured_on") if counters else None},
+            "tensor_pipe_pct": counters.get("tensor_pipe_pct") if counters else None,
+            "xu_pipe_pct": counters.get("xu_pipe_pct") if counters else None,
             "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks,
             "e2e": e2e,
