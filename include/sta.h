@@ -314,30 +314,32 @@ STA_API sta_status sta_pipe_destroy(sta_pipe_t pipe);
  * the device synchronisation cudaMalloc may cause, while it serves; a plugin
  * host that only hands a library the buffers it is meant to touch.  This call
  * takes the geometry, batch, heads and per-head windows of sta_plan and the
- * tensors of sta_forward (same layouts and rules), builds the plan on the host
- * without heap use, and keeps it in a fixed scratch array compiled into the
- * library: 4 MiB of device memory on every GPU that loads the library, held
- * until the process exits.
+ * tensors of sta_forward (same layouts and rules: tile-major q, k, v, o, lse),
+ * and keeps the plan in a fixed scratch array compiled into the library: 4 MiB
+ * of device memory on every GPU that loads the library, held until the process
+ * exits.  It computes the same results as sta_plan + sta_forward.
  *
  * Limits: every latent axis a multiple of its tile (padded latents need
  * sta_plan + sta_forward), heads <= 1024, and the plan must fit the scratch:
- *   256 + 16 * work_items + 4 * (n_windows * (tiles + 1) + sum over distinct
- *   windows of tiles * window_tiles) <= 4 MiB
- * (the 720p and 42x64x112 workloads of this library use 0.7 and 1.3 MiB).
+ *   256 + 16 * B * heads * tiles * (tile volume / 128)
+ *       + 4 * (n_windows * (tiles + 1) + sum over distinct windows of
+ *              tiles * window_tiles) <= 4 MiB
+ * (the 720p and 42x64x112 workloads of this library use 0.36 and 2.1 MiB).
  * Larger problems, heads > 1024 or a padded latent return STA_ERR_UNSUPPORTED
  * before any work.  batch 0 returns STA_OK at once (pointers unread).
  *
  * Behaviour: the first call on a device looks up the scratch's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture.  Each call copies the plan from a static host buffer into the
- * scratch on `stream` (this also clears the status word) and launches the
- * forward kernel.  Every call shares the one scratch array: calls whose work
- * overlaps on the GPU (different streams, or threads enqueueing concurrently)
- * race and must be serialised by the caller, e.g. by using one stream.  Host
- * threads are serialised inside the call.  A device-side timeout ends the
- * kernel cleanly but is not reported by this call (use sta_forward with a plan
- * and sta_last_device_status to observe it).  Errors: as sta_plan and
- * sta_forward, UNSUPPORTED beyond the limits, CUDA on a failed copy or launch. */
+ * capture.  Each call enqueues two kernels on `stream`: one writes the plan
+ * into the scratch (from the windows, which it receives as kernel arguments;
+ * nothing is copied from host memory) and clears the status word and work
+ * counter kept there, the second is the forward.  Every call shares the one
+ * scratch array: calls whose work overlaps on the GPU (different streams, or
+ * threads enqueueing concurrently) race and must be serialised by the caller,
+ * e.g. by using one stream.  A device-side timeout ends the kernel cleanly but
+ * is not reported by this call (use sta_forward with a plan and
+ * sta_last_device_status to observe it).  Errors: as sta_plan and
+ * sta_forward, UNSUPPORTED beyond the limits, CUDA on a failed launch. */
 STA_API sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int32_t heads,
                                        const int32_t* window_thw, const void* q, const void* k,
                                        const void* v, void* o, float* lse, int32_t head_dim,
@@ -356,11 +358,21 @@ STA_API const char* sta_last_error_detail(void);
 /* Static string naming a status code. */
 STA_API const char* sta_status_string(sta_status s);
 
-/* Debug only: when `enable` is non-zero, the next sta_forward calls make the
- * kernel's first wait run out on a barrier nothing arrives at (time limit
- * `limit_ms`), so the timeout path can be tested; the kernel then issues no
- * copy or MMA and exits, and sta_last_device_status returns TIMEOUT. */
-STA_API sta_status sta_debug_inject_timeout(int32_t enable, int32_t limit_ms);
+/* Debug only: makes a device-side wait of the next forward calls
+ * (sta_forward, sta_forward_raster) run out on a barrier nothing arrives at,
+ * so the timeout path can be tested without a fault.  Every wait of those
+ * calls then has the time limit `limit_ms` (1..10000).
+ *   mode 0: off (the default).
+ *   mode 1: the load warp's first wait runs out: the kernel issues no copy or
+ *           MMA and exits.
+ *   mode 2: in every CTA that takes a second work item, the S-issuing
+ *           thread's wait at the start of that item runs out after the first
+ *           item has been computed and the second item's query block and K/V
+ *           chunks have been issued; the kernel waits (bounded) for those
+ *           copies and its MMAs, frees TMEM and exits.
+ * In both cases the outputs are left partly written and
+ * sta_last_device_status returns TIMEOUT.  Any other mode: INVALID_ARG. */
+STA_API sta_status sta_debug_inject_timeout(int32_t mode, int32_t limit_ms);
 
 #ifdef __cplusplus
 }

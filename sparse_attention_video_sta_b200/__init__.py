@@ -483,8 +483,11 @@ def sta_last_device_status(plan: Plan, stream=None) -> int:
         return int(_lib.sta_last_device_status(plan.handle, _stream(stream)))
 
 
-def sta_debug_inject_timeout(enable: bool, limit_ms: int = 50) -> None:
-    _check(_lib.sta_debug_inject_timeout(1 if enable else 0, int(limit_ms)), "sta_debug_inject_timeout")
+def sta_debug_inject_timeout(mode, limit_ms: int = 50) -> None:
+    """Debug: make a device-side wait of the next forward calls run out
+    (``mode`` 0 off, 1 or True: before any copy, 2: at a CTA's second work
+    item with copies issued); see sta.h."""
+    _check(_lib.sta_debug_inject_timeout(int(mode), int(limit_ms)), "sta_debug_inject_timeout")
 
 
 def sta_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, plan: Plan,

@@ -212,7 +212,6 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
             real_block[blk] = (m[0] | m[1] | m[2] | m[3]) != 0u;
         }
 
-    P.items.clear();  // two-block items: no longer built (the forward runs one-block items)
     P.computed_pairs = 0;
     for (int32_t b = 0; b < batch; ++b)
         for (int32_t h = 0; h < heads; ++h) P.computed_pairs += int64_t(P.tiles_per_head) * list_len[P.head_win[h]];
@@ -270,7 +269,6 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
 void free_device(sta_plan_s* p) {
     if (p->d_off) cudaFree(p->d_off);
     if (p->d_ids) cudaFree(p->d_ids);
-    if (p->d_items) cudaFree(p->d_items);
     if (p->d_f1_items) cudaFree(p->d_f1_items);
     p->d_f1_items = nullptr;
     if (p->d_status) cudaFree(p->d_status);
@@ -289,7 +287,6 @@ void free_device(sta_plan_s* p) {
     p->d_bkv_items = nullptr;
     p->d_off = nullptr;
     p->d_ids = nullptr;
-    p->d_items = nullptr;
     p->d_status = nullptr;
     p->d_origin = nullptr;
     p->on_device = false;
@@ -454,7 +451,7 @@ sta_status sta_plan(const sta_geom* g, int32_t batch, int32_t heads,
 sta_status sta_plan_destroy(sta_plan_t p) {
     if (p == nullptr) return STA_OK;
     sta_status st = STA_OK;
-    if (p->on_device || p->d_off || p->d_ids || p->d_items || p->d_f1_items || p->d_status || p->d_origin || p->d_kmask ||
+    if (p->on_device || p->d_off || p->d_ids || p->d_f1_items || p->d_status || p->d_origin || p->d_kmask ||
         p->d_counters || p->d_toff ||
         p->d_tids || p->d_bq_items || p->d_bkv_items) {
         if (cudaDeviceSynchronize() != cudaSuccess) st = STA_ERR_CUDA;
@@ -598,9 +595,9 @@ sta_status sta_last_device_status(sta_plan_t p, void* stream) {
 
 const char* sta_last_error_detail(void) { return g_detail; }
 
-sta_status sta_debug_inject_timeout(int32_t enable, int32_t limit_ms) {
-    if (limit_ms < 1 || limit_ms > 10000) return STA_ERR_INVALID_ARG;
-    g_inject_timeout.store(enable ? 1 : 0);
+sta_status sta_debug_inject_timeout(int32_t mode, int32_t limit_ms) {
+    if (limit_ms < 1 || limit_ms > 10000 || mode < 0 || mode > 2) return STA_ERR_INVALID_ARG;
+    g_inject_timeout.store(mode);
     g_inject_limit_ms.store(limit_ms);
     return STA_OK;
 }

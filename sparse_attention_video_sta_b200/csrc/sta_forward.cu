@@ -7,38 +7,14 @@
 // hotaipapers.com, segments on tiles and on dense / empty / mixed blocks).  The
 // pages' own kernel splits a thread block into data warpgroups that load K/V and
 // manage the sparse tile list, and compute warpgroups doing dense attention math
-// (same transcript, segment on ThunderKittens); the designs below keep that
-// split but are built for Blackwell.  Two kernels share the roles and the
-// helpers:
+// (same transcript, segment on ThunderKittens); the kernel below keeps that
+// split but is built for Blackwell: one 128-row query block per work item,
+// every 128-key chunk split between two softmax warpgroups, S double buffered
+// in TMEM (see the kernel's own comment).
 //
-//   sta_fwd_split_kernel (sta_forward, sta_forward_raster): one 128-row query
-//   block per work item, every 128-key chunk split between two softmax
-//   warpgroups, S double buffered in TMEM; see its own comment.
-//
-//   sta_fwd_kernel (the allocation-free entry point, whose plan lives in a
-//   fixed scratch array; its padded-latent and raster branches are kept for
-//   comparison but not instantiated):
-//   warp 8 (load)      : TMA loads of the query blocks and of the 128-key K / V
-//                        chunks of the listed key tiles into a ring of stages
-//   warps 9, 10 (MMA)  : one thread each, for query slot 0 / 1, issues
-//                        tcgen05.mma: S = Q K^T into TMEM, then O += P V with P
-//                        read straight from TMEM.  A tcgen05.mma issue does not
-//                        return before the tensor pipe takes the instruction,
-//                        so a single issuing thread leaves the pipe idle
-//                        whenever it waits; two independent issuers keep it fed.
-//   warps 0-3, 4-7     : softmax for query slot 0 / 1 (one thread per row):
-//                        tcgen05.ld of S, online softmax (fp32 running max and
-//                        sum, exp2 with the scale folded in, lazy rescale of O),
-//                        bf16 P written back into TMEM over S, and the epilogue
-//                        O / l -> bf16, LSE
-//
-//   A work item is up to two 128-row query blocks (slots) of one (b, h).
-//   Blocks of the same tile share every K/V chunk load.  TMEM (512 columns):
-//   S0 | S1 | O0 | O1.
-//
-// Both kernels are persistent (one CTA per SM) over the plan's work list,
-// longest key lists first, items handed out at run time.  Every mbarrier wait
-// has a time limit; on expiry the kernel records STA timeout status, drains its
+// The kernel is persistent (one CTA per SM) over the plan's work list, longest
+// key lists first, items handed out at run time.  Every mbarrier wait has a
+// time limit; on expiry the kernel records STA timeout status, drains its
 // copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -56,9 +32,9 @@
 namespace sta {
 namespace {
 
-constexpr int kThreads = 384;  // 3 warpgroups: softmax slot 0, softmax slot 1, producers
+constexpr int kThreads = 384;  // 3 warpgroups: softmax half A, softmax half B, producers
 constexpr int kLoadWarp = 8;
-constexpr int kMmaWarp0 = 9;  // slot 0 issuer; also allocates TMEM.  Slot 1 issuer: warp 10.
+constexpr int kMmaWarp0 = 9;  // PV issuer; also allocates TMEM.  S issuer: warp 10.
 // Registers per thread: launched at 168 (384 threads, 3 warps per SM
 // sub-partition); the producer warpgroup (warps 8-11, warp 11 idle) gives
 // registers to the two softmax warpgroups.  128 * (208 + 208 + 88) is within the
@@ -73,36 +49,11 @@ constexpr uint32_t kTmemCols = 512;
 // grew a little) is redone against its own max, with O and l rescaled.
 constexpr float kRescaleRowSum = 256.0f;
 
-constexpr int kStagesD128 = 5;  // K/V ring stages of 32 KB at d = 128 (8 of 16 KB at d = 64)
 // Work items are handed out at run time: the load warp takes the next item
 // index from a global counter and passes it to the other roles through a
 // queue of this many entries in shared memory.  CTAs that run slower (their
 // SM's share of L2 and HBM, their items' tiles) then take fewer items.
 constexpr int kItemQ = 4;
-constexpr int kItemConsumers = 2 + 8;  // the two issuing threads and the eight softmax warps
-
-template <int D>
-struct Cfg {
-    static constexpr int kColBlocks = D / 64;             // 128-byte swizzle columns per row
-    static constexpr int kBoxBytes = 128 * 128;           // one TMA box: 128 rows x 128 bytes
-    static constexpr int kQBytes = kSubRows * D * 2;      // one 128-row query block
-    static constexpr int kKVBytes = kChunkKeys * D * 2;   // one 128-key K or V chunk
-    static constexpr int kStages = (D == 128) ? kStagesD128 : 8;
-    static constexpr int kQOff = 0;
-    static constexpr int kRingOff = 2 * kQBytes;
-    static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
-    // barriers: full[S], empty[S][2], q_full[2], q_empty[2], s_full[2], p_full[2],
-    // o_full[2], o_empty[2], dead, drain[2], turn[2], item_full[Q], item_empty[Q]
-    static constexpr int kNumBars = 3 * kStages + 17 + 2 * kItemQ;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base slot, abort flag, item queue
-    static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemQ + 1024;  // + alignment slack
-    // TMEM columns: S0 | S1 | O0 | O1
-    __host__ __device__ static constexpr uint32_t col_s(int slot) { return uint32_t(slot) * 128u; }
-    __host__ __device__ static constexpr uint32_t col_o(int slot) { return 256u + uint32_t(slot) * D; }
-    static_assert(256 + 2 * D <= int(kTmemCols), "TMEM budget");
-    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-    static_assert(kStages <= 16, "ring bookkeeping uses 2 bits per stage in a uint32");
-};
 
 struct FwdParams {
     const WorkItem* items;
@@ -120,6 +71,10 @@ struct FwdParams {
     float scale;
     uint32_t* status;
     uint64_t timeout_ns;
+    // Debug: 1 = the load warp's first wait runs out before any copy is
+    // issued; 2 = the S issuer's wait at the start of its CTA's second work
+    // item runs out, with that item's query block and K/V chunks already
+    // issued (copies in flight or landed, nothing consuming them).
     int32_t inject;
     RasterGeom rg;  // raster layout only
     // Padded latents (an axis not a multiple of the tile): real-key bits of
@@ -164,55 +119,6 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     return wait_bar_limited(bar, parity, abort_flag, p.status, p.timeout_ns);
 }
 
-// Padded latents: scores of the chunk's padding keys become -inf, so they take
-// no softmax weight.  `m` holds the chunk's real-key bits.
-__device__ __forceinline__ void mask_scores(uint32_t (&sr)[128], const uint4 m) {
-    const uint32_t w[4] = {m.x, m.y, m.z, m.w};
-#pragma unroll
-    for (int j = 0; j < 128; ++j)
-        if (!((w[j >> 5] >> (j & 31)) & 1u)) sr[j] = 0xff800000u;
-}
-
-// P = exp2(S * c - m * c) for one 128-score row, packed to bf16 pairs; returns
-// the fp32 row sum.
-__device__ __forceinline__ float softmax_exp(const uint32_t (&sr)[128], float c, float m, uint32_t (&pk)[64]) {
-    const uint64_t c2 = ptx::f2(c, c);
-    const uint64_t nmc2 = ptx::f2(-m * c, -m * c);
-    uint64_t acc0 = ptx::f2(0.0f, 0.0f), acc1 = acc0;
-#pragma unroll
-    for (int j = 0; j < 64; ++j) {
-        const float s0 = __uint_as_float(sr[2 * j]), s1 = __uint_as_float(sr[2 * j + 1]);
-        float x0, x1, p0, p1;
-        ptx::f2_split(ptx::f2_fma(ptx::f2(s0, s1), c2, nmc2), x0, x1);
-        p0 = ptx::ex2(x0);
-        p1 = ptx::ex2(x1);
-        if (j & 1)
-            acc1 = ptx::f2_add(acc1, ptx::f2(p0, p1));
-        else
-            acc0 = ptx::f2_add(acc0, ptx::f2(p0, p1));
-        pk[j] = ptx::pack_bf16x2(p0, p1);
-    }
-    float r0, r1, r2, r3;
-    ptx::f2_split(acc0, r0, r1);
-    ptx::f2_split(acc1, r2, r3);
-    return (r0 + r1) + (r2 + r3);
-}
-
-__device__ __forceinline__ float row_max(const uint32_t (&sr)[128]) {
-    float a0 = __uint_as_float(sr[0]), a1 = __uint_as_float(sr[1]);
-    float a2 = __uint_as_float(sr[2]), a3 = __uint_as_float(sr[3]);
-#pragma unroll
-    for (int j = 4; j < 124; j += 8) {
-        a0 = ptx::max3(a0, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
-        a1 = ptx::max3(a1, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
-        a2 = ptx::max3(a2, __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
-        a3 = ptx::max3(a3, __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
-    }
-    a0 = ptx::max3(a0, __uint_as_float(sr[124]), __uint_as_float(sr[125]));
-    a1 = ptx::max3(a1, __uint_as_float(sr[126]), __uint_as_float(sr[127]));
-    return ptx::max3(a0, a1, fmaxf(a2, a3));
-}
-
 // The same for one 64-score half row (key-split kernel): `lo`, `hi` hold the
 // real-key bits of the half's 64 keys.
 __device__ __forceinline__ void mask_scores64(uint32_t (&sr)[64], uint32_t lo, uint32_t hi) {
@@ -221,7 +127,12 @@ __device__ __forceinline__ void mask_scores64(uint32_t (&sr)[64], uint32_t lo, u
         if (!(((j < 32 ? lo : hi) >> (j & 31)) & 1u)) sr[j] = 0xff800000u;
 }
 
-// The same for one 64-score half row (key-split kernel).
+// P = exp2(S * c - m * c) for one 64-score half row, packed to bf16 pairs;
+// returns the fp32 sum of the bf16 values, the ones P V multiplies.  Summing
+// the rounded values keeps O / l a convex combination of V rows: with the
+// unrounded sum, a row dominated by one key whose P rounds by up to 2^-9 (the
+// running max is only updated lazily, so that P is rarely exactly 1) would
+// carry that rounding into O on top of O's own bf16 rounding.
 __device__ __forceinline__ float softmax_exp64(const uint32_t (&sr)[64], float c, float m, uint32_t (&pk)[32]) {
     const uint64_t c2 = ptx::f2(c, c);
     const uint64_t nmc2 = ptx::f2(-m * c, -m * c);
@@ -233,11 +144,12 @@ __device__ __forceinline__ float softmax_exp64(const uint32_t (&sr)[64], float c
         ptx::f2_split(ptx::f2_fma(ptx::f2(s0, s1), c2, nmc2), x0, x1);
         p0 = ptx::ex2(x0);
         p1 = ptx::ex2(x1);
-        if (j & 1)
-            acc1 = ptx::f2_add(acc1, ptx::f2(p0, p1));
-        else
-            acc0 = ptx::f2_add(acc0, ptx::f2(p0, p1));
         pk[j] = ptx::pack_bf16x2(p0, p1);
+        const uint64_t pr = ptx::f2(__uint_as_float(pk[j] << 16), __uint_as_float(pk[j] & 0xffff0000u));
+        if (j & 1)
+            acc1 = ptx::f2_add(acc1, pr);
+        else
+            acc0 = ptx::f2_add(acc0, pr);
     }
     float r0, r1, r2, r3;
     ptx::f2_split(acc0, r0, r1);
@@ -258,433 +170,6 @@ __device__ __forceinline__ float row_max64(const uint32_t (&sr)[64]) {
     a0 = ptx::max3(a0, __uint_as_float(sr[60]), __uint_as_float(sr[61]));
     a1 = ptx::max3(a1, __uint_as_float(sr[62]), __uint_as_float(sr[63]));
     return ptx::max3(a0, a1, fmaxf(a2, a3));
-}
-
-// kPadded: the latent has padding tokens (an axis that is not a multiple of
-// the tile): padding keys are masked and raster padding rows are not stored.
-template <int D, bool kRaster, bool kPadded>
-__global__ void __launch_bounds__(kThreads, 1)
-sta_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = Cfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw_base = ptx::smem_u32(smem_raw);
-    const uint32_t base = (raw_base + 1023u) & ~1023u;
-    uint8_t* smem = smem_raw + (base - raw_base);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    const uint32_t bar0 = base + C::kBarOff;
-    constexpr int S = C::kStages;
-    auto bar_full = [&](int r) { return bar0 + 8u * r; };
-    auto bar_empty = [&](int r, int s) { return bar0 + 8u * (S + 2 * r + s); };
-    auto bar_q_full = [&](int s) { return bar0 + 8u * (3 * S + 0 + s); };
-    auto bar_q_empty = [&](int s) { return bar0 + 8u * (3 * S + 2 + s); };
-    auto bar_s_full = [&](int s) { return bar0 + 8u * (3 * S + 4 + s); };
-    auto bar_p_full = [&](int s) { return bar0 + 8u * (3 * S + 6 + s); };
-    auto bar_o_full = [&](int s) { return bar0 + 8u * (3 * S + 8 + s); };
-    auto bar_o_empty = [&](int s) { return bar0 + 8u * (3 * S + 10 + s); };
-    const uint32_t bar_dead = bar0 + 8u * (3 * S + 12);
-    auto bar_drain = [&](int s) { return bar0 + 8u * (3 * S + 13 + s); };
-    auto bar_turn = [&](int s) { return bar0 + 8u * (3 * S + 15 + s); };
-    auto bar_item_full = [&](int q) { return bar0 + 8u * (3 * S + 17 + q); };
-    auto bar_item_empty = [&](int q) { return bar0 + 8u * (3 * S + 17 + kItemQ + q); };
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
-    volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(smem + C::kMiscOff + 8);
-    // Consumer side of the item queue: entry k holds the k-th item of this CTA
-    // (-1: none left).  Returns false when the CTA is aborting.
-    auto take_item = [&](uint32_t k, int32_t& u) -> bool {
-        const int q = int(k % kItemQ);
-        if (!wait_bar(bar_item_full(q), (k / kItemQ) & 1u, abort_flag, p)) return false;
-        u = item_q[q];
-        return true;
-    };
-
-    if (threadIdx.x == 0) {
-        for (int r = 0; r < S; ++r) {
-            ptx::mbar_init(bar_full(r), 1);
-            ptx::mbar_init(bar_empty(r, 0), 1);
-            ptx::mbar_init(bar_empty(r, 1), 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(bar_q_full(s), 1);
-            ptx::mbar_init(bar_q_empty(s), 1);
-            ptx::mbar_init(bar_s_full(s), 1);
-            ptx::mbar_init(bar_p_full(s), 4);  // one arrival per softmax warp
-            ptx::mbar_init(bar_o_full(s), 1);
-            ptx::mbar_init(bar_o_empty(s), 4);
-            ptx::mbar_init(bar_drain(s), 1);
-        }
-        ptx::mbar_init(bar_dead, 1);
-        ptx::mbar_init(bar_turn(0), 1);
-        ptx::mbar_init(bar_turn(1), 1);
-        for (int q = 0; q < kItemQ; ++q) {
-            ptx::mbar_init(bar_item_full(q), 1);
-            ptx::mbar_init(bar_item_empty(q), kItemConsumers);
-        }
-        *abort_flag = 0;
-        ptx::fence_barrier_init();
-        ptx::fence_proxy_async_smem();
-        ptx::mbar_arrive(bar_turn(0));  // slot 0 issues first
-    }
-    if (warp == kLoadWarp && lane == 0) {
-        ptx::prefetch_tensormap(&tm_q);
-        ptx::prefetch_tensormap(&tm_k);
-        ptx::prefetch_tensormap(&tm_v);
-    }
-    if (warp == kMmaWarp0) {
-        ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-
-    const int32_t SPT = p.sub_per_tile;
-
-    if (warp == kLoadWarp) {
-        ptx::regs_dec<kRegsProducer>();
-        if (lane == 0) {
-            // ------------------------------------------------------------ load
-            // Ring stage r holds one K or V chunk.  `users` keeps, 2 bits per
-            // stage, which issuers read the chunk now in it; `upar` keeps, per
-            // (stage, issuer), the parity of that issuer's uses of the stage.
-            // Before refilling a stage the previous readers' release is awaited.
-            uint32_t item = 0, qc0 = 0, qc1 = 0, users = 0, upar = 0;
-            bool ok = true;
-            if (p.inject) {
-                // Debug: wait on a barrier nothing arrives at; the limit runs out.
-                ok = wait_bar(bar_dead, 0, abort_flag, p);
-            }
-            auto issue = [&](const CUtensorMap* m, int32_t bh, int32_t tile, int4 org, int32_t sub,
-                             uint32_t mask) -> bool {
-                const int r = int(item % S);
-                const uint32_t prev = (users >> (2 * r)) & 3u;
-#pragma unroll
-                for (int s = 0; s < 2; ++s)
-                    if ((prev >> s) & 1u)
-                        if (!wait_bar(bar_empty(r, s), ((upar >> (2 * r + s)) & 1u) ^ 1u, abort_flag, p))
-                            return false;
-                users = (users & ~(3u << (2 * r))) | (mask << (2 * r));
-                upar ^= mask << (2 * r);
-                ptx::mbar_arrive_expect_tx(bar_full(r), C::kKVBytes);
-                load_block<kRaster>(base + C::kRingOff + r * C::kKVBytes, m, bar_full(r), p, bh, tile, org, sub,
-                                    C::kColBlocks, C::kBoxBytes);
-                ++item;
-                return true;
-            };
-            for (uint32_t k = 0; ok; ++k) {
-                // producer side of the item queue
-                int32_t u = p.item_counter != nullptr ? atomicAdd(p.item_counter, 1)
-                                                      : int32_t(blockIdx.x + k * gridDim.x);
-                if (u >= p.n_items) u = -1;
-                const int qe = int(k % kItemQ);
-                if (k >= uint32_t(kItemQ) &&
-                    !wait_bar(bar_item_empty(qe), ((k / kItemQ) - 1) & 1u, abort_flag, p)) {
-                    ok = false;
-                    break;
-                }
-                item_q[qe] = u;
-                ptx::mbar_arrive(bar_item_full(qe));
-                if (u < 0) break;
-                const WorkItem w = p.items[u];
-                const bool has_b = w.qb >= 0;
-                const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
-                const bool split = has_b && tile_a != tile_b;
-                const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
-                const int32_t* list_a = p.ids + off[tile_a];
-                const int32_t* list_b = p.ids + off[tile_b];
-                const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
-                // query blocks, one buffer per slot
-                if (!wait_bar(bar_q_empty(0), (qc0 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                ptx::mbar_arrive_expect_tx(bar_q_full(0), C::kQBytes);
-                load_block<kRaster>(base + C::kQOff, &tm_q, bar_q_full(0), p, w.bh, tile_a, tile_org<kRaster>(p, tile_a),
-                                    w.qa - tile_a * SPT, C::kColBlocks, C::kBoxBytes);
-                ++qc0;
-                if (has_b) {
-                    if (!wait_bar(bar_q_empty(1), (qc1 & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(bar_q_full(1), C::kQBytes);
-                    load_block<kRaster>(base + C::kQOff + C::kQBytes, &tm_q, bar_q_full(1), p, w.bh, tile_b,
-                                        tile_org<kRaster>(p, tile_b), w.qb - tile_b * SPT, C::kColBlocks,
-                                        C::kBoxBytes);
-                    ++qc1;
-                }
-                // K / V chunks in the order the issuers consume them: chunk kc of
-                // key tile kt is one 128-row block.  The key-tile ids of the next
-                // tile, and in raster layout their origins, are read one tile
-                // ahead so no TMA issue waits on a load.
-                const uint32_t both = has_b ? 3u : 1u;
-                const int32_t n_kt = n_chunks / SPT;
-                int32_t ta = __ldg(list_a), tb = __ldg(list_b);
-                int4 oa = tile_org<kRaster>(p, ta), ob = tile_org<kRaster>(p, tb);
-                for (int32_t kt = 0; ok && kt < n_kt; ++kt) {
-                    const int32_t nta = kt + 1 < n_kt ? __ldg(list_a + kt + 1) : ta;
-                    const int32_t ntb = kt + 1 < n_kt ? __ldg(list_b + kt + 1) : tb;
-                    const int4 noa = tile_org<kRaster>(p, nta), nob = tile_org<kRaster>(p, ntb);
-                    for (int32_t kc = 0; ok && kc < SPT; ++kc) {
-                        if (split) {
-                            ok = issue(&tm_k, w.bh, ta, oa, kc, 1u) && issue(&tm_k, w.bh, tb, ob, kc, 2u) &&
-                                 issue(&tm_v, w.bh, ta, oa, kc, 1u) && issue(&tm_v, w.bh, tb, ob, kc, 2u);
-                        } else {
-                            ok = issue(&tm_k, w.bh, ta, oa, kc, both) && issue(&tm_v, w.bh, ta, oa, kc, both);
-                        }
-                    }
-                    ta = nta;
-                    tb = ntb;
-                    oa = noa;
-                    ob = nob;
-                }
-            }
-            // Drain: the copies issued last into each stage, and the last query loads.
-            const uint32_t first = item > uint32_t(S) ? item - S : 0u;
-            for (uint32_t it = first; it < item; ++it)
-                drain_bar(bar_full(int(it % S)), (it / S) & 1u, p.timeout_ns);
-            if (qc0 > 0) drain_bar(bar_q_full(0), (qc0 - 1) & 1u, p.timeout_ns);
-            if (qc1 > 0) drain_bar(bar_q_full(1), (qc1 - 1) & 1u, p.timeout_ns);
-        }
-    } else if (warp == kMmaWarp0 + 2) {
-        // idle: completes the producer warpgroup for the register hand-over
-        ptx::regs_dec<kRegsProducer>();
-    } else if (warp == kMmaWarp0 || warp == kMmaWarp0 + 1) {
-        ptx::regs_dec<kRegsProducer>();
-        if (lane == 0) {
-            // ------------------------------------------------------------- MMA
-            const int s = warp - kMmaWarp0;  // the query slot this thread serves
-            constexpr uint32_t idesc_qk = ptx::idesc_bf16(128, kChunkKeys, false);
-            constexpr uint32_t idesc_pv = ptx::idesc_bf16(128, D, true);
-            const uint32_t tS = tmem + C::col_s(s), tO = tmem + C::col_o(s);
-            const uint32_t qaddr = base + C::kQOff + s * C::kQBytes;
-            uint32_t item = 0, qc = 0, pc = 0, oc = 0, tc = 0;
-            bool ok = true;
-            for (uint32_t kq = 0; ok; ++kq) {
-                int32_t u;
-                if (!take_item(kq, u)) { ok = false; break; }
-                ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
-                if (u < 0) break;
-                const WorkItem w = p.items[u];
-                const bool has_b = w.qb >= 0;
-                const int32_t tile_a = w.qa / SPT, tile_b = has_b ? w.qb / SPT : tile_a;
-                const bool split = has_b && tile_a != tile_b;
-                const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
-                const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
-                const uint32_t width = split ? 4u : 2u;
-                const uint32_t ubase = item;
-                item += uint32_t(n_chunks) * width;
-                if (s == 1 && !has_b) continue;
-                // ring positions: step i holds [K, V] (shared) or [K_a, K_b, V_a, V_b]
-                const uint32_t k_off = split ? uint32_t(s) : 0u, v_off = split ? 2u + uint32_t(s) : 1u;
-                if (!wait_bar(bar_q_full(s), qc & 1u, abort_flag, p)) { ok = false; break; }
-                ptx::tc_fence_after();
-                // With both slots busy the issuers take turns, one step's batch
-                // [PV_s(i-1), S_s(i)] each: the tensor pipe then runs slot 1's
-                // batch while slot 0's softmax works and the other way round.
-                // Each issuer finishes its own waits before it waits for the turn.
-                const bool turns = has_b;
-                for (int32_t i = 0; ok && i <= n_chunks; ++i) {
-                    const uint32_t v_it = ubase + uint32_t(i - 1) * width + v_off;
-                    const uint32_t k_it = ubase + uint32_t(i) * width + k_off;
-                    // Stage and O waits first: they are normally satisfied while this
-                    // slot's softmax still runs, so only the P wait gates the batch.
-                    if (i < n_chunks && !wait_bar(bar_full(int(k_it % S)), (k_it / S) & 1u, abort_flag, p)) {
-                        ok = false;
-                        break;
-                    }
-                    if (i >= 1) {
-                        if (!wait_bar(bar_full(int(v_it % S)), (v_it / S) & 1u, abort_flag, p)) { ok = false; break; }
-                        if (i == 1 && !wait_bar(bar_o_empty(s), (oc & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
-                        if (!wait_bar(bar_p_full(s), pc & 1u, abort_flag, p)) { ok = false; break; }
-                        ++pc;
-                    }
-                    if (turns) {
-                        if (!wait_bar(bar_turn(s), tc & 1u, abort_flag, p)) { ok = false; break; }
-                        ++tc;
-                    }
-                    ptx::tc_fence_after();
-                    if (i >= 1) {
-                        // O_s += P_s(i-1) V(i-1)
-                        const uint32_t vaddr = base + C::kRingOff + (v_it % S) * C::kKVBytes;
-#pragma unroll
-                        for (int kk = 0; kk < kChunkKeys / 16; ++kk)
-                            ptx::mma_ts(tO, tS + kk * 8, ptx::desc_mn_sw128(vaddr + kk * 16 * 128, C::kBoxBytes),
-                                        idesc_pv, (i > 1 || kk > 0) ? 1u : 0u);
-                    }
-                    if (i < n_chunks) {
-                        // S_s(i) = Q_s K(i)^T; in issue order after PV_s(i-1), which
-                        // reads the P that this S overwrites
-                        const uint32_t kaddr = base + C::kRingOff + (k_it % S) * C::kKVBytes;
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t coff = (kk >> 2) * C::kBoxBytes + (kk & 3) * 32;
-                            ptx::mma_ss(tS, ptx::desc_k_sw128(qaddr + coff), ptx::desc_k_sw128(kaddr + coff),
-                                        idesc_qk, kk > 0 ? 1u : 0u);
-                        }
-                    }
-                    if (turns) ptx::mbar_arrive(bar_turn(1 - s));
-                    if (i < n_chunks) ptx::mma_commit(bar_s_full(s));
-                    if (i >= 1) ptx::mma_commit(bar_empty(int(v_it % S), s));
-                    if (i < n_chunks) {
-                        ptx::mma_commit(bar_empty(int(k_it % S), s));
-                    } else {
-                        ptx::mma_commit(bar_o_full(s));
-                        ++oc;
-                    }
-                }
-                if (!ok) break;
-                ptx::mma_commit(bar_q_empty(s));
-                ++qc;
-            }
-            // Drain: every MMA this thread issued completes before TMEM is freed.
-            ptx::mma_commit(bar_drain(s));
-            drain_bar(bar_drain(s), 0, p.timeout_ns);
-        }
-    } else {
-        // ------------------------------------------------------------- softmax
-        ptx::regs_inc<kRegsSoftmax>();
-        const int slot = warp >> 2;
-        const int row = threadIdx.x & 127;
-        const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_addr + C::col_s(slot);
-        const uint32_t tO = tmem + lane_addr + C::col_o(slot);
-        const float c = p.scale_log2;
-        uint32_t scnt = 0, ocnt = 0;
-        bool ok = true;
-        for (uint32_t kq = 0; ok; ++kq) {
-            int32_t u = -1;
-            if (!__all_sync(0xffffffffu, take_item(kq, u))) {
-                ok = false;
-                break;
-            }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
-            if (u < 0) break;
-            const WorkItem w = p.items[u];
-            if (slot == 1 && w.qb < 0) continue;
-            const int32_t tile_a = w.qa / SPT;
-            const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
-            const int32_t n_chunks = (off[tile_a + 1] - off[tile_a]) * SPT;
-            const int32_t q_blk = slot == 0 ? w.qa : w.qb;
-            const int32_t kbeg = kPadded ? off[q_blk / SPT] : 0;  // this slot's key tiles
-            float m_used = 0.0f, l = 0.0f;
-            for (int32_t i = 0; i < n_chunks; ++i) {
-                if (!__all_sync(0xffffffffu, wait_bar(bar_s_full(slot), scnt & 1u, abort_flag, p))) {
-                    ok = false;
-                    break;
-                }
-                ++scnt;
-                ptx::tc_fence_after();
-                float rowsum;
-                bool rescale = false;
-                float alpha = 1.0f;
-                uint32_t sr[128];
-                const uint4* kmask =
-                    kPadded ? p.key_mask + int64_t(__ldg(p.ids + kbeg + i / SPT)) * SPT + i % SPT : nullptr;
-                ptx::tmem_ld128(tS, sr);
-                bool masked = false;  // warp-uniform: the chunk is one of an edge tile
-                if (kPadded) {
-                    const uint4 m = __ldg(kmask);
-                    masked = (m.x & m.y & m.z & m.w) != ~0u;
-                    if (masked) mask_scores(sr, m);
-                }
-                uint32_t pk[64];
-                if (i == 0) {
-                    // a tile's first chunk holds its first token, a real key: the max is finite
-                    m_used = row_max(sr);
-                    rowsum = softmax_exp(sr, c, m_used, pk);
-                } else {
-                    // Exponentiate against the running max (no max pass: it
-                    // costs an instruction per score pair on the critical
-                    // path); a row whose chunk sum says the max grew is redone
-                    // (rarely) against the chunk's own max (lazy rescale).
-                    rowsum = softmax_exp(sr, c, m_used, pk);
-                    const bool need = !(rowsum <= kRescaleRowSum);  // also catches inf
-                    rescale = __any_sync(0xffffffffu, need);
-                    if (rescale) {
-                        // S is still in TMEM (P has not been written over it yet)
-                        ptx::tmem_ld128(tS, sr);
-                        if (kPadded && masked) mask_scores(sr, __ldg(kmask));
-                        if (need) {
-                            const float mx = row_max(sr);
-                            if ((mx - m_used) * c > 0.0f) {
-                                alpha = ptx::ex2((m_used - mx) * c);
-                                m_used = mx;
-                            }
-                        }
-                        rowsum = softmax_exp(sr, c, m_used, pk);
-                    }
-                }
-                ptx::tmem_st64(tS, pk);
-                l = l * alpha + rowsum;
-                if (rescale) {
-                    // O_s holds P(0..i-1) V: PV_s(i-1) completed before S_s(i) was
-                    // signalled, and PV_s(i) waits for this warpgroup's P signal.
-                    const uint64_t alpha2 = ptx::f2(alpha, alpha);
-#pragma unroll 1
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        uint32_t orr[32];
-                        ptx::tmem_ld32(tO + cb * 32, orr);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            float o0, o1;
-                            ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(orr[2 * j]),
-                                                              __uint_as_float(orr[2 * j + 1])), alpha2),
-                                          o0, o1);
-                            orr[2 * j] = __float_as_uint(o0);
-                            orr[2 * j + 1] = __float_as_uint(o1);
-                        }
-                        ptx::tmem_st32(tO + cb * 32, orr);
-                    }
-                }
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
-                // One arrival per warp: 128 arrivals on one barrier serialise
-                // for hundreds of cycles on the critical path.
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar_p_full(slot));
-            }
-            if (!ok) break;
-            // epilogue: O / l -> bf16, LSE
-            if (!__all_sync(0xffffffffu, wait_bar(bar_o_full(slot), ocnt & 1u, abort_flag, p))) {
-                ok = false;
-                break;
-            }
-            ++ocnt;
-            ptx::tc_fence_after();
-            const float inv_l = 1.0f / l;
-            const int64_t grow = out_row<kRaster, kPadded>(p, w.bh, q_blk, row);
-            uint4* dst = reinterpret_cast<uint4*>(p.o + (grow < 0 ? 0 : grow) * D);
-#pragma unroll 1
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t orr[32];
-                ptx::tmem_ld32(tO + cb * 32, orr);  // every lane loads: the access is warp-wide
-                if (grow >= 0) {                   // a padding row of a raster output stores nothing
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint4 v;
-                        v.x = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 0]) * inv_l, __uint_as_float(orr[8 * j + 1]) * inv_l);
-                        v.y = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 2]) * inv_l, __uint_as_float(orr[8 * j + 3]) * inv_l);
-                        v.z = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 4]) * inv_l, __uint_as_float(orr[8 * j + 5]) * inv_l);
-                        v.w = ptx::pack_bf16x2(__uint_as_float(orr[8 * j + 6]) * inv_l, __uint_as_float(orr[8 * j + 7]) * inv_l);
-                        dst[cb * 4 + j] = v;
-                    }
-                }
-            }
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_o_empty(slot));
-            if (grow >= 0) p.lse[grow] = m_used * p.scale + logf(l);
-        }
-    }
-
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == kMmaWarp0) {
-        __syncwarp();
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, kTmemCols);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -835,8 +320,9 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             // Ring entries in the order the issuing thread consumes them: per
             // block, K(0), K(1), then V(i), K(i + 2) for i = 0, 1, ...
             uint32_t ring = 0;
+            uint32_t q_loads[2] = {0u, 0u};  // query loads issued into each buffer
             bool ok = true;
-            if (p.inject) ok = wait_bar(bar_dead, 0, abort_flag, p);
+            if (p.inject == 1) ok = wait_bar(bar_dead, 0, abort_flag, p);
             auto issue = [&](const CUtensorMap* m, int32_t bh, int32_t tile, int4 org, int32_t sub) -> bool {
                 const int r = int(ring % S);
                 if (ring >= uint32_t(S) && !wait_bar(bar_empty(r), ((ring / S) - 1) & 1u, abort_flag, p))
@@ -871,6 +357,7 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 ptx::mbar_arrive_expect_tx(bar_q_full(qb), C::kQBytes);
                 load_block<kRaster>(base + C::kQOff + qb * C::kQBytes, &tm_q, bar_q_full(qb), p, w.bh, tile_q,
                                     tile_org<kRaster>(p, tile_q), w.qa - tile_q * SPT, C::kColBlocks, C::kBoxBytes);
+                ++q_loads[qb];
                 // chunk c of the list is block c % SPT of key tile list[c / SPT]
                 auto load_chunk = [&](const CUtensorMap* m, int32_t c) -> bool {
                     const int32_t kt = __ldg(list + c / SPT);
@@ -882,9 +369,14 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     if (ok && i + 2 < n) ok = load_chunk(&tm_k, i + 2);
                 }
             }
+            // Drain before exit (after an abort some copies may still be in
+            // flight): the last copy into each ring stage and the last query
+            // block loaded into each buffer.
             const uint32_t first = ring > uint32_t(S) ? ring - S : 0u;
             for (uint32_t it = first; it < ring; ++it)
                 drain_bar(bar_full(int(it % S)), (it / S) & 1u, p.timeout_ns);
+            for (int b = 0; b < 2; ++b)
+                if (q_loads[b] > 0) drain_bar(bar_q_full(b), (q_loads[b] - 1u) & 1u, p.timeout_ns);
         }
     } else if (warp == kMmaWarp0 + 2) {
         ptx::regs_dec<kRegsProducer>();  // idle: completes the producer warpgroup for the register hand-over
@@ -952,6 +444,13 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 } else {
                     const int qb = int(kq & 1u);
                     const uint32_t qaddr = base + C::kQOff + qb * C::kQBytes;
+                    if (p.inject == 2 && kq == 1u) {
+                        // Debug: wait on a barrier nothing arrives at; the limit runs out
+                        // while this item's loads are issued and nothing consumes them.
+                        wait_bar(bar_dead, 0, abort_flag, p);
+                        ok = false;
+                        break;
+                    }
                     if (!wait_bar(bar_q_full(qb), (kq >> 1) & 1u, abort_flag, p)) { ok = false; break; }
                     for (uint32_t c = 0; ok && c < n; ++c) {
                         const uint32_t gc = g0 + c, bb = gc & 1u, e = e0 + entry_k(c);
@@ -1194,16 +693,6 @@ cudaError_t make_map(CUtensorMap* m, const void* ptr, int64_t rows, int d) {
 }
 
 template <int D, bool kRaster, bool kPadded>
-cudaError_t launch_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
-                          const CUtensorMap& mv, const FwdParams& fp) {
-    cudaError_t e = cudaFuncSetAttribute(sta_fwd_kernel<D, kRaster, kPadded>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    sta_fwd_kernel<D, kRaster, kPadded><<<grid, kThreads, Cfg<D>::kSmemBytes, stream>>>(mq, mk, mv, fp);
-    return cudaGetLastError();
-}
-
-template <int D, bool kRaster, bool kPadded>
 cudaError_t launch_split_kernel(int grid, cudaStream_t stream, const CUtensorMap& mq, const CUtensorMap& mk,
                                 const CUtensorMap& mv, const FwdParams& fp) {
     constexpr int kSmem = split::Cfg<D>::kSmemBytes;
@@ -1237,9 +726,10 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
         if (e == cudaSuccess) e = make_map(&mv, v, rows, D);
     }
     if (e != cudaSuccess) return e;
-    FwdParams fp;
-    fp.items = pl->d_items;
-    fp.n_items = int32_t(P.items.size());
+    // One-block work items, longest key lists first.
+    FwdParams fp{};
+    fp.items = pl->d_f1_items;
+    fp.n_items = int32_t(P.f1_items.size());
     fp.off = pl->d_off;
     fp.ids = pl->d_ids;
     fp.tiles_per_head = P.tiles_per_head;
@@ -1259,10 +749,6 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    // The key-split kernel over one-block items (with per-chunk key masks on
-    // padded latents).
-    fp.items = pl->d_f1_items;
-    fp.n_items = int32_t(P.f1_items.size());
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
     fp.item_counter = pl->d_counters + pl->launch_seq.fetch_add(1) % uint32_t(kCounterPool);
@@ -1314,6 +800,7 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     FwdParams fp{};
     fp.items = pv.items;
     fp.n_items = pv.n_items;
+    fp.item_counter = pv.item_counter;
     fp.off = pv.off;
     fp.ids = pv.ids;
     fp.tiles_per_head = pv.tiles_per_head;
@@ -1333,8 +820,8 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     if (e != cudaSuccess) return e;
     const int grid = fp.n_items < sms ? fp.n_items : sms;
     if (grid <= 0) return cudaSuccess;
-    if (head_dim == 128) return launch_kernel<128, false, false>(grid, stream, mq, mk, mv, fp);
-    return launch_kernel<64, false, false>(grid, stream, mq, mk, mv, fp);
+    if (head_dim == 128) return launch_split_kernel<128, false, false>(grid, stream, mq, mk, mv, fp);
+    return launch_split_kernel<64, false, false>(grid, stream, mq, mk, mv, fp);
 }
 
 }  // namespace sta

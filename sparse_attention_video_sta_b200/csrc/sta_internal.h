@@ -21,13 +21,12 @@ constexpr int kChunkKeys = 128;
 // Device status bits written by kernels (OR-ed).
 constexpr uint32_t kDevTimeout = 1u;
 
-// One work item of the forward kernel: up to two 128-row query blocks of the
-// same (b, h), each with its own key-tile list.  qb < 0 means one block only.
-// When both blocks belong to the same tile they share every K/V load.
+// One work item of the forward and backward kernels: one 128-row block of
+// one (b, h) (a query block, or a key block for the dK / dV kernel).
 struct WorkItem {
     int32_t bh;   // b * heads + h
-    int32_t qa;   // query row block within the head: tile * sub_per_tile + sub
-    int32_t qb;   // second row block or -1
+    int32_t qa;   // row block within the head: tile * sub_per_tile + sub
+    int32_t qb;   // unused, -1
     int32_t win;  // distinct-window id of head h
 };
 static_assert(sizeof(WorkItem) == 16, "WorkItem is loaded as one int4");
@@ -43,7 +42,6 @@ struct PlanHost {
     std::vector<int32_t> win_ext;            // [n_win][3] clamped extents in tiles
     std::vector<int32_t> csr_off;            // [n_win][tiles_per_head + 1], global offsets
     std::vector<int32_t> csr_ids;            // key-tile ids, ascending per list
-    std::vector<WorkItem> items;             // forward work list (two-block items)
     std::vector<WorkItem> f1_items;          // forward work list of one-block items, longest lists first
     // Backward: for each key tile the query tiles whose window holds it
     // (the forward lists transposed), and one-block work lists for the dQ
@@ -66,7 +64,6 @@ struct sta_plan_s {
     int device = -1;
     int32_t* d_off = nullptr;
     int32_t* d_ids = nullptr;
-    sta::WorkItem* d_items = nullptr;
     sta::WorkItem* d_f1_items = nullptr;
     uint32_t* d_status = nullptr;
     int32_t* d_origin = nullptr;  // device copy of tile_origin (16-byte rows)
@@ -106,8 +103,9 @@ cudaError_t launch_forward(const sta_plan_s* p, const void* q, const void* k, co
 // (used by the no-allocation entry point, sta_noalloc.cu).
 struct RawPlanView {
     int32_t batch, heads, tiles_per_head, tile_tokens, sub_per_tile;
-    const WorkItem* items;
+    const WorkItem* items;  // one-block items
     int32_t n_items;
+    int32_t* item_counter;  // zero before the launch (the run-time item hand-out)
     const int32_t* off;
     const int32_t* ids;
     uint32_t* status;

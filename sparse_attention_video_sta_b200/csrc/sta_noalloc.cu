@@ -12,14 +12,15 @@
 // The scratch is a file-scope __device__ array (every GPU that loads the library
 // holds it until the process exits).  Host code cannot use its name as a device
 // address, so its address is looked up once per device with
-// cudaGetSymbolAddress and passed to the kernel.  The plan is written into a
-// static host staging buffer (no heap use) and copied into the scratch on the
-// caller's stream; that copy also zeroes the kernel's status word.
+// cudaGetSymbolAddress and passed to the kernels.  Each call first runs a small
+// kernel that writes the plan into the scratch -- key-tile lists, work list,
+// a zeroed status word and work counter -- from the per-head windows it takes
+// as a kernel parameter, then the forward kernel over that plan.  No host
+// buffer is copied to the device.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
-#include <cstring>
 #include <mutex>
 
 #include "sta.h"
@@ -30,10 +31,24 @@ namespace {
 using sta::WorkItem;
 
 constexpr size_t kScratchBytes = size_t(4) << 20;  // 4 MiB
-constexpr size_t kHeaderBytes = 256;               // status word, padded
+constexpr size_t kHeaderBytes = 256;               // status word, work counter, padding
 constexpr int kMaxHeads = 1024;
 constexpr int kMaxDevices = 64;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanBlocks = 64;
+
+// The problem, passed by value to the plan-writing kernel (about 6 KB of
+// kernel parameters: no host-to-device copy is needed).
+struct PlanArgs {
+    int32_t batch, heads;
+    int32_t n[3];             // tile grid
+    int32_t sub_per_tile;     // 128-row blocks per tile
+    int32_t tiles;            // tiles per head
+    int32_t n_win;            // distinct clamped windows
+    uint32_t items_at, off_at, ids_at;  // byte offsets in the scratch
+    uint16_t ext[kMaxHeads][3];         // clamped window extent of each head, in tiles
+};
 
 }  // namespace
 
@@ -42,16 +57,113 @@ static __device__ __align__(256) uint8_t g_scratch[kScratchBytes];
 
 namespace {
 
-alignas(256) uint8_t g_staging[kScratchBytes];  // host-side image of the scratch
-std::mutex g_mutex;                             // guards g_staging and g_scratch_ptr
-void* g_scratch_ptr[kMaxDevices] = {};
-
-int32_t window_start(int32_t q, int32_t e, int32_t n) {
+__device__ __forceinline__ int32_t window_start_dev(int32_t q, int32_t e, int32_t n) {
     int32_t s = q - e / 2;
-    if (s < 0) s = 0;
-    if (s > n - e) s = n - e;
-    return s;
+    s = s < 0 ? 0 : s;
+    return s > n - e ? n - e : s;
 }
+
+// Writes the plan of one call into the scratch (every CTA derives the same
+// per-head tables, then writes its share of the arrays):
+//   - distinct windows in order of first appearance among the heads, each with
+//     the ascending key-tile list of every query tile (CSR, the same lists as
+//     sta_plan's);
+//   - one work item per (b, h, 128-row block), ordered by descending list
+//     length, then b, then h (the order sta_plan gives);
+//   - the status word and the work counter, zeroed.
+__global__ void __launch_bounds__(kPlanThreads) noalloc_plan_kernel(const PlanArgs a, uint8_t* scratch) {
+    __shared__ int32_t s_vol[kMaxHeads];   // list length of each head's window
+    __shared__ int32_t s_first[kMaxHeads]; // first head with the same window
+    __shared__ int32_t s_win[kMaxHeads];   // distinct-window id of each head
+    __shared__ int32_t s_rank[kMaxHeads];  // (b, h) order: heads with longer lists, same-length heads
+    __shared__ int32_t s_eq[kMaxHeads];    // heads with the same list length
+    __shared__ int32_t s_wbase[kMaxHeads + 1];  // CSR start of each distinct window (in ids)
+    __shared__ int32_t s_whead[kMaxHeads];      // a head of each distinct window
+    const int H = a.heads;
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        s_vol[h] = int32_t(a.ext[h][0]) * a.ext[h][1] * a.ext[h][2];
+        int32_t f = h;
+        for (int g = 0; g < h; ++g)
+            if (a.ext[g][0] == a.ext[h][0] && a.ext[g][1] == a.ext[h][1] && a.ext[g][2] == a.ext[h][2]) {
+                f = g;
+                break;
+            }
+        s_first[h] = f;
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
+        int32_t id = 0, gt = 0, eq = 0, eqlt = 0;
+        for (int g = 0; g < H; ++g) {
+            if (g < s_first[h] && s_first[g] == g) ++id;
+            gt += s_vol[g] > s_vol[h];
+            eq += s_vol[g] == s_vol[h];
+            eqlt += (g < h) && s_vol[g] == s_vol[h];
+        }
+        s_win[h] = id;
+        s_rank[h] = gt * a.batch + eqlt;  // + b * eq for batch b
+        s_eq[h] = eq;
+        if (s_first[h] == h) s_whead[id] = h;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int w = 0; w < a.n_win; ++w) {
+            s_wbase[w] = acc;
+            acc += a.tiles * s_vol[s_whead[w]];
+        }
+        s_wbase[a.n_win] = acc;
+    }
+    __syncthreads();
+
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t tid = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (tid == 0) {
+        reinterpret_cast<uint32_t*>(scratch)[0] = 0u;  // status word
+        reinterpret_cast<int32_t*>(scratch)[1] = 0;    // work counter
+    }
+    // CSR offsets: window w's list of query tile q starts at base(w) + q vol(w).
+    int32_t* off = reinterpret_cast<int32_t*>(scratch + a.off_at);
+    const int64_t n_off = int64_t(a.n_win) * (a.tiles + 1);
+    for (int64_t i = tid; i < n_off; i += stride) {
+        const int32_t w = int32_t(i / (a.tiles + 1)), q = int32_t(i % (a.tiles + 1));
+        off[i] = s_wbase[w] + q * s_vol[s_whead[w]];
+    }
+    // Key-tile ids: entry j of query tile q's list, raster order over the
+    // window's (t, h, w) offsets, which is ascending tile id.
+    int32_t* ids = reinterpret_cast<int32_t*>(scratch + a.ids_at);
+    const int64_t n_ids = s_wbase[a.n_win];
+    for (int64_t i = tid; i < n_ids; i += stride) {
+        int32_t lo = 0, hi = a.n_win - 1;  // the window holding entry i
+        while (lo < hi) {
+            const int32_t mid = (lo + hi + 1) >> 1;
+            if (s_wbase[mid] <= i) lo = mid; else hi = mid - 1;
+        }
+        const int32_t hw = s_whead[lo];
+        const int32_t e0 = a.ext[hw][0], e1 = a.ext[hw][1], e2 = a.ext[hw][2];
+        const int32_t vol = e0 * e1 * e2;
+        const int32_t r = int32_t(i - s_wbase[lo]);
+        const int32_t q = r / vol, j = r % vol;
+        const int32_t qw = q % a.n[2], qh = (q / a.n[2]) % a.n[1], qt = q / (a.n[2] * a.n[1]);
+        const int32_t jw = j % e2, jh = (j / e2) % e1, jt = j / (e2 * e1);
+        const int32_t kt = window_start_dev(qt, e0, a.n[0]) + jt;
+        const int32_t kh = window_start_dev(qh, e1, a.n[1]) + jh;
+        const int32_t kw = window_start_dev(qw, e2, a.n[2]) + jw;
+        ids[i] = (kt * a.n[1] + kh) * a.n[2] + kw;
+    }
+    // Work items: (b, h) groups in descending list length, then b, then h.
+    WorkItem* items = reinterpret_cast<WorkItem*>(scratch + a.items_at);
+    const int32_t per_head = a.tiles * a.sub_per_tile;
+    const int64_t n_items = int64_t(a.batch) * H * per_head;
+    for (int64_t i = tid; i < n_items; i += stride) {
+        const int32_t bh = int32_t(i / per_head), blk = int32_t(i % per_head);
+        const int32_t b = bh / H, h = bh % H;
+        const int64_t rank = int64_t(s_rank[h]) + int64_t(b) * s_eq[h];
+        items[rank * per_head + blk] = WorkItem{bh, blk, -1, s_win[h]};
+    }
+}
+
+std::mutex g_mutex;  // guards g_scratch_ptr
+void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_scratch on the current device (looked up once per device).
 cudaError_t scratch_ptr(void** out) {
@@ -59,6 +171,7 @@ cudaError_t scratch_ptr(void** out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
     if (g_scratch_ptr[dev] == nullptr) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_scratch);
@@ -93,6 +206,7 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
         }
     if (head_dim != 64 && head_dim != 128) return STA_ERR_UNSUPPORTED;
     if (heads > kMaxHeads) return STA_ERR_UNSUPPORTED;
+    if (n[0] > 65535 || n[1] > 65535 || n[2] > 65535) return STA_ERR_UNSUPPORTED;
     const int64_t n_tok = int64_t(L[0]) * L[1] * L[2];
     const int32_t tile_tokens = T[0] * T[1] * T[2];
     if (tile_tokens % sta::kSubRows != 0) return STA_ERR_UNSUPPORTED;
@@ -106,103 +220,50 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
     const int32_t tiles = n[0] * n[1] * n[2];
     const int32_t S = tile_tokens / sta::kSubRows;
 
-    // ---- distinct clamped windows, longest lists first (no heap: fixed arrays)
-    static int32_t head_win[kMaxHeads];
-    static int32_t win_e[kMaxHeads][3];
-    static int32_t order[kMaxHeads];
-    std::lock_guard<std::mutex> lock(g_mutex);
+    // ---- clamped windows; distinct ones counted for the scratch layout
+    PlanArgs a;
+    a.batch = batch;
+    a.heads = heads;
+    for (int d = 0; d < 3; ++d) a.n[d] = n[d];
+    a.sub_per_tile = S;
+    a.tiles = tiles;
     int32_t n_win = 0;
-    for (int32_t h = 0; h < heads; ++h) {
-        int32_t e[3];
-        for (int d = 0; d < 3; ++d) {
-            e[d] = window_thw[3 * h + d] / T[d];
-            if (e[d] > n[d]) e[d] = n[d];
-        }
-        int32_t id = -1;
-        for (int32_t w = 0; w < n_win && id < 0; ++w)
-            if (win_e[w][0] == e[0] && win_e[w][1] == e[1] && win_e[w][2] == e[2]) id = w;
-        if (id < 0) {
-            id = n_win++;
-            for (int d = 0; d < 3; ++d) win_e[id][d] = e[d];
-        }
-        head_win[h] = id;
-    }
-    for (int32_t w = 0; w < n_win; ++w) order[w] = w;
-    auto vol = [&](int32_t w) { return win_e[w][0] * win_e[w][1] * win_e[w][2]; };
-    for (int32_t i = 1; i < n_win; ++i)  // insertion sort, descending list length, stable
-        for (int32_t j = i; j > 0 && vol(order[j]) > vol(order[j - 1]); --j) {
-            const int32_t t = order[j];
-            order[j] = order[j - 1];
-            order[j - 1] = t;
-        }
-
-    // ---- sizes and layout of the scratch image
-    const int64_t items_per_head = int64_t(tiles) * (S / 2) + ((S % 2) ? (tiles + 1) / 2 : 0);
-    const int64_t n_items = items_per_head * heads * batch;
     int64_t n_ids = 0;
-    for (int32_t w = 0; w < n_win; ++w) n_ids += int64_t(tiles) * vol(w);
+    for (int32_t h = 0; h < heads; ++h) {
+        for (int d = 0; d < 3; ++d) {
+            const int32_t e = window_thw[3 * h + d] / T[d];
+            a.ext[h][d] = uint16_t(e < n[d] ? e : n[d]);
+        }
+        bool seen = false;
+        for (int32_t g2 = 0; g2 < h && !seen; ++g2)
+            seen = a.ext[g2][0] == a.ext[h][0] && a.ext[g2][1] == a.ext[h][1] && a.ext[g2][2] == a.ext[h][2];
+        if (!seen) {
+            ++n_win;
+            n_ids += int64_t(tiles) * a.ext[h][0] * a.ext[h][1] * a.ext[h][2];
+        }
+    }
+    a.n_win = n_win;
+
+    // ---- sizes and layout of the scratch
+    const int64_t n_items = int64_t(batch) * heads * tiles * S;
     const int64_t n_off = int64_t(n_win) * (tiles + 1);
     const size_t items_at = kHeaderBytes;
     const size_t off_at = items_at + size_t(n_items) * sizeof(WorkItem);
     const size_t ids_at = off_at + size_t(n_off) * sizeof(int32_t);
     const size_t total = ids_at + size_t(n_ids) * sizeof(int32_t);
     if (total > kScratchBytes || n_items > INT32_MAX) return STA_ERR_UNSUPPORTED;
+    a.items_at = uint32_t(items_at);
+    a.off_at = uint32_t(off_at);
+    a.ids_at = uint32_t(ids_at);
 
-    // ---- write the plan into the host staging image
-    std::memset(g_staging, 0, kHeaderBytes);  // status word starts at zero
-    int32_t* off = reinterpret_cast<int32_t*>(g_staging + off_at);
-    int32_t* ids = reinterpret_cast<int32_t*>(g_staging + ids_at);
-    int32_t pos = 0;
-    for (int32_t w = 0; w < n_win; ++w) {
-        const int32_t* e = win_e[w];
-        for (int32_t qt = 0; qt < n[0]; ++qt)
-            for (int32_t qh = 0; qh < n[1]; ++qh)
-                for (int32_t qw = 0; qw < n[2]; ++qw) {
-                    off[int64_t(w) * (tiles + 1) + (qt * n[1] + qh) * n[2] + qw] = pos;
-                    const int32_t st = window_start(qt, e[0], n[0]);
-                    const int32_t sh = window_start(qh, e[1], n[1]);
-                    const int32_t sw = window_start(qw, e[2], n[2]);
-                    for (int32_t kt = st; kt < st + e[0]; ++kt)
-                        for (int32_t kh = sh; kh < sh + e[1]; ++kh)
-                            for (int32_t kw = sw; kw < sw + e[2]; ++kw)
-                                ids[pos++] = (kt * n[1] + kh) * n[2] + kw;
-                }
-        off[int64_t(w) * (tiles + 1) + tiles] = pos;
-    }
-    WorkItem* items = reinterpret_cast<WorkItem*>(g_staging + items_at);
-    int64_t it = 0;
-    for (int32_t oi = 0; oi < n_win; ++oi) {
-        const int32_t w = order[oi];
-        for (int32_t b = 0; b < batch; ++b)
-            for (int32_t h = 0; h < heads; ++h) {
-                if (head_win[h] != w) continue;
-                const int32_t bh = b * heads + h;
-                int32_t pending = -1;
-                for (int32_t t = 0; t < tiles; ++t) {
-                    for (int32_t s = 0; s + 1 < S; s += 2) items[it++] = WorkItem{bh, t * S + s, t * S + s + 1, w};
-                    if (S % 2 == 1) {
-                        const int32_t blk = t * S + S - 1;
-                        if (pending < 0) {
-                            pending = blk;
-                        } else {
-                            items[it++] = WorkItem{bh, pending, blk, w};
-                            pending = -1;
-                        }
-                    }
-                }
-                if (pending >= 0) items[it++] = WorkItem{bh, pending, -1, w};
-            }
-    }
-    if (it != n_items) return STA_ERR_UNSUPPORTED;  // cannot happen: sizes above match the loops
-
-    // ---- copy into the device scratch and launch
+    // ---- write the plan into the scratch on the stream, then launch the forward
     void* base = nullptr;
     if (scratch_ptr(&base) != cudaSuccess) return STA_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // Returns once the pageable staging image has been taken; the transfer is
-    // ordered on `s` before the kernel.
-    if (cudaMemcpyAsync(base, g_staging, total, cudaMemcpyHostToDevice, s) != cudaSuccess) return STA_ERR_CUDA;
     uint8_t* dev = static_cast<uint8_t*>(base);
+    (void)cudaGetLastError();  // a status describes this call only
+    noalloc_plan_kernel<<<kPlanBlocks, kPlanThreads, 0, s>>>(a, dev);
+    if (cudaGetLastError() != cudaSuccess) return STA_ERR_CUDA;
     sta::RawPlanView pv;
     pv.batch = batch;
     pv.heads = heads;
@@ -211,6 +272,7 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
     pv.sub_per_tile = S;
     pv.items = reinterpret_cast<const WorkItem*>(dev + items_at);
     pv.n_items = int32_t(n_items);
+    pv.item_counter = reinterpret_cast<int32_t*>(dev + 4);
     pv.off = reinterpret_cast<const int32_t*>(dev + off_at);
     pv.ids = reinterpret_cast<const int32_t*>(dev + ids_at);
     pv.status = reinterpret_cast<uint32_t*>(dev);

@@ -89,6 +89,8 @@ def test_calls_rejected_before_launch():
     assert lib.sta_forward(None, a, a, a, a, a, 64, 0.125, None) == INV
     assert lib.sta_last_device_status(hp.handle, None) == INV
     assert lib.sta_debug_inject_timeout(1, 0) == INV
+    assert lib.sta_debug_inject_timeout(3, 30) == INV
+    assert lib.sta_debug_inject_timeout(-1, 30) == INV
     assert lib.sta_plan_query(hp.handle, 2, 0, None, 0, ctypes.byref(ctypes.c_int32())) == INV
     assert lib.sta_plan_query(hp.handle, 0, 27, None, 0, ctypes.byref(ctypes.c_int32())) == INV
     hp.destroy()

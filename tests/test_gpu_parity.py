@@ -179,6 +179,31 @@ def test_device_timeout_is_reported_and_context_survives(sta):
     assert torch.equal(o2, o_ok) and torch.equal(l2, l_ok)
 
 
+def test_timeout_with_copies_in_flight_is_reported_and_next_call_is_clean(sta):
+    """A wait runs out at each CTA's second work item, after the first item
+    was computed and the second item's query block and K/V chunks were issued:
+    the kernel drains those copies and its MMAs and exits.  The status is
+    TIMEOUT, and the next call gives the same bits as a clean one."""
+    latent, tile, B, H, d = (30, 48, 80), (6, 8, 8), 1, 2, 128
+    N = latent[0] * latent[1] * latent[2]
+    g = torch.Generator(device="cuda").manual_seed(909)
+    q, k, v = (torch.randn(B, H, N, d, generator=g, device="cuda").to(torch.bfloat16) for _ in range(3))
+    plan = sta.sta_plan(latent, tile, B, H, [(18, 24, 24), (30, 40, 40)])
+    assert plan.stats()[1] >= 2 * 148  # every CTA takes a second item
+    for fused in (True, False):
+        o_ok, l_ok = sta.sta_attention(q, k, v, plan, fused=fused)
+        assert sta.sta_last_device_status(plan) == 0
+        sta.sta_debug_inject_timeout(2, 30)
+        try:
+            sta.sta_attention(q, k, v, plan, fused=fused)
+            assert sta.sta_last_device_status(plan) == sta.STA_ERR_TIMEOUT
+        finally:
+            sta.sta_debug_inject_timeout(0, 30)
+        o2, l2 = sta.sta_attention(q, k, v, plan, fused=fused)
+        assert sta.sta_last_device_status(plan) == 0
+        assert torch.equal(o2, o_ok) and torch.equal(l2, l_ok)
+
+
 def test_shape_mismatch_rejected_before_launch(sta):
     plan = sta.sta_plan((18, 24, 24), (6, 8, 8), 1, 2, [(12, 16, 16)] * 2)
     q = torch.zeros(1, 2, 10368, 64, dtype=torch.bfloat16, device="cuda")

@@ -6,7 +6,8 @@ keeps its own running maximum m, row sum l and output accumulator O in fp32:
 its first chunk sets m (a stand-in 0 when that chunk holds padding keys
 only), later chunks are exponentiated against m, and a chunk whose row sum
 exceeds 256 is redone against its own maximum with O and l rescaled (lazy
-rescale).  P is rounded to bf16 before P V.  The epilogue merges the halves
+rescale).  P is rounded to bf16 before P V, and the row sum l adds those
+rounded values.  The epilogue merges the halves
 (m = max of the two, each side scaled by 2^((m_h - m) c); a half that met no
 real key has l = 0 and drops out) and writes O / l in bf16 and LSE.
 
@@ -80,14 +81,14 @@ def emulate_block(qr, k, v, key_tiles, latent, tile, scale):
                 else:
                     with np.errstate(over="ignore"):  # inf here is caught by the row-sum test
                         p = np.exp2(s * c - m[:, None] * c).astype(np.float32)
-                    need = ~(p.sum(axis=1, dtype=np.float32) <= RESCALE_ROW_SUM)
+                    need = ~(bf16(p).sum(axis=1, dtype=np.float32) <= RESCALE_ROW_SUM)
                     if need.any():  # warp-uniform in the kernel; per row here, same result
                         mx = s.max(axis=1)
                         grow = need & ((mx - m) * c > 0)
                         alpha = np.exp2(np.where(grow, (m - mx) * c, 0.0)).astype(np.float32)
                         m = np.where(grow, mx, m).astype(np.float32)
                         p = np.exp2(s * c - m[:, None] * c).astype(np.float32)
-                rowsum = p.sum(axis=1, dtype=np.float32)
+                rowsum = bf16(p).sum(axis=1, dtype=np.float32)  # the bf16 values P V multiplies
                 o = o * alpha[:, None] + bf16(p) @ bf16(vv)
                 l = l * alpha + rowsum
         halves.append((m, l, o))
