@@ -44,10 +44,6 @@ constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsProducer = 88;
 static_assert(128 * (2 * kRegsSoftmax + kRegsProducer) <= kThreads * 168, "register split exceeds the launch");
 constexpr uint32_t kTmemCols = 512;
-// Lazy rescale: a chunk is exponentiated against the running max; only a row
-// whose chunk sum exceeds this (its max grew by more than 2^8, or many scores
-// grew a little) is redone against its own max, with O and l rescaled.
-constexpr float kRescaleRowSum = 256.0f;
 
 // Work items are handed out at run time: the load warp takes the next item
 // index from a global counter and passes it to the other roles through a
@@ -176,37 +172,51 @@ __device__ __forceinline__ float row_max64(const uint32_t (&sr)[64]) {
 // Key-split forward kernel.
 //
 // One work item is one 128-row query block.  Every 128-key chunk is split in
-// two halves of 64 keys: softmax warpgroup A (warps 0-3) owns keys 0-63 of each
-// chunk, warpgroup B (warps 4-7) keys 64-127, each with its own running max,
-// row sum and output accumulator (O_A, O_B in TMEM), merged once per block in
-// the epilogue (the usual combination of partial softmaxes).  Both halves'
+// two halves of 64 keys: softmax warpgroup A (warps 0-3) exponentiates keys
+// 0-63 of each chunk, warpgroup B (warps 4-7) keys 64-127, so both halves'
 // exponentials run at once, two warps per SM sub-partition, which keeps the
-// MUFU pipe busier than one warp can (measured: 0.91 of its rate against 0.82).
-// S is double buffered in TMEM, so while the softmax works on chunk g the
-// tensor pipe already holds the scores of chunk g + 1.
+// MUFU pipe busier than one warp can (measured: 0.91 of its rate against
+// 0.82).  The two warps that own the same 32 rows (warp w of A, warp w + 4 of
+// B) keep one running maximum per row between them, so both halves' P V
+// products accumulate into one O; each keeps its own row sum, added in the
+// epilogue.  S is triple buffered in TMEM: the S of chunk c + 3 only waits for
+// the P V of chunk c, whose P it overwrites, so the tensor pipe runs up to
+// three chunks ahead of the softmax.
 //
 //   warp 8 (load)   : TMA loads of the query block (two buffers: the next
 //                     block's query loads while the current one runs) and of
-//                     K(0), K(1), then V(i), K(i + 2) for i = 0, 1, ... into the
-//                     ring, the order in which they are consumed
-//   warp 9 (PV)     : O_h += P_h V_h (keys 64 h .. 64 h + 63) as soon as half
-//                     h's P is in TMEM
-//   warp 10 (S)     : S(c) = Q K(c)^T into buffer c % 2, once the PVs of chunk
-//                     c - 2, which read that buffer, have completed
+//                     K(0), K(1), K(2), then V(i), K(i + 3) for i = 0, 1, ...
+//                     into the ring, the order in which they are consumed
+//   warp 9 (PV)     : O += P_A V_A, then O += P_B V_B (keys 64 h .. 64 h + 63
+//                     of the chunk) as each half's P lands in TMEM
+//   warp 10 (S)     : S(c) = Q K(c)^T into buffer c % 3, once the PVs of chunk
+//                     c - 3, which read that buffer, have completed
 //   warps 0-7       : softmax halves and the epilogue
 //
-// TMEM (512 columns): S0 | S1 | O_A | O_B (d = 128).  P_A (bf16) is written
-// over the first 32 columns of its half of S, P_B over the first 32 of its.
-// The epilogue exchanges the halves' running max and sum through the query
-// buffer of the finished block.  Padded latents (kPadded): each half masks
-// its padding keys from the chunk's real-key bits, and a half that meets no
-// real key in the whole block (a block whose key tiles are all edge tiles)
-// keeps l = 0 and drops out of the merge.  The two-slot kernel's ping-pong needed the
-// chain [PV, S] batch -> softmax -> P to fit in two batches; here the softmax
-// of chunk g + 1 only needs S(g + 1), issued a chunk earlier.
+// TMEM (512 columns): S0 | S1 | S2 | O (d = 128).  P_A (bf16) is written over
+// the first 32 columns of its half of S, P_B over the first 32 of its.
+//
+// Shared running maximum.  A chunk is exponentiated against the row's running
+// maximum m without a max pass; the warp pair meets once per chunk on a named
+// barrier whose reduction says whether either warp needs the slow path: the
+// block's first chunk (m is set from both halves' maxima), a chunk whose
+// half-row sum exceeds kRescaleRowSum (m is raised to the maximum of both
+// halves' scores, and O and both row sums are rescaled, each half rescaling
+// its own half of O's columns), or an abort (both warps leave together, so
+// neither is left waiting at a later barrier).  Row sums add the bf16 P values
+// (see softmax_exp64).  Padded latents (kPadded): each half masks its padding
+// keys from the chunk's real-key bits; a first chunk without a real key in
+// either half starts from a finite stand-in maximum of 0, which the rescale
+// moves once real keys arrive.
 namespace split {
 
 constexpr int kItemConsumers = 2 + 8;  // the two issuing threads and the eight softmax warps
+constexpr int kSBufs = 3;              // S buffers in TMEM
+// A half-row sum above this (the scores grew far past the running maximum,
+// or an exponential overflowed) takes the slow path.  The sums add bf16 P
+// values, whose rounding is relative, so P far above 1 costs no accuracy;
+// the bound only keeps O and l far from fp32 overflow.
+constexpr float kRescaleRowSum = 65536.0f;
 
 template <int D>
 struct Cfg {
@@ -218,14 +228,16 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kRingOff = 2 * kQBytes;
     static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
-    // full[S], empty[S], q_full[2], q_empty[2], s_full[2], p_full[2][2], pv_buf[2], pv_done,
-    // o_full, o_empty, xch[4], dead, drain[2], item_full[Q], item_empty[Q]
-    static constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 4 + 2 + 1 + 1 + 1 + 4 + 1 + 2 + 2 * kItemQ;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    // full[S], empty[S], q_full[2], q_empty[2], s_full[3], p_full[2][3], pv_buf[3],
+    // o_full, o_empty, dead, drain[2], item_full[Q], item_empty[Q]
+    static constexpr int kNumBars = 2 * kStages + 2 + 2 + kSBufs + 2 * kSBufs + kSBufs + 1 + 1 + 1 + 2 +
+                                    2 * kItemQ;
+    static constexpr int kXchOff = kBarOff + kNumBars * 8;  // [2 halves][128 rows] fp32 exchange
+    static constexpr int kMiscOff = kXchOff + 2 * kSubRows * 4;  // tmem base slot, abort flag, item queue
     static constexpr int kSmemBytes = kMiscOff + 8 + 4 * kItemQ + 1024;
     __host__ __device__ static constexpr uint32_t col_s(int buf) { return uint32_t(buf) * 128u; }
-    __host__ __device__ static constexpr uint32_t col_o(int half) { return 256u + uint32_t(half) * D; }
-    static_assert(256 + 2 * D <= int(kTmemCols), "TMEM budget");
+    static constexpr uint32_t kColO = kSBufs * 128u;
+    static_assert(kSBufs * 128 + D <= int(kTmemCols), "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -246,21 +258,22 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
     const uint32_t bar0 = base + C::kBarOff;
     constexpr int S = C::kStages;
+    constexpr int NB = kSBufs;
     auto bar_full = [&](int r) { return bar0 + 8u * r; };
     auto bar_empty = [&](int r) { return bar0 + 8u * (S + r); };
     auto bar_q_full = [&](int b) { return bar0 + 8u * (2 * S + b); };
     auto bar_q_empty = [&](int b) { return bar0 + 8u * (2 * S + 2 + b); };
     auto bar_s_full = [&](int b) { return bar0 + 8u * (2 * S + 4 + b); };
-    auto bar_p_full = [&](int h, int b) { return bar0 + 8u * (2 * S + 6 + 2 * h + b); };
-    auto bar_pv_buf = [&](int b) { return bar0 + 8u * (2 * S + 10 + b); };
-    const uint32_t bar_pv_done = bar0 + 8u * (2 * S + 12);
-    const uint32_t bar_o_full = bar0 + 8u * (2 * S + 13);
-    const uint32_t bar_o_empty = bar0 + 8u * (2 * S + 14);
-    auto bar_xch = [&](int pair) { return bar0 + 8u * (2 * S + 15 + pair); };
-    const uint32_t bar_dead = bar0 + 8u * (2 * S + 19);
-    auto bar_drain = [&](int h) { return bar0 + 8u * (2 * S + 20 + h); };
-    auto bar_item_full = [&](int q) { return bar0 + 8u * (2 * S + 22 + q); };
-    auto bar_item_empty = [&](int q) { return bar0 + 8u * (2 * S + 22 + kItemQ + q); };
+    auto bar_p_full = [&](int h, int b) { return bar0 + 8u * (2 * S + 4 + NB + NB * h + b); };
+    auto bar_pv_buf = [&](int b) { return bar0 + 8u * (2 * S + 4 + 3 * NB + b); };
+    const uint32_t bar_o_full = bar0 + 8u * (2 * S + 4 + 4 * NB);
+    const uint32_t bar_o_empty = bar0 + 8u * (2 * S + 5 + 4 * NB);
+    const uint32_t bar_dead = bar0 + 8u * (2 * S + 6 + 4 * NB);
+    auto bar_drain = [&](int h) { return bar0 + 8u * (2 * S + 7 + 4 * NB + h); };
+    auto bar_item_full = [&](int q) { return bar0 + 8u * (2 * S + 9 + 4 * NB + q); };
+    auto bar_item_empty = [&](int q) { return bar0 + 8u * (2 * S + 9 + 4 * NB + kItemQ + q); };
+    static_assert(2 * S + 9 + 4 * NB + 2 * kItemQ == C::kNumBars, "barrier count");
+    float* xch = reinterpret_cast<float*>(smem + C::kXchOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
     volatile int32_t* item_q = reinterpret_cast<volatile int32_t*>(smem + C::kMiscOff + 8);
@@ -278,17 +291,17 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         for (int b = 0; b < 2; ++b) {
             ptx::mbar_init(bar_q_full(b), 1);
-            ptx::mbar_init(bar_q_empty(b), 8);  // every softmax warp, after the epilogue
-            ptx::mbar_init(bar_s_full(b), 1);
-            ptx::mbar_init(bar_p_full(0, b), 4);
-            ptx::mbar_init(bar_p_full(1, b), 4);
-            ptx::mbar_init(bar_pv_buf(b), 1);
+            ptx::mbar_init(bar_q_empty(b), 1);  // the block's last S products completed
             ptx::mbar_init(bar_drain(b), 1);
         }
-        ptx::mbar_init(bar_pv_done, 1);
+        for (int b = 0; b < NB; ++b) {
+            ptx::mbar_init(bar_s_full(b), 1);
+            ptx::mbar_init(bar_p_full(0, b), 4);  // one arrival per softmax warp of the half
+            ptx::mbar_init(bar_p_full(1, b), 4);
+            ptx::mbar_init(bar_pv_buf(b), 1);
+        }
         ptx::mbar_init(bar_o_full, 1);
         ptx::mbar_init(bar_o_empty, 8);
-        for (int i = 0; i < 4; ++i) ptx::mbar_init(bar_xch(i), 2);
         ptx::mbar_init(bar_dead, 1);
         for (int q = 0; q < kItemQ; ++q) {
             ptx::mbar_init(bar_item_full(q), 1);
@@ -317,8 +330,8 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::regs_dec<kRegsProducer>();
         if (lane == 0) {
             // ------------------------------------------------------------ load
-            // Ring entries in the order the issuing thread consumes them: per
-            // block, K(0), K(1), then V(i), K(i + 2) for i = 0, 1, ...
+            // Ring entries in the order the issuing threads consume them: per
+            // block, K(0), K(1), K(2), then V(i), K(i + 3) for i = 0, 1, ...
             uint32_t ring = 0;
             uint32_t q_loads[2] = {0u, 0u};  // query loads issued into each buffer
             bool ok = true;
@@ -351,7 +364,7 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const int32_t* off = p.off + int64_t(w.win) * (p.tiles_per_head + 1);
                 const int32_t* list = p.ids + off[tile_q];
                 const int32_t n = (off[tile_q + 1] - off[tile_q]) * SPT;
-                // query block into buffer k % 2 (free once block k - 2's epilogue is done)
+                // query block into buffer k % 2 (free once block k - 2's S products completed)
                 const int qb = int(k & 1u);
                 if (!wait_bar(bar_q_empty(qb), ((k >> 1) & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
                 ptx::mbar_arrive_expect_tx(bar_q_full(qb), C::kQBytes);
@@ -363,10 +376,10 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     const int32_t kt = __ldg(list + c / SPT);
                     return issue(m, w.bh, kt, tile_org<kRaster>(p, kt), c % SPT);
                 };
-                for (int32_t c = 0; ok && c < n && c < 2; ++c) ok = load_chunk(&tm_k, c);
+                for (int32_t c = 0; ok && c < n && c < NB; ++c) ok = load_chunk(&tm_k, c);
                 for (int32_t i = 0; ok && i < n; ++i) {
                     ok = load_chunk(&tm_v, i);
-                    if (ok && i + 2 < n) ok = load_chunk(&tm_k, i + 2);
+                    if (ok && i + NB < n) ok = load_chunk(&tm_k, i + NB);
                 }
             }
             // Drain before exit (after an abort some copies may still be in
@@ -384,9 +397,9 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::regs_dec<kRegsProducer>();
         if (lane == 0) {
             // ------------------------------------------------------------- MMA
-            // Two issuing threads.  Warp 9 issues O_h += P_h V_h as soon as a
-            // half's P is in TMEM; warp 10 issues S = Q K^T for chunk c + 2 once
-            // both PVs of chunk c (which read the S buffer S(c + 2) overwrites)
+            // Two issuing threads.  Warp 9 issues O += P_h V_h as soon as a
+            // half's P is in TMEM; warp 10 issues S = Q K^T for chunk c + 3 once
+            // both PVs of chunk c (which read the S buffer S(c + 3) overwrites)
             // have completed.  A tcgen05.mma issue holds its thread until the
             // pipe takes it, so with one thread for both kinds the P hand-off
             // waited behind the previous step's S batch.
@@ -396,9 +409,11 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             uint32_t e0 = 0, g = 0;  // ring entries and chunks of the blocks before this one
             bool ok = true;
             // Ring entry of chunk c's K and V in a block of n chunks (the load
-            // order: K(0), K(1), then V(i), K(i + 2) for i = 0, 1, ...).
-            auto entry_k = [](uint32_t c) { return c < 2u ? c : 2u * c - 1u; };
-            auto entry_v = [](uint32_t i, uint32_t n) { return i + 2u <= n ? 2u + 2u * i : 2u * n - 1u; };
+            // order: K(0), K(1), K(2), then V(i), K(i + 3) for i = 0, 1, ...).
+            auto entry_k = [](uint32_t c) { return c < uint32_t(NB) ? c : 2u * c - uint32_t(NB - 1); };
+            auto entry_v = [](uint32_t i, uint32_t n) {
+                return i + uint32_t(NB) <= n ? uint32_t(NB) + 2u * i : n + i;
+            };
             auto wait_entry = [&](uint32_t e, uint32_t& addr) -> bool {
                 const int r = int(e % S);
                 if (!wait_bar(bar_full(r), (e / S) & 1u, abort_flag, p)) return false;
@@ -416,27 +431,29 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 const uint32_t n = uint32_t(off[tile_q + 1] - off[tile_q]) * uint32_t(SPT);
                 const uint32_t g0 = g;
                 if (pv_role) {
+                    const uint32_t tO = tmem + C::kColO;
                     for (uint32_t i = 0; ok && i < n; ++i) {
-                        const uint32_t gi = g0 + i, bb = gi & 1u, e = e0 + entry_v(i, n);
+                        const uint32_t gi = g0 + i, bb = gi % uint32_t(NB), e = e0 + entry_v(i, n);
                         uint32_t vaddr;
                         if (!wait_entry(e, vaddr)) { ok = false; break; }
                         if (i == 0 && !wait_bar(bar_o_empty, (kq & 1u) ^ 1u, abort_flag, p)) { ok = false; break; }
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            // O_h += P_h(gi) V_h(gi): keys 64 h .. 64 h + 63 of the chunk
-                            if (!wait_bar(bar_p_full(h, int(bb)), (gi >> 1) & 1u, abort_flag, p)) { ok = false; break; }
+                            // O += P_h(gi) V_h(gi): keys 64 h .. 64 h + 63 of the chunk
+                            if (!wait_bar(bar_p_full(h, int(bb)), (gi / uint32_t(NB)) & 1u, abort_flag, p)) {
+                                ok = false;
+                                break;
+                            }
                             ptx::tc_fence_after();
                             const uint32_t tP = tmem + C::col_s(int(bb)) + uint32_t(h) * 64u;
-                            const uint32_t tO = tmem + C::col_o(h);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 ptx::mma_ts(tO, tP + kk * 8,
                                             ptx::desc_mn_sw128(vaddr + (h * 4 + kk) * 16 * 128, C::kBoxBytes),
-                                            idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+                                            idesc_pv, (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
                         }
                         if (!ok) break;
-                        ptx::mma_commit(bar_pv_done);       // for the softmax's lazy rescale
-                        ptx::mma_commit(bar_pv_buf(int(bb)));  // S buffer bb is free again
+                        ptx::mma_commit(bar_pv_buf(int(bb)));  // S buffer bb is free again; O holds P(.. gi) V
                         ptx::mma_commit(bar_empty(int(e % S)));
                     }
                     if (!ok) break;
@@ -453,9 +470,10 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     }
                     if (!wait_bar(bar_q_full(qb), (kq >> 1) & 1u, abort_flag, p)) { ok = false; break; }
                     for (uint32_t c = 0; ok && c < n; ++c) {
-                        const uint32_t gc = g0 + c, bb = gc & 1u, e = e0 + entry_k(c);
-                        // S(gc) overwrites buffer bb, read by the PVs of chunk gc - 2
-                        if (gc >= 2u && !wait_bar(bar_pv_buf(int(bb)), ((gc >> 1) - 1u) & 1u, abort_flag, p)) {
+                        const uint32_t gc = g0 + c, bb = gc % uint32_t(NB), e = e0 + entry_k(c);
+                        // S(gc) overwrites buffer bb, read by the PVs of chunk gc - 3
+                        if (gc >= uint32_t(NB) &&
+                            !wait_bar(bar_pv_buf(int(bb)), ((gc / uint32_t(NB)) - 1u) & 1u, abort_flag, p)) {
                             ok = false;
                             break;
                         }
@@ -473,6 +491,7 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         ptx::mma_commit(bar_empty(int(e % S)));
                     }
                     if (!ok) break;
+                    ptx::mma_commit(bar_q_empty(qb));  // the query buffer is free once these S products complete
                 }
                 g = g0 + n;
                 e0 += 2u * n;
@@ -486,19 +505,23 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         ptx::regs_inc<kRegsSoftmax>();
         const int half = warp >> 2;  // 0: keys 0-63 of every chunk, 1: keys 64-127
         const int row = threadIdx.x & 127;
+        const uint32_t pair_bar = 1u + uint32_t(warp & 3);  // named barrier of warps w and w + 4
         const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
-        const uint32_t tO = tmem + lane_addr + C::col_o(half);
+        const uint32_t tOh = tmem + lane_addr + C::kColO + uint32_t(half) * (D / 2);  // this half's O columns
+        float* x_mine = xch + half * kSubRows + row;
+        const float* x_other = xch + (1 - half) * kSubRows + row;
         const float c = p.scale_log2;
         uint32_t g = 0;
         bool ok = true;
         for (uint32_t kq = 0; ok; ++kq) {
             int32_t u = -1;
-            if (!__all_sync(0xffffffffu, take_item(kq, u))) {
+            const bool took = __all_sync(0xffffffffu, take_item(kq, u));
+            __syncwarp();
+            if (took && lane == 0) ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
+            if (ptx::bar_red_or(pair_bar, 64, !took)) {  // leave together
                 ok = false;
                 break;
             }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_item_empty(int(kq % kItemQ)));
             if (u < 0) break;
             const WorkItem w = p.items[u];
             const int32_t tile_q = w.qa / SPT;
@@ -507,128 +530,125 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const int32_t kbeg = off[tile_q];  // this block's key tiles (padded latents: their masks)
             float m_used = 0.0f, l = 0.0f;
             for (uint32_t i = 0; i < n; ++i, ++g) {
-                const uint32_t b = g & 1u;
-                if (!__all_sync(0xffffffffu, wait_bar(bar_s_full(int(b)), (g >> 1) & 1u, abort_flag, p))) {
-                    ok = false;
-                    break;
-                }
-                ptx::tc_fence_after();
+                const uint32_t b = g % uint32_t(NB);
+                const bool wok =
+                    __all_sync(0xffffffffu, wait_bar(bar_s_full(int(b)), (g / uint32_t(NB)) & 1u, abort_flag, p));
                 const uint32_t tS = tmem + lane_addr + C::col_s(int(b)) + uint32_t(half) * 64u;
-                uint32_t sr[64];
-                uint32_t mlo = ~0u, mhi = ~0u;  // real-key bits of this half's 64 keys
-                if (kPadded) {
-                    const uint4 m4 = __ldg(p.key_mask + int64_t(__ldg(p.ids + kbeg + int32_t(i) / SPT)) * SPT +
-                                           int32_t(i) % SPT);
-                    mlo = half == 0 ? m4.x : m4.z;
-                    mhi = half == 0 ? m4.y : m4.w;
-                }
-                ptx::tmem_ld64(tS, sr);
-                if (kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
-                uint32_t pk[32];
-                float rowsum, alpha = 1.0f;
-                bool rescale = false;
-                if (i == 0) {
-                    m_used = row_max64(sr);
-                    // Padded latents: this half of the first chunk may hold no real
-                    // key; any finite reference works, the lazy rescale below
-                    // moves it once real keys arrive.
-                    if (kPadded && m_used == -INFINITY) m_used = 0.0f;
-                    rowsum = softmax_exp64(sr, c, m_used, pk);
-                } else {
-                    rowsum = softmax_exp64(sr, c, m_used, pk);
-                    const bool need = !(rowsum <= kRescaleRowSum);
-                    rescale = __any_sync(0xffffffffu, need);
-                    if (rescale) {
-                        if (need) {
-                            const float mx = row_max64(sr);
-                            if ((mx - m_used) * c > 0.0f) {
-                                alpha = ptx::ex2((m_used - mx) * c);
-                                m_used = mx;
-                            }
-                        }
+                uint32_t sr[64], pk[32];
+                float rowsum = 0.0f;
+                bool need = false;
+                if (wok) {
+                    ptx::tc_fence_after();
+                    uint32_t mlo = ~0u, mhi = ~0u;  // real-key bits of this half's 64 keys
+                    if (kPadded) {
+                        const uint4 m4 = __ldg(p.key_mask + int64_t(__ldg(p.ids + kbeg + int32_t(i) / SPT)) * SPT +
+                                               int32_t(i) % SPT);
+                        mlo = half == 0 ? m4.x : m4.z;
+                        mhi = half == 0 ? m4.y : m4.w;
+                    }
+                    ptx::tmem_ld64(tS, sr);
+                    if (kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
+                    if (i > 0) {
+                        // Exponentiate against the running max (no max pass);
+                        // P goes to TMEM at once and stays unless the pair
+                        // takes the slow path below.
                         rowsum = softmax_exp64(sr, c, m_used, pk);
+                        need = !(rowsum <= kRescaleRowSum);  // also catches inf
+                        ptx::tmem_st32(tS, pk);
                     }
                 }
-                ptx::tmem_st32(tS, pk);
-                l = l * alpha + rowsum;
-                if (rescale) {
-                    // O_h holds P_h(.. gi - 1) V: wait for PV_h(g - 1), the one
-                    // PV of this half that may still be running
-                    if (!__all_sync(0xffffffffu, wait_bar(bar_pv_done, (g - 1u) & 1u, abort_flag, p))) {
+                if (ptx::bar_red_or(pair_bar, 64, !wok || need || i == 0)) {
+                    // ---- slow path: the block's first chunk, a rescale, or an abort.
+                    // Both warps of the pair take it, exchange this chunk's
+                    // maxima of their rows and agree on the new running max.
+                    *x_mine = wok ? row_max64(sr) : -INFINITY;
+                    if (ptx::bar_red_or(pair_bar, 64, !wok)) {
                         ok = false;
                         break;
                     }
-                    ptx::tc_fence_after();
-                    const uint64_t alpha2 = ptx::f2(alpha, alpha);
-#pragma unroll 1
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        uint32_t orr[32];
-                        ptx::tmem_ld32(tO + cb * 32, orr);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            float o0, o1;
-                            ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(orr[2 * j]),
-                                                              __uint_as_float(orr[2 * j + 1])), alpha2),
-                                          o0, o1);
-                            orr[2 * j] = __float_as_uint(o0);
-                            orr[2 * j + 1] = __float_as_uint(o1);
-                        }
-                        ptx::tmem_st32(tO + cb * 32, orr);
+                    const float mx = fmaxf(*x_mine, *x_other);
+                    float alpha = 1.0f;
+                    if (i == 0) {
+                        // padded latents: a first chunk without a real key in this
+                        // row's window takes a finite stand-in, moved later
+                        m_used = mx == -INFINITY ? 0.0f : mx;
+                    } else if ((mx - m_used) * c > 0.0f) {
+                        alpha = ptx::ex2((m_used - mx) * c);
+                        m_used = mx;
                     }
+                    rowsum = softmax_exp64(sr, c, m_used, pk);
+                    ptx::tmem_st32(tS, pk);
+                    l = l * alpha + rowsum;
+                    bool pv_ok = true;
+                    if (i > 0) {
+                        // O holds P(.. g - 1) V: wait for PV(g - 1), the one that
+                        // may still run, then rescale this half's columns of O.
+                        // Its buffer's barrier is at most one phase behind here
+                        // (S(g) waited for PV(g - 3)), so the parity wait is exact.
+                        const uint32_t gp = g - 1u;
+                        pv_ok = __all_sync(0xffffffffu, wait_bar(bar_pv_buf(int(gp % uint32_t(NB))),
+                                                                 (gp / uint32_t(NB)) & 1u, abort_flag, p));
+                        if (pv_ok && __any_sync(0xffffffffu, alpha != 1.0f)) {
+                            ptx::tc_fence_after();
+                            const uint64_t alpha2 = ptx::f2(alpha, alpha);
+#pragma unroll 1
+                            for (int cb = 0; cb < D / 64; ++cb) {
+                                uint32_t orr[32];
+                                ptx::tmem_ld32(tOh + cb * 32, orr);
+#pragma unroll
+                                for (int j = 0; j < 16; ++j) {
+                                    float o0, o1;
+                                    ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(orr[2 * j]),
+                                                                      __uint_as_float(orr[2 * j + 1])), alpha2),
+                                                  o0, o1);
+                                    orr[2 * j] = __float_as_uint(o0);
+                                    orr[2 * j + 1] = __float_as_uint(o1);
+                                }
+                                ptx::tmem_st32(tOh + cb * 32, orr);
+                            }
+                        }
+                    }
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
+                    // both halves' rescales of O are done before either half's P is signalled
+                    if (ptx::bar_red_or(pair_bar, 64, !pv_ok)) {
+                        ok = false;
+                        break;
+                    }
+                } else {
+                    l += rowsum;
+                    ptx::tmem_wait_st();
+                    ptx::tc_fence_before();
                 }
-                ptx::tmem_wait_st();
-                ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar_p_full(half, int(b)));
             }
-            // ---- epilogue: merge the halves, O -> bf16, LSE.  Both warps of a
-            // pair (same rows) always reach the exchange, even when aborting, so
-            // neither waits for the other in vain.
-            const int qb = int(kq & 1u);
-            float* xch = reinterpret_cast<float*>(smem + C::kQOff + qb * C::kQBytes);
-            bool got = ok && __all_sync(0xffffffffu, wait_bar(bar_o_full, kq & 1u, abort_flag, p));
-            if (got) {
-                // the block's query buffer is free: every S of this block has completed
-                xch[(half * 128 + row) * 2 + 0] = m_used;
-                xch[(half * 128 + row) * 2 + 1] = l;
-            }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(bar_xch(warp & 3));
-            got = __all_sync(0xffffffffu, wait_bar(bar_xch(warp & 3), kq & 1u, abort_flag, p)) && got;
-            if (!got) {
+            if (!ok) break;
+            // ---- epilogue: O / (l_A + l_B) -> bf16, LSE.  Each half stores its
+            // half of the columns.
+            const bool ook = __all_sync(0xffffffffu, wait_bar(bar_o_full, kq & 1u, abort_flag, p));
+            *x_mine = l;
+            if (ptx::bar_red_or(pair_bar, 64, !ook)) {
                 ok = false;
                 break;
             }
             ptx::tc_fence_after();
-            const float m_o = xch[((1 - half) * 128 + row) * 2 + 0];
-            const float l_o = xch[((1 - half) * 128 + row) * 2 + 1];
-            const float m_a = half == 0 ? m_used : m_o, l_a = half == 0 ? l : l_o;
-            const float m_b = half == 0 ? m_o : m_used, l_b = half == 0 ? l_o : l;
-            // A half that met no real key (padded latents only) has l = 0 and
-            // O = 0 and takes no part in the merge.
-            const float m = l_a == 0.0f ? m_b : (l_b == 0.0f ? m_a : fmaxf(m_a, m_b));
-            const float a_a = l_a == 0.0f ? 0.0f : ptx::ex2((m_a - m) * c);
-            const float a_b = l_b == 0.0f ? 0.0f : ptx::ex2((m_b - m) * c);
-            const float l_sum = a_a * l_a + a_b * l_b;
+            const float l_sum = l + *x_other;
             const float inv_l = 1.0f / l_sum;
-            const uint64_t f_a = ptx::f2(a_a * inv_l, a_a * inv_l), f_b = ptx::f2(a_b * inv_l, a_b * inv_l);
+            const uint64_t f2inv = ptx::f2(inv_l, inv_l);
             const int64_t grow = out_row<kRaster, kPadded>(p, w.bh, w.qa, row);
-            // this warp's half of the columns: [half * D / 2, half * D / 2 + D / 2)
             uint4* dst = reinterpret_cast<uint4*>(p.o + (grow < 0 ? 0 : grow) * D + half * (D / 2));
-            const uint32_t tOa = tmem + lane_addr + C::col_o(0) + uint32_t(half) * (D / 2);
-            const uint32_t tOb = tmem + lane_addr + C::col_o(1) + uint32_t(half) * (D / 2);
 #pragma unroll 1
             for (int cb = 0; cb < D / 64; ++cb) {
-                uint32_t oa[32], ob[32];
-                ptx::tmem_ld32(tOa + cb * 32, oa);
-                ptx::tmem_ld32(tOb + cb * 32, ob);
+                uint32_t orr[32];
+                ptx::tmem_ld32(tOh + cb * 32, orr);  // every lane loads: the access is warp-wide
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    const uint64_t va = ptx::f2(__uint_as_float(oa[2 * j]), __uint_as_float(oa[2 * j + 1]));
-                    const uint64_t vb = ptx::f2(__uint_as_float(ob[2 * j]), __uint_as_float(ob[2 * j + 1]));
                     float o0, o1;
-                    ptx::f2_split(ptx::f2_fma(va, f_a, ptx::f2_mul(vb, f_b)), o0, o1);
+                    ptx::f2_split(ptx::f2_mul(ptx::f2(__uint_as_float(orr[2 * j]), __uint_as_float(orr[2 * j + 1])),
+                                              f2inv),
+                                  o0, o1);
                     pk[j] = ptx::pack_bf16x2(o0, o1);
                 }
                 if (grow >= 0) {  // a padding row of a raster output stores nothing
@@ -637,14 +657,10 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         dst[cb * 4 + j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                 }
             }
-            if (half == 0 && grow >= 0) p.lse[grow] = m * p.scale + logf(l_sum);
+            if (half == 0 && grow >= 0) p.lse[grow] = m_used * p.scale + logf(l_sum);
             ptx::tc_fence_before();
-            ptx::fence_proxy_async_smem();  // the exchange writes precede the next query load into this buffer
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(bar_o_empty);
-                ptx::mbar_arrive(bar_q_empty(qb));
-            }
+            if (lane == 0) ptx::mbar_arrive(bar_o_empty);
         }
     }
 

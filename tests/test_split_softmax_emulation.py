@@ -1,23 +1,25 @@
 """CPU emulation of the forward kernel's key-split arithmetic against the oracle.
 
 The forward kernel splits every 128-key chunk of a query block's key list
-between two softmax halves (keys 0-63 and 64-127 of the chunk).  Each half
-keeps its own running maximum m, row sum l and output accumulator O in fp32:
-its first chunk sets m (a stand-in 0 when that chunk holds padding keys
-only), later chunks are exponentiated against m, and a chunk whose row sum
-exceeds 256 is redone against its own maximum with O and l rescaled (lazy
-rescale).  P is rounded to bf16 before P V, and the row sum l adds those
-rounded values.  The epilogue merges the halves
-(m = max of the two, each side scaled by 2^((m_h - m) c); a half that met no
-real key has l = 0 and drops out) and writes O / l in bf16 and LSE.
+between two softmax halves (keys 0-63 and 64-127 of the chunk).  The two warps
+that own the same 32 rows keep one running maximum m per row and one fp32
+output accumulator O between them; each half keeps its own row sum.  The
+block's first chunk sets m to the maximum of both halves' scores (a stand-in 0
+when that chunk holds padding keys only); later chunks are exponentiated
+against m, and when any row of the 32-row group has a half-row sum above
+65536 the group raises m to the maximum of m and both halves' chunk maxima,
+rescaling O and both row sums (the slow path).  P is rounded to bf16 before
+P V, and the row sums add those rounded values.  The epilogue writes
+O / (l_A + l_B) in bf16 and LSE = m scale + ln(l_A + l_B).
 
 This file restates those steps in numpy, in the kernel's order and
 precisions, and checks them against the fp64 oracle with the tolerances of
 the GPU parity tests.  It pins the algorithm, not the CUDA code: cases cover a
 divisible latent, a padded one, a latent whose second halves never hold a
-real key (one t-slice), and inputs that force the lazy rescale.  Planting a
-missing rescale, a merge without the 2^((m_h - m) c) factors or unmasked
-padding keys here fails 1, 5 and 2 of its cases.
+real key (one t-slice), and inputs that force the rescale (at the largest
+factor the exponentials would overflow fp32 without it).  Planting a missing
+rescale of O, a row sum of only one half, or unmasked padding keys here fails
+some of its cases.
 """
 import math
 
@@ -30,7 +32,7 @@ import sparse_attention_video_sta_b200 as sta
 from parity_util import LSE_REL_TOL, O_MEAN_TOL, o_bound
 
 LOG2E = 1.4426950408889634
-RESCALE_ROW_SUM = 256.0
+RESCALE_ROW_SUM = 65536.0
 
 
 def bf16(x):
@@ -57,47 +59,43 @@ def emulate_block(qr, k, v, key_tiles, latent, tile, scale):
     Returns O [128, d] (bf16 values) and LSE [128]."""
     c = np.float32(scale * LOG2E)
     d = qr.shape[1]
-    halves = []
-    for h in range(2):
-        m = np.zeros(128, np.float32)
-        l = np.zeros(128, np.float32)
-        o = np.zeros((128, d), np.float32)
-        first = True
-        for kt in key_tiles:
-            toks = tile_major_tokens(latent, tile, kt)
-            for ch in range(len(toks) // 128):
+    m = np.zeros(128, np.float32)
+    lh = [np.zeros(128, np.float32), np.zeros(128, np.float32)]
+    o = np.zeros((128, d), np.float32)
+    first = True
+    for kt in key_tiles:
+        toks = tile_major_tokens(latent, tile, kt)
+        for ch in range(len(toks) // 128):
+            s_h, v_h = [], []
+            for h in range(2):
                 keys = toks[ch * 128 + 64 * h: ch * 128 + 64 * h + 64]
                 real = keys >= 0
                 kk = np.where(real[:, None], k[np.maximum(keys, 0)], 0.0).astype(np.float32)
-                vv = np.where(real[:, None], v[np.maximum(keys, 0)], 0.0).astype(np.float32)
+                v_h.append(np.where(real[:, None], v[np.maximum(keys, 0)], 0.0).astype(np.float32))
                 s = (qr.astype(np.float64) @ kk.astype(np.float64).T).astype(np.float32)
                 s[:, ~real] = -np.inf
-                alpha = np.ones(128, np.float32)
-                if first:
-                    m = s.max(axis=1)
-                    m[m == -np.inf] = 0.0  # stand-in maximum for a half without real keys yet
-                    p = np.exp2(s * c - m[:, None] * c).astype(np.float32)
-                    first = False
-                else:
-                    with np.errstate(over="ignore"):  # inf here is caught by the row-sum test
-                        p = np.exp2(s * c - m[:, None] * c).astype(np.float32)
-                    need = ~(bf16(p).sum(axis=1, dtype=np.float32) <= RESCALE_ROW_SUM)
-                    if need.any():  # warp-uniform in the kernel; per row here, same result
-                        mx = s.max(axis=1)
-                        grow = need & ((mx - m) * c > 0)
-                        alpha = np.exp2(np.where(grow, (m - mx) * c, 0.0)).astype(np.float32)
-                        m = np.where(grow, mx, m).astype(np.float32)
-                        p = np.exp2(s * c - m[:, None] * c).astype(np.float32)
-                rowsum = bf16(p).sum(axis=1, dtype=np.float32)  # the bf16 values P V multiplies
-                o = o * alpha[:, None] + bf16(p) @ bf16(vv)
-                l = l * alpha + rowsum
-        halves.append((m, l, o))
-    (ma, la, oa), (mb, lb, ob) = halves
-    m = np.where(la == 0, mb, np.where(lb == 0, ma, np.maximum(ma, mb)))
-    aa = np.where(la == 0, 0.0, np.exp2((ma - m) * c)).astype(np.float32)
-    ab = np.where(lb == 0, 0.0, np.exp2((mb - m) * c)).astype(np.float32)
-    lsum = aa * la + ab * lb
-    out = (oa * (aa / lsum)[:, None] + ob * (ab / lsum)[:, None]).astype(np.float32)
+                s_h.append(s)
+            mx = np.maximum(s_h[0].max(axis=1), s_h[1].max(axis=1))
+            alpha = np.ones(128, np.float32)
+            if first:
+                m = np.where(mx == -np.inf, 0.0, mx).astype(np.float32)
+            else:
+                with np.errstate(over="ignore"):  # inf here is caught by the row-sum test
+                    sums = [bf16(np.exp2(s * c - m[:, None] * c)).sum(axis=1, dtype=np.float32) for s in s_h]
+                need = ~(sums[0] <= RESCALE_ROW_SUM) | ~(sums[1] <= RESCALE_ROW_SUM)
+                slow = np.repeat(need.reshape(4, 32).any(axis=1), 32)  # per 32-row warp pair
+                grow = slow & ((mx - m) * c > 0)
+                alpha = np.exp2(np.where(grow, (m - mx) * c, 0.0)).astype(np.float32)
+                m = np.where(grow, mx, m).astype(np.float32)
+            o = o * alpha[:, None]
+            for h in range(2):
+                p = bf16(np.exp2(s_h[h] * c - m[:, None] * c).astype(np.float32))
+                lh[h] = lh[h] * alpha + p.sum(axis=1, dtype=np.float32)
+                o = o + p @ bf16(v_h[h])
+            if first:
+                first = False
+    lsum = lh[0] + lh[1]
+    out = (o * (np.float32(1.0) / lsum)[:, None]).astype(np.float32)
     lse = m * np.float32(scale) + np.log(lsum)
     return bf16(out), lse
 
