@@ -529,38 +529,59 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             const uint32_t n = uint32_t(off[tile_q + 1] - off[tile_q]) * uint32_t(SPT);
             const int32_t kbeg = off[tile_q];  // this block's key tiles (padded latents: their masks)
             float m_used = 0.0f, l = 0.0f;
+            // The scores of the next chunk are loaded while this chunk's P is
+            // stored and handed over (`pre`: sr already holds S(g)).
+            uint32_t sr[64];
+            bool pre = false;
             for (uint32_t i = 0; i < n; ++i, ++g) {
-                const uint32_t b = g % uint32_t(NB);
-                const bool wok =
-                    __all_sync(0xffffffffu, wait_bar(bar_s_full(int(b)), (g / uint32_t(NB)) & 1u, abort_flag, p));
+                const uint32_t b = g % uint32_t(NB), b1 = (g + 1u) % uint32_t(NB);
                 const uint32_t tS = tmem + lane_addr + C::col_s(int(b)) + uint32_t(half) * 64u;
-                uint32_t sr[64], pk[32];
+                const uint32_t tS1 = tmem + lane_addr + C::col_s(int(b1)) + uint32_t(half) * 64u;
+                bool wok = true;
+                if (!pre) {
+                    wok = __all_sync(0xffffffffu,
+                                     wait_bar(bar_s_full(int(b)), (g / uint32_t(NB)) & 1u, abort_flag, p));
+                    if (wok) {
+                        ptx::tc_fence_after();
+                        ptx::tmem_ld64(tS, sr);
+                    }
+                }
+                pre = false;
+                uint32_t mlo = ~0u, mhi = ~0u;  // real-key bits of this half's 64 keys
+                if (kPadded) {
+                    const uint4 m4 = __ldg(p.key_mask + int64_t(__ldg(p.ids + kbeg + int32_t(i) / SPT)) * SPT +
+                                           int32_t(i) % SPT);
+                    mlo = half == 0 ? m4.x : m4.z;
+                    mhi = half == 0 ? m4.y : m4.w;
+                }
+                if (wok && kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
+                // Is S(g + 1) of this block complete?  Tested before the
+                // exponentials, so the answer has arrived when it is read.
+                const bool can_pre = wok && i > 0 && i + 1 < n;
+                const bool t_next =
+                    can_pre && ptx::mbar_test_wait(bar_s_full(int(b1)), ((g + 1u) / uint32_t(NB)) & 1u);
+                uint32_t pk[32];
                 float rowsum = 0.0f;
                 bool need = false;
-                if (wok) {
+                if (wok && i > 0) {
+                    // Exponentiate against the running max (no max pass).
+                    rowsum = softmax_exp64(sr, c, m_used, pk);
+                    need = !(rowsum <= kRescaleRowSum);  // also catches inf
+                }
+                const bool nxt = can_pre && __all_sync(0xffffffffu, t_next);
+                if (nxt) {
                     ptx::tc_fence_after();
-                    uint32_t mlo = ~0u, mhi = ~0u;  // real-key bits of this half's 64 keys
-                    if (kPadded) {
-                        const uint4 m4 = __ldg(p.key_mask + int64_t(__ldg(p.ids + kbeg + int32_t(i) / SPT)) * SPT +
-                                               int32_t(i) % SPT);
-                        mlo = half == 0 ? m4.x : m4.z;
-                        mhi = half == 0 ? m4.y : m4.w;
-                    }
-                    ptx::tmem_ld64(tS, sr);
-                    if (kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
-                    if (i > 0) {
-                        // Exponentiate against the running max (no max pass);
-                        // P goes to TMEM at once and stays unless the pair
-                        // takes the slow path below.
-                        rowsum = softmax_exp64(sr, c, m_used, pk);
-                        need = !(rowsum <= kRescaleRowSum);  // also catches inf
-                        ptx::tmem_st32(tS, pk);
-                    }
+                    ptx::tmem_ld64_start(tS1, sr);
                 }
                 if (ptx::bar_red_or(pair_bar, 64, !wok || need || i == 0)) {
                     // ---- slow path: the block's first chunk, a rescale, or an abort.
                     // Both warps of the pair take it, exchange this chunk's
                     // maxima of their rows and agree on the new running max.
+                    if (nxt) {
+                        ptx::tmem_wait_ld(sr);
+                        ptx::tmem_ld64(tS, sr);  // S(g) again: P(g) is not stored yet
+                        if (kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);
+                    }
                     *x_mine = wok ? row_max64(sr) : -INFINITY;
                     if (ptx::bar_red_or(pair_bar, 64, !wok)) {
                         ok = false;
@@ -615,11 +636,15 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                         ok = false;
                         break;
                     }
+                    if (nxt) ptx::tmem_ld64(tS1, sr);  // S(g + 1) again
                 } else {
+                    ptx::tmem_st32(tS, pk);
                     l += rowsum;
                     ptx::tmem_wait_st();
                     ptx::tc_fence_before();
+                    if (nxt) ptx::tmem_wait_ld(sr);
                 }
+                pre = nxt;
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar_p_full(half, int(b)));
             }
