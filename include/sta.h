@@ -67,7 +67,8 @@ typedef enum {
     STA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (e.g. head_dim) */
     STA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
     STA_ERR_TIMEOUT = 4,     /* a device-side wait ran past its time limit */
-    STA_ERR_OOM = 5          /* device or host allocation failed */
+    STA_ERR_OOM = 5,         /* device or host allocation failed */
+    STA_ERR_BOUNDS = 6       /* a plan index failed a device-side check (debug build, libsta_debug.so) */
 } sta_status;
 
 /* Latent and tile extents in tokens, (t, h, w) order. */
@@ -347,8 +348,27 @@ STA_API sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int32_t
 
 /* Synchronise `stream`, then report (and clear) the first asynchronous error
  * of work enqueued with this plan: CUDA for a launch or execution fault,
- * TIMEOUT when a device-side wait gave up. */
+ * BOUNDS when a kernel of the debug build found a plan index out of range
+ * (it then stops without using it), TIMEOUT when a device-side wait gave up. */
 STA_API sta_status sta_last_device_status(sta_plan_t p, void* stream);
+
+/* Check every index of a plan's host copy against the plan's extents: CSR
+ * offsets non-decreasing and inside the id arrays, key and query tile ids
+ * inside the tile grid, work items inside (b, h), row block and window
+ * ranges, each transposed list the transpose of the forward lists, tile
+ * origins inside the padded latent.  sta_plan and sta_plan_host run it on
+ * every plan they build.  Returns INVALID_ARG (text in
+ * sta_last_error_detail) for the first violation, OK otherwise. */
+STA_API sta_status sta_plan_validate(sta_plan_t p);
+
+/* Debug only: overwrite one plan entry, on the host copy and, for a plan on
+ * a device, in its device array (synchronous copy), to test sta_plan_validate
+ * and the device-side checks of the debug build.  which = 0: forward key-tile
+ * id csr_ids[index]; 1: field index % 4 of forward work item index / 4 (bh,
+ * block, unused, window); 2: forward CSR offset csr_off[index]; 3: transposed
+ * query-tile id tcsr_ids[index].  INVALID_ARG for an index outside the array.
+ * A plan changed this way must only run on the debug build. */
+STA_API sta_status sta_debug_plan_poke(sta_plan_t p, int32_t which, int64_t index, int32_t value);
 
 /* Name and text of the last CUDA error met by a libsta call in the calling
  * thread (e.g. "cudaErrorLaunchOutOfResources: ..."), or "no error".  The

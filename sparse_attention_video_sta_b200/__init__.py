@@ -37,7 +37,10 @@ __all__ = [
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG_DIR, "libsta.so")
+# STA_LIBRARY=debug loads libsta_debug.so, the build whose kernels check every
+# plan index before use (status STA_ERR_BOUNDS instead of a fault).
+_LIB_NAME = "libsta_debug.so" if os.environ.get("STA_LIBRARY", "") == "debug" else "libsta.so"
+_LIB_PATH = os.path.join(_PKG_DIR, _LIB_NAME)
 
 STA_OK = 0
 STA_ERR_INVALID_ARG = 1
@@ -45,6 +48,7 @@ STA_ERR_UNSUPPORTED = 2
 STA_ERR_CUDA = 3
 STA_ERR_TIMEOUT = 4
 STA_ERR_OOM = 5
+STA_ERR_BOUNDS = 6
 
 EXPORTED_SYMBOLS = (
     "sta_plan", "sta_plan_host", "sta_plan_destroy", "sta_plan_query", "sta_plan_stats",
@@ -52,7 +56,7 @@ EXPORTED_SYMBOLS = (
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
     "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy", "sta_backward_raster",
-    "sta_plan_backward_items",
+    "sta_plan_backward_items", "sta_plan_validate", "sta_debug_plan_poke",
 )
 
 
@@ -64,8 +68,8 @@ class _Geom(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(_LIB_PATH):
         raise ImportError(
-            f"libsta.so not found at {_LIB_PATH}; build it with "
-            "`python sparse_attention_video_sta_b200/_build.py` (nvcc, sm_100a)")
+            f"{_LIB_NAME} not found at {_LIB_PATH}; build it with "
+            "`python sparse_attention_video_sta_b200/_build.py --debug` (nvcc, sm_100a)")
     L = ctypes.CDLL(_LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     G = ctypes.POINTER(_Geom)
@@ -93,6 +97,8 @@ def _load() -> ctypes.CDLL:
         "sta_pipe_destroy": [vp],
         "sta_last_device_status": [vp, vp],
         "sta_debug_inject_timeout": [i32, i32],
+        "sta_plan_validate": [vp],
+        "sta_debug_plan_poke": [vp, i32, i64, i32],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -257,6 +263,10 @@ class Plan:
         """Attention FLOPs over computed tiles: pairs * 4 * |tile|^2 * d."""
         vol = self.tile[0] * self.tile[1] * self.tile[2]
         return float(self.stats()[0]) * 4.0 * vol * vol * head_dim
+
+    def validate(self) -> None:
+        """Check every index of the plan's host copy (sta_plan_validate)."""
+        _check(_lib.sta_plan_validate(self.handle), "sta_plan_validate")
 
     def destroy(self) -> None:
         if self._h:

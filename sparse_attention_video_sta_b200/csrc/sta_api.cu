@@ -97,6 +97,8 @@ void order_rounds(std::vector<WorkItem>& items, const Len& len, int32_t ctas) {
     items.swap(out);
 }
 
+sta_status validate_plan_host(const PlanHost& P);
+
 // `ctas`: the persistent grid the backward work lists are ordered for (the
 // device's SM count; 148 for host-only plans).
 sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
@@ -263,6 +265,67 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
     };
     order_rounds(P.bq_items, qlen, ctas);
     order_rounds(P.bkv_items, tlen, ctas);
+    return validate_plan_host(P);
+}
+
+// Every index of the host plan against the plan's extents (see
+// sta_plan_validate); on a violation the detail names the array and entry.
+sta_status validate_plan_host(const PlanHost& P) {
+    auto fail = [](const char* what, int64_t i) {
+        snprintf(g_detail, sizeof g_detail, "plan index out of range: %s[%lld]", what, (long long)i);
+        return STA_ERR_INVALID_ARG;
+    };
+    const int32_t T = P.tiles_per_head, S = P.sub_per_tile;
+    const int64_t n_win = int64_t(P.win_ext.size() / 3);
+    const int64_t n_bh = int64_t(P.batch) * P.heads;
+    if (int64_t(P.head_win.size()) != P.heads) return fail("head_win", int64_t(P.head_win.size()));
+    for (int32_t h = 0; h < P.heads; ++h)
+        if (P.head_win[h] < 0 || P.head_win[h] >= n_win) return fail("head_win", h);
+    for (int pass = 0; pass < 2; ++pass) {
+        const std::vector<int32_t>& off = pass == 0 ? P.csr_off : P.tcsr_off;
+        const std::vector<int32_t>& ids = pass == 0 ? P.csr_ids : P.tcsr_ids;
+        const char* on = pass == 0 ? "csr_off" : "tcsr_off";
+        const char* in = pass == 0 ? "csr_ids" : "tcsr_ids";
+        if (int64_t(off.size()) != n_win * (T + 1)) return fail(on, int64_t(off.size()));
+        for (int64_t w = 0; w < n_win; ++w)
+            for (int32_t t = 0; t < T; ++t) {
+                const int64_t i = w * (T + 1) + t;
+                if (off[i] < 0 || off[i] > off[i + 1] || off[i + 1] > int64_t(ids.size())) return fail(on, i);
+            }
+        for (size_t i = 0; i < ids.size(); ++i)
+            if (ids[i] < 0 || ids[i] >= T) return fail(in, int64_t(i));
+    }
+    // The transposed lists hold exactly the forward pairs: as many pairs,
+    // each list strictly ascending, and every (key tile, query tile) pair of
+    // them found (binary search) in the query tile's ascending forward list.
+    for (int64_t w = 0; w < n_win; ++w) {
+        const int32_t* off = &P.csr_off[size_t(w) * (T + 1)];
+        const int32_t* toff = &P.tcsr_off[size_t(w) * (T + 1)];
+        if (toff[T] - toff[0] != off[T] - off[0]) return fail("tcsr_off", w * (T + 1) + T);
+        for (int32_t k = 0; k < T; ++k)
+            for (int32_t j = toff[k]; j < toff[k + 1]; ++j) {
+                const int32_t q = P.tcsr_ids[j];
+                if (j > toff[k] && q <= P.tcsr_ids[j - 1]) return fail("tcsr_ids", j);
+                const int32_t* a = P.csr_ids.data() + off[q];
+                const int32_t* b = P.csr_ids.data() + off[q + 1];
+                if (!std::binary_search(a, b, k)) return fail("tcsr_ids", j);
+            }
+    }
+    const std::vector<WorkItem>* lists[3] = {&P.f1_items, &P.bq_items, &P.bkv_items};
+    const char* names[3] = {"f1_items", "bq_items", "bkv_items"};
+    for (int l = 0; l < 3; ++l)
+        for (size_t i = 0; i < lists[l]->size(); ++i) {
+            const WorkItem& it = (*lists[l])[i];
+            if (it.bh < 0 || it.bh >= n_bh || it.qa < 0 || it.qa >= T * S || it.win < 0 || it.win >= n_win ||
+                it.win != P.head_win[it.bh % P.heads])
+                return fail(names[l], int64_t(i));
+        }
+    const int32_t Lp[3] = {P.n_tiles[0] * P.g.tile_t, P.n_tiles[1] * P.g.tile_h, P.n_tiles[2] * P.g.tile_w};
+    for (int32_t t = 0; t < T; ++t) {
+        const int32_t* o = &P.tile_origin[size_t(t) * 4];
+        if (o[0] < 0 || o[0] >= Lp[2] || o[1] < 0 || o[1] >= Lp[1] || o[2] < 0 || o[2] >= Lp[0])
+            return fail("tile_origin", t);
+    }
     return STA_OK;
 }
 
@@ -402,6 +465,7 @@ const char* sta_status_string(sta_status s) {
         case STA_ERR_CUDA: return "STA_ERR_CUDA";
         case STA_ERR_TIMEOUT: return "STA_ERR_TIMEOUT";
         case STA_ERR_OOM: return "STA_ERR_OOM";
+        case STA_ERR_BOUNDS: return "STA_ERR_BOUNDS";
     }
     return "STA_ERR_UNKNOWN";
 }
@@ -589,11 +653,42 @@ sta_status sta_last_device_status(sta_plan_t p, void* stream) {
     if (word != 0) {
         if (cudaError_t e = cudaMemset(p->d_status, 0, sizeof word); e != cudaSuccess) return cuda_status(e);
     }
+    if (word & sta::kDevBounds) return STA_ERR_BOUNDS;
     if (word & sta::kDevTimeout) return STA_ERR_TIMEOUT;
     return STA_OK;
 }
 
 const char* sta_last_error_detail(void) { return g_detail; }
+
+sta_status sta_plan_validate(sta_plan_t p) {
+    if (p == nullptr) return STA_ERR_INVALID_ARG;
+    return validate_plan_host(p->h);
+}
+
+sta_status sta_debug_plan_poke(sta_plan_t p, int32_t which, int64_t index, int32_t value) {
+    if (p == nullptr || index < 0) return STA_ERR_INVALID_ARG;
+    PlanHost& P = p->h;
+    int32_t* host = nullptr;
+    void* dev = nullptr;
+    int64_t n = 0;
+    switch (which) {
+        case 0: n = int64_t(P.csr_ids.size()); host = P.csr_ids.data(); dev = p->d_ids; break;
+        case 1: n = int64_t(P.f1_items.size()) * 4; host = reinterpret_cast<int32_t*>(P.f1_items.data());
+                dev = p->d_f1_items; break;
+        case 2: n = int64_t(P.csr_off.size()); host = P.csr_off.data(); dev = p->d_off; break;
+        case 3: n = int64_t(P.tcsr_ids.size()); host = P.tcsr_ids.data(); dev = p->d_tids; break;
+        default: return STA_ERR_INVALID_ARG;
+    }
+    if (index >= n) return STA_ERR_INVALID_ARG;
+    host[index] = value;
+    if (p->on_device && dev != nullptr) {
+        if (cudaError_t e = cudaMemcpy(static_cast<int32_t*>(dev) + index, &value, sizeof value,
+                                       cudaMemcpyHostToDevice);
+            e != cudaSuccess)
+            return cuda_status(e);
+    }
+    return STA_OK;
+}
 
 sta_status sta_debug_inject_timeout(int32_t mode, int32_t limit_ms) {
     if (limit_ms < 1 || limit_ms > 10000 || mode < 0 || mode > 2) return STA_ERR_INVALID_ARG;

@@ -43,6 +43,7 @@
 
 #include <mutex>
 
+#include "sta_bounds.cuh"
 #include "sta_internal.h"
 #include "sta_ptx.cuh"
 #include "sta_raster.cuh"
@@ -88,6 +89,7 @@ struct BwdParams {
     uint64_t timeout_ns;
     RasterGeom rg;          // raster layout only
     int32_t* item_counter;  // next item to hand out (zeroed before the launch); null: fixed stride
+    PlanBounds pb;          // extents of the plan arrays (checked by the debug build)
 };
 
 __device__ __forceinline__ bool wait_bw(uint32_t bar, uint32_t parity, volatile int* abort_flag, const BwdParams& p) {
@@ -108,6 +110,10 @@ __device__ __forceinline__ int32_t put_item(uint32_t k, uint32_t full0, uint32_t
                                             volatile int* abort_flag, const BwdParams& p) {
     int32_t u = p.item_counter != nullptr ? atomicAdd(p.item_counter, 1) : int32_t(blockIdx.x + k * gridDim.x);
     if (u >= p.n_items) u = -1;
+    if (kDebugBounds && u >= 0 && !item_in_bounds(p.items, p.n_items, u, p.off, p.ids, p.pb, p.status)) {
+        *abort_flag = 1;  // no more items: every role leaves its loop
+        u = -1;
+    }
     const uint32_t e = k % kItemQ;
     if (k >= uint32_t(kItemQ) && !wait_bw(empty0 + 8u * e, ((k / kItemQ) - 1) & 1u, abort_flag, p)) return -2;
     q[e] = u;
@@ -982,6 +988,9 @@ cudaError_t launch_bwd_d(const sta_plan_s* pl, const void* q, const void* k, con
     bp.status = pl->d_status;
     bp.timeout_ns = timeout_ns;
     bp.rg = raster_geom(pl);
+    // the forward lists and their transpose have the same extents
+    bp.pb = PlanBounds{int32_t(int64_t(P.batch) * P.heads), P.tiles_per_head, P.sub_per_tile, P.tile_tokens,
+                       int32_t(P.win_ext.size() / 3), int32_t(P.csr_ids.size())};
     if (raster)
         return P.padded ? launch_bwd_variant<D, true, true>(pl, mq, mk, mv, mdo, bp, o, dout, lse, dq, dk, dv, ws, rows,
                                                             sms, stream)

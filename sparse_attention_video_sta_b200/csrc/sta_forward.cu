@@ -24,6 +24,7 @@
 
 #include <mutex>
 
+#include "sta_bounds.cuh"
 #include "sta_internal.h"
 #include "sta_ptx.cuh"
 #include "sta_raster.cuh"
@@ -76,6 +77,7 @@ struct FwdParams {
     // Padded latents (an axis not a multiple of the tile): real-key bits of
     // every 128-key chunk, [tiles][sub_per_tile] x 4 words; null otherwise.
     const uint4* key_mask;
+    PlanBounds pb;  // extents of the plan arrays (checked by the debug build)
 };
 
 // Load 128-row block `sub` of tile `tile` of head bh.  Tile-major layout: one
@@ -350,6 +352,10 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 int32_t u = p.item_counter != nullptr ? atomicAdd(p.item_counter, 1)
                                                       : int32_t(blockIdx.x + k * gridDim.x);
                 if (u >= p.n_items) u = -1;
+                if (kDebugBounds && u >= 0 && !item_in_bounds(p.items, p.n_items, u, p.off, p.ids, p.pb, p.status)) {
+                    *abort_flag = 1;  // no more items: every role leaves its loop
+                    u = -1;
+                }
                 const int qe = int(k % kItemQ);
                 if (k >= uint32_t(kItemQ) &&
                     !wait_bar(bar_item_empty(qe), ((k / kItemQ) - 1) & 1u, abort_flag, p)) {
@@ -786,6 +792,8 @@ cudaError_t launch_d(const sta_plan_s* pl, const void* q, const void* k, const v
     fp.inject = inject;
     fp.rg = raster_geom(pl);
     fp.key_mask = reinterpret_cast<const uint4*>(pl->d_kmask);
+    fp.pb = PlanBounds{int32_t(bh), P.tiles_per_head, P.sub_per_tile, P.tile_tokens,
+                       int32_t(P.win_ext.size() / 3), int32_t(P.csr_ids.size())};
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -855,6 +863,7 @@ cudaError_t launch_forward_raw(const RawPlanView& pv, const void* q, const void*
     fp.status = pv.status;
     fp.timeout_ns = pv.timeout_ns;
     fp.inject = 0;
+    fp.pb = PlanBounds{pv.batch * pv.heads, pv.tiles_per_head, pv.sub_per_tile, pv.tile_tokens, pv.n_win, pv.n_ids};
     int dev = 0, sms = 0;
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

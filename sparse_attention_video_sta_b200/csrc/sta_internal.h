@@ -20,6 +20,17 @@ constexpr int kChunkKeys = 128;
 
 // Device status bits written by kernels (OR-ed).
 constexpr uint32_t kDevTimeout = 1u;
+constexpr uint32_t kDevBounds = 2u;  // a plan index failed its check (debug build)
+
+// Extents a plan's device arrays must respect (checked by the debug build).
+struct PlanBounds {
+    int32_t n_bh;          // batch * heads
+    int32_t tiles;         // tiles per head
+    int32_t sub_per_tile;  // 128-row blocks per tile
+    int32_t tile_tokens;
+    int32_t n_win;         // distinct windows
+    int32_t n_ids;         // entries of the CSR id array walked
+};
 
 // One work item of the forward and backward kernels: one 128-row block of
 // one (b, h) (a query block, or a key block for the dK / dV kernel).
@@ -110,6 +121,7 @@ struct RawPlanView {
     const int32_t* ids;
     uint32_t* status;
     uint64_t timeout_ns;
+    int32_t n_win, n_ids;  // CSR extents (checked by the debug build)
 };
 
 // Forward launch from a RawPlanView (sta_forward.cu).  Returns a CUDA error code.

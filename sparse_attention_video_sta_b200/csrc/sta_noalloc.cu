@@ -277,6 +277,8 @@ extern "C" sta_status sta_forward_noalloc(const sta_geom* g, int32_t batch, int3
     pv.ids = reinterpret_cast<const int32_t*>(dev + ids_at);
     pv.status = reinterpret_cast<uint32_t*>(dev);
     pv.timeout_ns = kTimeoutNs;
+    pv.n_win = n_win;
+    pv.n_ids = int32_t(n_ids);
     const cudaError_t e = sta::launch_forward_raw(pv, q, k, v, o, lse, head_dim, softmax_scale, s);
     return e == cudaSuccess ? STA_OK : STA_ERR_CUDA;
 }
