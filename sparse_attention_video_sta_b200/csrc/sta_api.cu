@@ -218,13 +218,35 @@ sta_status build_plan_host(const sta_geom* g, int32_t batch, int32_t heads,
     for (int32_t b = 0; b < batch; ++b)
         for (int32_t h = 0; h < heads; ++h) P.computed_pairs += int64_t(P.tiles_per_head) * list_len[P.head_win[h]];
     // Forward work items (the key-split kernel): every real row block once,
-    // in (head, block) order, longest lists first (stable: neighbouring tiles
-    // stay together for L2 reuse).
+    // head by head, longest lists first (stable sort).
+    // Inside a head the query tiles follow a Morton (Z) order of their tile
+    // coordinates, so the ~one SM count of blocks in flight at once covers a
+    // compact 3D neighbourhood whose key windows overlap most (fewer distinct
+    // K / V tiles live in L2 at a time than with raster order).
+    std::vector<int32_t> zorder(size_t(P.tiles_per_head));
+    {
+        std::vector<std::pair<uint64_t, int32_t>> code(zorder.size());
+        for (int32_t qt = 0; qt < nt; ++qt)
+            for (int32_t qh = 0; qh < nh; ++qh)
+                for (int32_t qw = 0; qw < nw; ++qw) {
+                    uint64_t c = 0;
+                    for (int bit = 0; bit < 21; ++bit)
+                        c |= (uint64_t((qw >> bit) & 1) << (3 * bit)) | (uint64_t((qh >> bit) & 1) << (3 * bit + 1)) |
+                             (uint64_t((qt >> bit) & 1) << (3 * bit + 2));
+                    const int32_t q = (qt * nh + qh) * nw + qw;
+                    code[size_t(q)] = {c, q};
+                }
+        std::sort(code.begin(), code.end());
+        for (size_t i = 0; i < code.size(); ++i) zorder[i] = code[i].second;
+    }
     P.f1_items.clear();
     for (int32_t b = 0; b < batch; ++b)
         for (int32_t h = 0; h < heads; ++h)
-            for (int32_t blk = 0; blk < P.tiles_per_head * S; ++blk)
-                if (real_block[size_t(blk)]) P.f1_items.push_back(WorkItem{b * heads + h, blk, -1, P.head_win[h]});
+            for (int32_t r = 0; r < P.tiles_per_head; ++r)
+                for (int32_t sub = 0; sub < S; ++sub) {
+                    const int32_t blk = zorder[size_t(r)] * S + sub;
+                    if (real_block[size_t(blk)]) P.f1_items.push_back(WorkItem{b * heads + h, blk, -1, P.head_win[h]});
+                }
     std::stable_sort(P.f1_items.begin(), P.f1_items.end(), [&](const WorkItem& a, const WorkItem& b) {
         return list_len[a.win] > list_len[b.win];
     });
