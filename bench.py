@@ -44,7 +44,8 @@ FWD_SOURCES = ["sparse_attention_video_sta_b200/csrc/sta_forward.cu",
                "sparse_attention_video_sta_b200/csrc/sta_ptx.cuh",
                "sparse_attention_video_sta_b200/csrc/sta_internal.h",
                "sparse_attention_video_sta_b200/csrc/sta_raster.cuh",
-               "sparse_attention_video_sta_b200/csrc/sta_wait.cuh"]
+               "sparse_attention_video_sta_b200/csrc/sta_wait.cuh",
+               "sparse_attention_video_sta_b200/csrc/sta_bounds.cuh"]
 COUNTERS_FILE = os.path.join(ROOT, "profiles", "sta_fwd_counters.json")
 
 
