@@ -273,6 +273,30 @@ STA_API sta_status sta_window_stats(const float* lse_w, const float* lse_full, c
                                     const void* o_full, int64_t slices, int64_t tokens, int32_t head_dim,
                                     double* recall, double* mse, void* stream);
 
+/* Pick a window per head from profiled candidates (host only, no CUDA call).
+ * The pages profile a predefined list of windows per head and keep, per head,
+ * one that preserves quality ("Fast Video Generation with Sliding Tile
+ * Attention": podcast transcript at hotaipapers.com, segment on head
+ * specialisation; dianyo.github.io ICML-2025 post, STA section); they give no
+ * selection rule.  This library's reading: each head takes the candidate with
+ * the fewest attended tiles (ties: the one listed first) whose recall and
+ * output error meet every given bound; the window covering the volume when
+ * none does.
+ *   g         : geometry (tile counts per candidate: prod_d min(W_d / T_d, n_d))
+ *   heads     : H >= 1;  n_cand >= 0 candidates
+ *   cand_thw  : host int32 [n_cand][3], windows in tokens (positive multiples
+ *               of the tile, as for sta_plan)
+ *   recall    : host fp64 [n_cand][heads], e.g. sta_window_stats' recall
+ *               averaged over the batch
+ *   mse       : host fp64 [n_cand][heads], the same for the output error
+ *   max_mse   : upper bound on mse, or a negative value for none
+ *   min_recall: lower bound on recall, or a negative value for none
+ *   out_thw   : host int32 [heads][3] (written), window per head in tokens
+ * INVALID_ARG on a bad geometry, count, candidate or null pointer. */
+STA_API sta_status sta_window_pick(const sta_geom* g, int32_t heads, int32_t n_cand, const int32_t* cand_thw,
+                                   const double* recall, const double* mse, double max_mse, double min_recall,
+                                   int32_t* out_thw);
+
 /* Forward pipeline from host memory (no counterpart on the pages: a runtime
  * piece for callers whose Q, K, V live in host memory).  At the pages' 720p
  * size the PCIe copies of one call take longer than its attention, so the

@@ -33,7 +33,7 @@ __all__ = [
     "sta_forward", "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status",
     "sta_status_string", "sta_debug_inject_timeout", "sta_attention", "raster_supported", "library_path", "EXPORTED_SYMBOLS",
     "sta_backward", "sta_attention_backward", "StaAttention", "sta_window_stats", "sta_window_search",
-    "Pipe", "sta_pipe_create", "sta_backward_raster",
+    "Pipe", "sta_pipe_create", "sta_backward_raster", "sta_window_pick",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -56,7 +56,7 @@ EXPORTED_SYMBOLS = (
     "sta_forward_raster", "sta_forward_noalloc", "sta_last_device_status", "sta_status_string", "sta_debug_inject_timeout",
     "sta_last_error_detail", "sta_plan_key_query", "sta_backward", "sta_window_stats",
     "sta_pipe_create", "sta_pipe_submit", "sta_pipe_wait", "sta_pipe_destroy", "sta_backward_raster",
-    "sta_plan_backward_items", "sta_plan_validate", "sta_debug_plan_poke",
+    "sta_plan_backward_items", "sta_plan_validate", "sta_debug_plan_poke", "sta_window_pick",
 )
 
 
@@ -99,6 +99,7 @@ def _load() -> ctypes.CDLL:
         "sta_debug_inject_timeout": [i32, i32],
         "sta_plan_validate": [vp],
         "sta_debug_plan_poke": [vp, i32, i64, i32],
+        "sta_window_pick": [G, i32, i32, i32p, vp, vp, ctypes.c_double, ctypes.c_double, i32p],
     }
     for name, args in sig.items():
         f = getattr(L, name)
@@ -637,19 +638,31 @@ def sta_window_search(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, latent,
         tiles.append(math.prod(min(c[i] // int(tile[i]), n[i]) for i in range(3)))
         plan.destroy()
     full.destroy()
-    recall = torch.stack(rec).cpu().numpy() if rec else None
-    mse = torch.stack(err).cpu().numpy() if err else None
-    order = sorted(range(len(cands)), key=lambda i: tiles[i])
-    chosen = []
-    for h in range(H):
-        pick = lat
-        for i in order:
-            if (max_mse is None or mse[i, h] <= max_mse) and (min_recall is None or recall[i, h] >= min_recall):
-                pick = cands[i]
-                break
-        chosen.append(list(pick))
-    return {"windows": chosen, "recall": recall, "mse": mse, "candidates": [list(c) for c in cands],
-            "tiles": tiles}
+    recall = torch.stack(rec).cpu().double().contiguous() if rec else None
+    mse = torch.stack(err).cpu().double().contiguous() if err else None
+    chosen = sta_window_pick(lat, tile, H, cands, recall, mse, max_mse, min_recall)
+    return {"windows": chosen, "recall": recall.numpy() if rec else None, "mse": mse.numpy() if err else None,
+            "candidates": [list(c) for c in cands], "tiles": tiles}
+
+
+def sta_window_pick(latent, tile, heads: int, candidates, recall, mse, max_mse: float | None = None,
+                    min_recall: float | None = None) -> list:
+    """Per head, the candidate window with the fewest attended tiles meeting
+    the bounds (the C call ``sta_window_pick``); recall and mse are
+    ``[len(candidates), heads]`` host arrays.  Returns ``[heads][3]``."""
+    cands = [tuple(int(x) for x in c) for c in candidates]
+    C, H = len(cands), int(heads)
+    flat = (ctypes.c_int32 * max(3 * C, 3))(*[x for c in cands for x in c])
+    r = torch.as_tensor(recall if C else [0.0], dtype=torch.float64).contiguous()
+    m = torch.as_tensor(mse if C else [0.0], dtype=torch.float64).contiguous()
+    if C and (tuple(r.shape) != (C, H) or tuple(m.shape) != (C, H)):
+        raise ValueError(f"recall and mse must be [{C}, {H}]")
+    out = (ctypes.c_int32 * (3 * H))()
+    geom = _geom(latent, tile)
+    _check(_lib.sta_window_pick(ctypes.byref(geom), H, C, flat, ctypes.c_void_p(r.data_ptr()),
+                                ctypes.c_void_p(m.data_ptr()), -1.0 if max_mse is None else float(max_mse),
+                                -1.0 if min_recall is None else float(min_recall), out), "sta_window_pick")
+    return [list(out[3 * h:3 * h + 3]) for h in range(H)]
 
 
 class Pipe:

@@ -682,6 +682,38 @@ sta_status sta_last_device_status(sta_plan_t p, void* stream) {
 
 const char* sta_last_error_detail(void) { return g_detail; }
 
+sta_status sta_window_pick(const sta_geom* g, int32_t heads, int32_t n_cand, const int32_t* cand_thw,
+                           const double* recall, const double* mse, double max_mse, double min_recall,
+                           int32_t* out_thw) {
+    if (!geom_valid(g) || heads < 1 || n_cand < 0 || out_thw == nullptr) return STA_ERR_INVALID_ARG;
+    if (n_cand > 0 && (cand_thw == nullptr || recall == nullptr || mse == nullptr)) return STA_ERR_INVALID_ARG;
+    const int32_t L[3] = {g->lat_t, g->lat_h, g->lat_w}, T[3] = {g->tile_t, g->tile_h, g->tile_w};
+    int32_t n[3];
+    for (int d = 0; d < 3; ++d) n[d] = (L[d] + T[d] - 1) / T[d];
+    std::vector<int64_t> tiles(size_t(n_cand), 1);
+    for (int32_t c = 0; c < n_cand; ++c)
+        for (int d = 0; d < 3; ++d) {
+            const int32_t w = cand_thw[3 * c + d];
+            if (w <= 0 || w % T[d] != 0) return STA_ERR_INVALID_ARG;
+            tiles[size_t(c)] *= std::min(w / T[d], n[d]);
+        }
+    std::vector<int32_t> order(static_cast<size_t>(n_cand));
+    for (int32_t c = 0; c < n_cand; ++c) order[size_t(c)] = c;
+    std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) { return tiles[a] < tiles[b]; });
+    for (int32_t h = 0; h < heads; ++h) {
+        const int32_t* pick = L;  // the window covering the volume
+        for (int32_t c : order) {
+            const double r = recall[size_t(c) * heads + h], e = mse[size_t(c) * heads + h];
+            if ((max_mse < 0.0 || e <= max_mse) && (min_recall < 0.0 || r >= min_recall)) {
+                pick = cand_thw + 3 * c;
+                break;
+            }
+        }
+        for (int d = 0; d < 3; ++d) out_thw[3 * h + d] = pick[d];
+    }
+    return STA_OK;
+}
+
 sta_status sta_plan_validate(sta_plan_t p) {
     if (p == nullptr) return STA_ERR_INVALID_ARG;
     return validate_plan_host(p->h);
