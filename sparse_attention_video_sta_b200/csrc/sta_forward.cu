@@ -561,8 +561,8 @@ sta_fwd_split_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                     mhi = half == 0 ? m4.y : m4.w;
                 }
                 if (wok && kPadded && (mlo & mhi) != ~0u) mask_scores64(sr, mlo, mhi);  // warp-uniform
-                // Is S(g + 1) of this block complete?  Tested before the
-                // exponentials, so the answer has arrived when it is read.
+                // Is S(g + 1) of this block complete?  If so, its load starts
+                // right after the exponentials and overlaps the P hand-over.
                 const bool can_pre = wok && i > 0 && i + 1 < n;
                 const bool t_next =
                     can_pre && ptx::mbar_test_wait(bar_s_full(int(b1)), ((g + 1u) / uint32_t(NB)) & 1u);
