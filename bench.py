@@ -27,6 +27,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -103,22 +104,57 @@ def measured_counters(workload_name: str):
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    """SM clock, its maximum, board power and clock-event reasons sampled
+    every 10 ms by a background thread through NVML (reads only), so that the
+    record covers the timed region itself: the samples taken between begin()
+    and end().  Without NVML, nvidia-smi at 100 ms over the whole window."""
 
+    REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                   0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device: int):
+        self.samples = []
+        self.t_begin = self.t_end = None
+        self.thread = None
         self.proc = None
-        self.file = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.done = False
+        self.nvml = self.handle = None
         try:
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
-            self.sel = ["-i", uuid]
         except Exception:
-            self.sel = []
+            uuid = None
+        self.sel = ["-i", uuid] if uuid else []
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid
+                           else pynvml.nvmlDeviceGetHandleByIndex(device))
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = self.handle = None
+
+    def _loop(self):
+        n, h = self.nvml, self.handle
+        while not self.done:
+            try:
+                self.samples.append((time.perf_counter(), float(n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)),
+                                     float(n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)),
+                                     n.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     int(n.nvmlDeviceGetCurrentClocksEventReasons(h))))
+            except Exception:
+                pass
+            time.sleep(0.01)
 
     def start(self):
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._loop, daemon=True)
+            self.thread.start()
+            time.sleep(0.05)
+            return
+        self.file = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", *self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -127,7 +163,28 @@ class ClockSampler:
             self.proc = None
         time.sleep(0.3)
 
+    def begin(self):
+        self.t_begin = time.perf_counter()
+
+    def end(self):
+        self.t_end = time.perf_counter()
+
     def stop(self):
+        if self.thread is not None:
+            self.done = True
+            self.thread.join(timeout=5)
+            inside = [x for x in self.samples
+                      if self.t_begin is not None and self.t_end is not None and self.t_begin <= x[0] <= self.t_end]
+            use = inside if len(inside) >= 3 else self.samples
+            if not use:
+                return None
+            reasons = sorted({name for x in use for bit, name in self.REASON_BITS.items() if x[4] & bit})
+            rec = {"sm_mhz": statistics.median(x[1] for x in use), "sm_mhz_min": min(x[1] for x in use),
+                   "sm_max_mhz": max(x[2] for x in use), "power_w": round(statistics.median(x[3] for x in use), 1),
+                   "samples": len(use), "window": "timed region" if use is inside else "whole sampling window",
+                   "source": "nvml, 10 ms", "reasons": reasons}
+            rec["rejected"] = clocks_rejected(rec)
+            return rec
         if self.proc is None:
             return None
         time.sleep(0.15)
@@ -156,12 +213,12 @@ class ClockSampler:
             return None
         busy = [s for s in sm if s > 0.5 * max(sm)] or sm
         rec = {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx), "samples": len(sm),
-               "reasons": sorted(reasons)}
+               "window": "whole sampling window", "source": "nvidia-smi, 100 ms", "reasons": sorted(reasons)}
         rec["rejected"] = clocks_rejected(rec)
         return rec
 
 
-REJECTED_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+REJECTED_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "hw_power_brake_slowdown"}
 
 
 def clocks_rejected(clocks) -> bool:
@@ -346,12 +403,15 @@ def time_calls(fn, reps: int, warmup: int, dev, sample_clocks: bool):
     sampler = ClockSampler(dev.index) if sample_clocks else None
     if sampler:
         sampler.start()
+        sampler.begin()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(reps):
         fn()
     e1.record()
     torch.cuda.synchronize()
+    if sampler:
+        sampler.end()
     clocks = sampler.stop() if sampler else None
     return e0.elapsed_time(e1) / reps, clocks
 
@@ -512,12 +572,16 @@ def main():
             sampler.start()
         barrier()
         torch.cuda.synchronize()
+        if sampler:
+            sampler.begin()
         start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         start.record()
         for _ in range(args.steps):
             step(record=True)
         stop.record()
         torch.cuda.synchronize()
+        if sampler:
+            sampler.end()
         barrier()
         clocks = sampler.stop() if sampler else None
         return (start.elapsed_time(stop) / args.steps, statistics.mean(a.elapsed_time(b) for a, b in ev_fwd),

@@ -76,3 +76,37 @@ def test_clock_records_that_are_measured_again():
                                       "reasons": ["sw_power_cap", bad]})
     # clocks far below their maximum with no reason: a clock lock left behind
     assert bench.clocks_rejected({"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "samples": 5, "reasons": []})
+
+
+def test_clock_record_covers_only_the_timed_region(monkeypatch):
+    """The NVML sampler keeps only the samples taken between begin() and end()
+    (a fake NVML stands in for the driver: idle clocks outside the region,
+    power-capped clocks inside it)."""
+    import time
+    import types
+    import bench
+    inside = {"on": False}
+    fake = types.ModuleType("pynvml")
+    fake.NVML_CLOCK_SM = 1
+    fake.nvmlInit = lambda: None
+    fake.nvmlDeviceGetHandleByUUID = lambda u: "gpu"
+    fake.nvmlDeviceGetHandleByIndex = lambda i: "gpu"
+    fake.nvmlDeviceGetClockInfo = lambda h, c: 1575 if inside["on"] else 1965
+    fake.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    fake.nvmlDeviceGetPowerUsage = lambda h: 990000 if inside["on"] else 150000
+    fake.nvmlDeviceGetCurrentClocksEventReasons = lambda h: 0x4 if inside["on"] else 0x1
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setattr(torch.cuda, "get_device_properties", lambda d: types.SimpleNamespace(uuid="fake"))
+    s = bench.ClockSampler(0)
+    s.start()
+    time.sleep(0.1)  # idle samples before the region
+    inside["on"] = True
+    s.begin()
+    time.sleep(0.2)
+    s.end()
+    inside["on"] = False
+    time.sleep(0.1)  # idle samples after it
+    rec = s.stop()
+    assert rec["window"] == "timed region" and rec["samples"] >= 3
+    assert rec["sm_mhz"] == 1575.0 and rec["sm_max_mhz"] == 1965.0 and rec["power_w"] == 990.0
+    assert rec["reasons"] == ["sw_power_cap"] and not rec["rejected"]
