@@ -354,8 +354,8 @@ STA_API sta_status sta_pipe_destroy(sta_pipe_t pipe);
  * before any work.  batch 0 returns STA_OK at once (pointers unread).
  *
  * Behaviour: the first call on a device looks up the scratch's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any stream
- * capture.  Each call enqueues two kernels on `stream`: one writes the plan
+ * (cudaGetSymbolAddress) and caches it.  Each call enqueues two kernels on
+ * `stream`: one writes the plan
  * into the scratch (from the windows, which it receives as kernel arguments;
  * nothing is copied from host memory) and clears the status word and work
  * counter kept there, the second is the forward.  Every call shares the one
