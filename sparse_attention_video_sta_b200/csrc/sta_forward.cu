@@ -9,7 +9,7 @@
 // manage the sparse tile list, and compute warpgroups doing dense attention math
 // (same transcript, segment on ThunderKittens); the kernel below keeps that
 // split but is built for Blackwell: one 128-row query block per work item,
-// every 128-key chunk split between two softmax warpgroups, S double buffered
+// every 128-key chunk split between two softmax warpgroups, S triple buffered
 // in TMEM (see the kernel's own comment).
 //
 // The kernel is persistent (one CTA per SM) over the plan's work list, longest
